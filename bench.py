@@ -1,0 +1,462 @@
+#!/usr/bin/env python3
+"""Benchmark of the Nystromformer attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl native|reference]
+
+One step = one whole forward (landmarks, kernel_2 + iterative inverse,
+kernel_3 V, W = Z k3V, output with the depthwise conv) over one batch of
+the workload, through the C ABI (nys_attn_forward). Default workload: the
+n=16384 bf16 correlated-token shape (B=4, H=8, d=64, m=256, conv on).
+
+Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
+(a 256 MiB device write, outside the timed interval) and bracketed by CUDA
+events on the launching stream; a barrier and a device synchronisation on
+both sides; the maximum over ranks is reported. Per-kernel device times come
+from CUDA events the library records around each launch during the same
+timed steps. SM clocks and throttle reasons are sampled with nvidia-smi
+during the timed steps.
+
+Multi-GPU: the forward has no exchange step; each rank runs an independent
+replica on its own seeded batch ("replicas only", weak scaling).
+
+--impl reference times the fp64 CPU oracle on this machine's host cores instead
+(rank 0 only), on a bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import HEADLINE, WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "Nystrom attention tokens/s (B*H*n/s) at n=16384 bf16"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+N_SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "nystr_self_attention_scale_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+# ---------------------------------------------------------------- algorithmic work per launch
+
+def kernel_work(w, kernel):
+    """(algorithmic bytes, algorithmic flops, compute unit) of one launch of `kernel`.
+
+    Bytes count each input element read once and each output written once;
+    flops count 2 per multiply-add of the dense contractions (softmax
+    exponentials are not counted)."""
+    elt = 4 if w.dtype == "f32" else 2
+    BH, n, d, m = w.BH, w.n, w.d, w.m
+    tensor = BH * n * d * elt
+    unit = "alu" if w.dtype == "f32" else "tensor"
+    if kernel == "landmarks":
+        return 2 * tensor + 2 * BH * m * d * 4, 0, "alu"
+    if kernel == "pinv":
+        return BH * 2 * m * d * 4 + BH * m * m * 4, BH * (2 * m * m * d + w.n_iter * 8 * m ** 3), \
+            "alu" if w.dtype == "f32" else "tensor_tf32"
+    if kernel == "k3v_partial":
+        return 2 * tensor + BH * m * d * 4, BH * 4 * n * m * d, unit
+    if kernel == "k3v_combine":
+        return BH * m * d * 8, 0, "alu"
+    if kernel == "w_product":
+        return BH * (m * m + 2 * m * d) * 4, BH * 2 * m * m * d, "alu"
+    if kernel == "output":
+        return 3 * tensor + BH * 2 * m * d * 4, BH * (4 * n * m * d + (2 * 65 * n * d if w.conv else 0)), unit
+    raise KeyError(kernel)
+
+
+def compute_peak_tflops(unit, peaks, kernel_impl_simt):
+    """Peak of the unit a kernel runs on, in TFLOP/s."""
+    if unit == "alu" or kernel_impl_simt:
+        return N_SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    if unit == "tensor_tf32":
+        return peaks["bf16_tflops"] * 0.5   # nominal tf32 : bf16 dense ratio 1.1 : 2.25
+    return peaks["bf16_tflops"]
+
+
+SIMT_KERNELS = {"landmarks", "k3v_combine", "w_product"}
+
+
+def roofline_for(w, kernel, avg_ms, peaks, simt_set, traffic):
+    nbytes, flops, unit = kernel_work(w, kernel)
+    simt = kernel in simt_set
+    t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
+    cpk = compute_peak_tflops(unit, peaks, simt)
+    t_cmp = flops / (cpk * 1e12) if flops else 0.0
+    sec = avg_ms * 1e-3
+    if t_mem >= t_cmp:
+        achieved = nbytes / sec / 1e9
+        r = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    else:
+        achieved = flops / sec / 1e12
+        bound = "alu" if (simt or unit == "alu") else "tensor"
+        r = {"bound": bound, "achieved": round(achieved, 3), "peak": round(cpk, 1), "unit": "TFLOP/s"}
+    r["frac"] = round(achieved / r["peak"], 4)
+    r["traffic"] = traffic
+    r["kernel"] = kernel
+    r["algorithmic_bytes"] = nbytes
+    r["algorithmic_flops"] = flops
+    r["avg_launch_us"] = round(avg_ms * 1e3, 2)
+    return r
+
+
+def roofline_bound_time(w, peaks):
+    """t_roof = max(ideal bytes / HBM, total flops / bf16 peak) of the whole step."""
+    elt = 4 if w.dtype == "f32" else 2
+    nbytes = 4 * w.BH * w.n * w.d * elt
+    m, n, d = w.m, w.n, w.d
+    flops = w.BH * (4 * 2 * n * m * d + 2 * 2 * m * m * d + w.n_iter * 8 * m ** 3 +
+                    (2 * 65 * n * d if w.conv else 0))
+    peak = peaks["bf16_tflops"] if w.dtype == "bf16" else compute_peak_tflops("alu", peaks, True)
+    return max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peak * 1e12)), nbytes, flops
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "20"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.t = threading.Thread(target=self._read, daemon=True)
+        self.t.start()
+        time.sleep(0.3)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
+                "power_w_max": max(power), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def oracle_sample(w, x, heads, rows=None, threads=0):
+    import oracle
+    b_idx = [b for b, _ in heads]
+    h_idx = [h for _, h in heads]
+    # gather the sampled heads into one [1, S, n, d] batch (head h keeps its conv weight)
+    q = np.ascontiguousarray(x["q"][b_idx, h_idx][None])
+    k = np.ascontiguousarray(x["k"][b_idx, h_idx][None])
+    v = np.ascontiguousarray(x["v"][b_idx, h_idx][None])
+    cw = None if x["conv_w"] is None else np.ascontiguousarray(x["conv_w"][h_idx])
+    if x["mask"] is not None and len(set(b_idx)) > 1:
+        raise ValueError("masked sample must come from one sequence")
+    mask = None if x["mask"] is None else x["mask"][b_idx[0]:b_idx[0] + 1]
+    t0 = time.perf_counter()
+    oracle.forward(q, k, v, mask, cw, m=w.m, n_iter=w.n_iter, rows=rows, threads=threads)
+    return time.perf_counter() - t0
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, x):
+    import oracle
+    oracle.build()
+    cores = cpu_cores()
+    nh = max(1, min(w.BH, cores))
+    heads = [(i // w.H, i % w.H) for i in range(nh)]
+    if x["mask"] is not None:
+        heads = [(0, i % w.H) for i in range(min(nh, w.H))]
+    sec = oracle_sample(w, x, heads, threads=min(cores, len(heads)))
+    toks = len(heads) * w.n
+    return {"value": round(toks / sec, 1), "unit": UNIT, "cores": min(cores, len(heads)),
+            "kind": "oracle",
+            "sample": f"{len(heads)} of {w.BH} heads, all {w.n} rows each, fp64 C oracle, "
+                      f"{sec:.1f} s wall on {min(cores, len(heads))} threads"}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import oracle
+    oracle.build()
+    x = make_inputs(w, seed=0)
+    cores = cpu_cores()
+    nh = max(1, min(w.BH, cores))
+    heads = [(i // w.H, i % w.H) for i in range(nh)]
+    if x["mask"] is not None:
+        heads = [(0, i % w.H) for i in range(min(nh, w.H))]
+    threads = min(cores, len(heads))
+    budget = float(os.environ.get("NYS_REFERENCE_BUDGET_S", "150"))
+    t_warm = 0.0
+    for _ in range(min(args.warmup, 1)):
+        t_warm = oracle_sample(w, x, heads, threads=threads)
+    per = t_warm if t_warm > 0 else None
+    steps_done, total = 0, 0.0
+    while steps_done < args.steps:
+        if per is not None and total + per > budget and steps_done > 0:
+            break
+        dt = oracle_sample(w, x, heads, threads=threads)
+        total += dt
+        per = dt
+        steps_done += 1
+    toks = len(heads) * w.n * steps_done
+    value = toks / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": steps_done, "steps_requested": args.steps,
+        "warmup": min(args.warmup, 1), "ms_per_step": round(1e3 * total / steps_done, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, see workloads/)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "m": w.m,
+                   "n_iter": w.n_iter, "conv": w.conv, "sample_heads": len(heads)},
+        "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"per step {len(heads)} of {w.BH} heads x all {w.n} rows; "
+                                   f"run capped at {budget:.0f} s"},
+        "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=HEADLINE, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-flush", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    import nystr_self_attention_scale_b200 as nys
+
+    x = make_inputs(w, seed=rank)
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    q = torch.from_numpy(x["q"]).to(dt).cuda()
+    k = torch.from_numpy(x["k"]).to(dt).cuda()
+    v = torch.from_numpy(x["v"]).to(dt).cuda()
+    mask = None if x["mask"] is None else torch.from_numpy(x["mask"]).cuda()
+    conv_w = None if x["conv_w"] is None else torch.from_numpy(x["conv_w"]).cuda()
+    out = torch.empty_like(q)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        nys.forward(q, k, v, mask=mask, conv_w=conv_w, m=w.m, n_iter=w.n_iter, out=out)
+
+    for _ in range(args.warmup):
+        if not args.no_flush:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert nys.device_status() == 0
+
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
+    except Exception:
+        gpu_id = None
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    nys.profile_enable(True)
+    for i in range(args.steps):
+        if not args.no_flush:
+            flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    prof = nys.profile_read()
+    nys.profile_enable(False)
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    status = nys.device_status()
+    if world > 1:
+        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    tokens_all = w.tokens * world * args.steps
+    value = tokens_all / (total_ms * 1e-3)
+
+    peaks, peak_src = load_peaks()
+    launches = sum(n for n, _ in prof.values())
+    kernels = {name: {"launches": n, "total_ms": round(ms, 4),
+                      "avg_us": round(1e3 * ms / n, 2) if n else None}
+               for name, (n, ms) in prof.items()}
+    kernel_ms_total = sum(ms for _, ms in prof.values()) or 1.0
+    for name in kernels:
+        kernels[name]["share"] = round(prof[name][1] / kernel_ms_total, 4)
+    dom = max(prof, key=lambda kname: prof[kname][1])
+    traffic = None
+    tf = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tf):
+        with open(tf) as f:
+            tr = json.load(f)
+        ent = tr.get(dom)
+        if ent and ent.get("source_digest") == source_digest() and ent.get("workload") == w.name:
+            traffic = ent.get("bytes_per_launch")
+    simt = set(SIMT_KERNELS)
+    if w.dtype == "f32" or True:  # the first CUDA path runs every stage on CUDA cores
+        simt |= {"pinv", "k3v_partial", "output"}
+    roof = roofline_for(w, dom, prof[dom][1] / max(1, prof[dom][0]), peaks, simt, traffic)
+    roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
+    t_roof, ideal_bytes, total_flops = roofline_bound_time(w, peaks)
+
+    e2e = None
+    if not args.no_e2e:
+        qh = torch.from_numpy(x["q"]).to(dt).pin_memory()
+        kh = torch.from_numpy(x["k"]).to(dt).pin_memory()
+        vh = torch.from_numpy(x["v"]).to(dt).pin_memory()
+        mh = None if x["mask"] is None else torch.from_numpy(x["mask"]).pin_memory()
+        wh = None if x["conv_w"] is None else torch.from_numpy(x["conv_w"]).pin_memory()
+        oh = torch.empty_like(qh).pin_memory()
+        for _ in range(2):
+            nys.forward_host(qh, kh, vh, mask=mh, conv_w=wh, m=w.m, n_iter=w.n_iter, out=oh)
+        if world > 1:
+            dist.barrier()
+        e_ms = 0.0
+        for _ in range(args.e2e_steps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            nys.forward_host(qh, kh, vh, mask=mh, conv_w=wh, m=w.m, n_iter=w.n_iter, out=oh)
+            b.record(stream)
+            b.synchronize()
+            e_ms += a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        elt = qh.element_size()
+        h2d = 3 * qh.numel() * elt + (0 if mh is None else mh.numel()) + (0 if wh is None else wh.numel() * 4)
+        e2e = {"value": round(w.tokens * world * args.e2e_steps / (e_ms * 1e-3), 1), "unit": UNIT,
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(oh.numel() * elt),
+               "steps": args.e2e_steps, "ms_per_step": round(e_ms / args.e2e_steps, 3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded numpy inputs, see workloads/)",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "m": w.m,
+                       "n_iter": w.n_iter, "conv": w.conv, "mask": w.lengths is not None,
+                       "inputs": w.dist, "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "not flushed" if args.no_flush else "flushed before every step (256 MiB write, untimed)"},
+            "roofline": roof,
+            "step_roofline": {"t_roof_us": round(t_roof * 1e6, 2), "frac": round(t_roof / (ms_per_step * 1e-3), 4),
+                              "ideal_bytes": ideal_bytes, "flops": total_flops},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "kernels": kernels, "clocks": clocks, "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

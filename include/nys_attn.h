@@ -1,0 +1,145 @@
+/*
+ * nys_attn.h -- C ABI of the B200 (sm_100a) Nystromformer self-attention forward.
+ *
+ * The operation (per batch b and head h), as the Nystromformer source
+ * walkthrough (blog.gitcode.com) describes it in section 2:
+ *   2.2  Qs = d^-1/4 Q,  Ks = d^-1/4 K            (1/sqrt(d) split over Q and K)
+ *   2.3  Q_l[j] = mean_{t < L} Qs[j L + t],  K_l likewise,  L = n / m
+ *   2.4  k1 = softmax_row(Qs K_l^T)    [n x m]
+ *        k2 = softmax_row(Q_l K_l^T)   [m x m]
+ *        k3 = softmax_row(Q_l Ks^T + mask)   [m x n], padded keys -> probability 0
+ *   2.5  Z  = iterative Moore-Penrose inverse of k2: Z_0 = c k2^T with
+ *        c = 1 / (max column sum * max row sum); n_iter times
+ *        Z <- 1/4 Z (13 I - X (15 I - X (7 I - X))),  X = k2 Z
+ *   2.4  out = k1 Z (k3 V)            (computed as k1 (Z (k3 V)))
+ *   2.6  out += depthwise conv of V along the sequence, 65 taps per head,
+ *        zero padding 32 on each side, no bias (Conv2d kernel (65,1), groups = H)
+ *
+ * Layouts: q, k, v, out are [B, H, n, d] row-major and contiguous (the head
+ * split of walkthrough 2.2). key_mask is [B, n] uint8 with 1 = valid key and
+ * 0 = padded key (the model API's attention_mask convention; HF docs,
+ * NystromformerModel forward). conv_w is [H, 65] float32, the depthwise
+ * Conv2d weight [H, 1, 65, 1] flattened; tap t multiplies V[i + t - 32].
+ *
+ * Ownership: every pointer belongs to the caller; the library keeps none of
+ * them after the call returns. Calls are reentrant.
+ *
+ * Errors: every entry point returns an nys_status_t. Argument checks happen
+ * before anything is launched; NYS_ERR_CUDA wraps a CUDA error reported at
+ * launch time. Device-side waits are bounded: a wait that runs out records
+ * NYS_ERR_TIMEOUT in a device status word that nys_attn_device_status()
+ * returns (and clears).
+ *
+ * Precondition (documented, not checked): every sequence has at least one
+ * valid key; otherwise kernel_3 is 0/0 for that sequence.
+ */
+#ifndef NYS_ATTN_H
+#define NYS_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Depthwise conv taps: the conv_kernel_size default of NystromformerConfig
+ * (walkthrough section 3.1; HF docs NystromformerConfig). */
+#define NYS_CONV_TAPS 65
+/* Default iteration count of the iterative inverse (walkthrough 2.5). */
+#define NYS_DEFAULT_N_ITER 6
+
+typedef enum {
+    NYS_F32 = 0,   /* float32 in, float32 out, float32 arithmetic               */
+    NYS_BF16 = 1   /* bf16 in, bf16 out (round to nearest even), float32 accumulate */
+} nys_dtype_t;
+
+typedef enum {
+    NYS_OK = 0,
+    NYS_ERR_INVALID_ARG = -1,  /* null pointer, non-positive size, n % m != 0, m > n, n_iter < 0 */
+    NYS_ERR_UNSUPPORTED = -2,  /* shape or dtype outside what the kernels implement            */
+    NYS_ERR_CUDA = -3,         /* a CUDA call failed                                           */
+    NYS_ERR_NOMEM = -4,        /* workspace allocation failed                                  */
+    NYS_ERR_TIMEOUT = -5       /* a bounded device-side wait ran out                           */
+} nys_status_t;
+
+/*
+ * nys_attn_forward -- the whole forward of walkthrough section 2 on device memory.
+ *
+ *   q, k, v   device pointers, [B, H, n, d], element type `dtype`
+ *   key_mask  device pointer [B, n] uint8 (1 valid, 0 padded), or NULL for no mask
+ *   conv_w    device pointer [H, 65] float32, or NULL to skip the conv
+ *             (the conv_kernel_size = None case of walkthrough 2.6)
+ *   m         landmarks; n % m == 0 (segment length L = n / m)
+ *   n_iter    iterations of the iterative inverse (the pages' default is 6)
+ *   out       device pointer [B, H, n, d], element type `dtype`; must not alias inputs
+ *   stream    a cudaStream_t (NULL = legacy default stream)
+ *
+ * Supported: d in {32, 64}. float32: 1 <= m <= 256. bf16: m in {64, 128, 256}
+ * and n % 128 == 0. Anything else returns NYS_ERR_UNSUPPORTED.
+ *
+ * Asynchronous: work is enqueued on `stream` and the call returns without a
+ * host synchronisation. Scratch memory comes from cudaMallocAsync on
+ * `stream` and is released with cudaFreeAsync on the same stream.
+ */
+int nys_attn_forward(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                     const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
+                     int dtype, void* out, void* stream);
+
+/*
+ * nys_attn_forward_host -- the same operation on HOST buffers (same shapes,
+ * layouts and checks). Copies the inputs to the device, runs the forward on
+ * `stream`, copies the result back into `out` and synchronises `stream`
+ * before returning. Host buffers should be pinned (cudaHostAlloc) for full
+ * copy bandwidth; pageable memory works but is slower. Device buffers are
+ * taken with cudaMallocAsync and released before return.
+ */
+int nys_attn_forward_host(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                          const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
+                          int dtype, void* out, void* stream);
+
+/*
+ * nys_attn_forward_debug -- nys_attn_forward plus copies of the intermediate
+ * stages, for tests. Each stage pointer is a device float32 buffer or NULL:
+ *   q_l, k_l [B, H, m, d]   landmarks of the scaled Q and K (walkthrough 2.3)
+ *   z        [B, H, m, m]   iterative inverse of kernel_2 (2.5)
+ *   k3v      [B, H, m, d]   kernel_3 V (2.4)
+ *   w        [B, H, m, d]   Z (kernel_3 V)
+ * The main output is written as in nys_attn_forward.
+ */
+int nys_attn_forward_debug(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                           const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
+                           int dtype, void* out, float* q_l, float* k_l, float* z, float* k3v,
+                           float* w, void* stream);
+
+/* Synchronises the current device, then returns and clears the device status
+ * word (NYS_OK or NYS_ERR_TIMEOUT); NYS_ERR_CUDA if the synchronisation fails. */
+int nys_attn_device_status(void);
+
+/* Bytes of device scratch nys_attn_forward takes for this shape (0 if invalid). */
+size_t nys_attn_workspace_bytes(int B, int H, int n, int d, int m, int dtype);
+
+/* Short English text for a status code; never NULL. */
+const char* nys_strerror(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int nys_attn_version(void);
+
+/*
+ * Per-kernel timing, for benchmarks. While enabled, each kernel launch of
+ * the forward is bracketed by two CUDA events recorded on the stream the
+ * kernel runs on. nys_attn_profile_enable() clears the counters (and turns
+ * recording on or off); nys_attn_profile_read() waits for the recorded
+ * events and returns, for one kernel id in [0, nys_attn_kernel_count()),
+ * the number of timed launches and their summed device time in ms.
+ */
+int nys_attn_profile_enable(int on);
+int nys_attn_profile_read(int kernel_id, int* launches, double* total_ms);
+int nys_attn_kernel_count(void);
+const char* nys_attn_kernel_name(int kernel_id);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NYS_ATTN_H */

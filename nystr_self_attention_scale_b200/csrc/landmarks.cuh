@@ -1,0 +1,73 @@
+// landmarks.cuh -- fused d^-1/4 scale + segment means of Q and K.
+//
+// Walkthrough (blog.gitcode.com) 2.2 and 2.3: Q_l[j] = mean over the L = n/m
+// consecutive rows j*L .. j*L+L-1 of d^-1/4 * Q; the same for K.
+//
+// One thread owns one 16-byte column slice (4 fp32 or 8 bf16 elements) of one
+// landmark and walks the L rows of its segment; the d/kVec threads of a
+// landmark read each row as one contiguous 64- or 128-byte run, so every load
+// is a full 128-bit access and each warp touches whole 32-byte sectors only.
+// The sum is accumulated in fp32 and multiplied once by fl(d^-1/4) / L.
+#pragma once
+
+#include "common.cuh"
+
+namespace nys {
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+landmarks_kernel(const T* __restrict__ q, const T* __restrict__ k, float* __restrict__ ql,
+                 float* __restrict__ kl, __nv_bfloat16* __restrict__ ql16,
+                 __nv_bfloat16* __restrict__ kl16, int BH, int n, int d, int m) {
+    constexpr int V = Elt<T>::kVec;
+    const int slices = d / V;                                 // threads per landmark row
+    const long long per_tensor = (long long)BH * m * slices;
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int which = blockIdx.y;                             // 0: Q, 1: K
+    if (gid >= per_tensor) return;
+    const int slice = (int)(gid % slices);
+    const long long lm = gid / slices;                        // (bh, j) flattened
+    const int j = (int)(lm % m);
+    const long long bh = lm / m;
+    const int L = n / m;
+    const T* src = (which == 0 ? q : k) + ((bh * n + (long long)j * L) * d) + slice * V;
+
+    float acc[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[e] = 0.f;
+    int t = 0;
+    for (; t + 4 <= L; t += 4) {
+        float x0[V], x1[V], x2[V], x3[V];
+        Elt<T>::load16(src + (long long)(t + 0) * d, x0);
+        Elt<T>::load16(src + (long long)(t + 1) * d, x1);
+        Elt<T>::load16(src + (long long)(t + 2) * d, x2);
+        Elt<T>::load16(src + (long long)(t + 3) * d, x3);
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] += (x0[e] + x1[e]) + (x2[e] + x3[e]);
+    }
+    for (; t < L; ++t) {
+        float x0[V];
+        Elt<T>::load16(src + (long long)t * d, x0);
+#pragma unroll
+        for (int e = 0; e < V; ++e) acc[e] += x0[e];
+    }
+    const float scale = split_scale(d) / (float)L;
+    float* dst = (which == 0 ? ql : kl) + lm * d + slice * V;
+    __nv_bfloat16* dst16 = which == 0 ? ql16 : kl16;
+#pragma unroll
+    for (int e = 0; e < V; e += 4) {
+        float4 o = make_float4(acc[e] * scale, acc[e + 1] * scale, acc[e + 2] * scale,
+                               acc[e + 3] * scale);
+        *reinterpret_cast<float4*>(dst + e) = o;
+        if (dst16) {
+            __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(dst16 + lm * d + slice * V + e) = pk;
+        }
+    }
+}
+
+}  // namespace nys

@@ -1,0 +1,379 @@
+// nys_attn.cu -- C ABI and launch sequence of the Nystromformer attention forward.
+//
+// Per call (walkthrough, blog.gitcode.com, section 2):
+//   1. landmarks: fused d^-1/4 scale + segment means of Q and K      (2.2, 2.3)
+//   2. kernel_2 + iterative inverse -> Z, on a forked stream           (2.4, 2.5)
+//   3. kernel_3 V: online softmax over key splits + combine            (2.4)
+//   4. W = Z (kernel_3 V)                                              (2.4)
+//   5. output: softmax(Qs K_l^T) W + dwconv65(V)                       (2.4, 2.6)
+// Steps 2 and 3 are independent and overlap; 4 joins them.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <mutex>
+#include <vector>
+
+#include "common.cuh"
+#include "landmarks.cuh"
+#include "simt.cuh"
+
+namespace nys {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool ready = false;
+    int sm_count = 0;
+    cudaStream_t aux = nullptr;       // forked stream for the iterative inverse
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex launch_mu;             // serialises the fork/join event use of one device
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+int device_state(DeviceState** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NYS_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.ready) {
+        if (cudaDeviceGetAttribute(&st.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return NYS_ERR_CUDA;
+        if (cudaStreamCreateWithFlags(&st.aux, cudaStreamNonBlocking) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&st.fork, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
+        // Keep freed async allocations in the pool so per-call workspace is cheap.
+        cudaMemPool_t pool;
+        if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+            uint64_t keep = UINT64_MAX;
+            cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        }
+        const size_t big = 200 * 1024;
+        cudaFuncSetAttribute(k3v_partial_simt_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(k3v_partial_simt_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(k3v_partial_simt_kernel<__nv_bfloat16, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(k3v_partial_simt_kernel<__nv_bfloat16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(output_simt_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(output_simt_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(output_simt_kernel<__nv_bfloat16, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(output_simt_kernel<__nv_bfloat16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        if (cudaGetLastError() != cudaSuccess) return NYS_ERR_CUDA;
+        st.ready = true;
+    }
+    *out = &st;
+    return NYS_OK;
+}
+
+size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- per-kernel timing
+// When enabled, every launch is bracketed by two CUDA events on the stream it
+// runs on; nys_attn_profile_read() sums their elapsed times per kernel.
+enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_COUNT };
+const char* const kKernelNames[K_COUNT] = {"landmarks", "pinv", "k3v_partial", "k3v_combine",
+                                           "w_product", "output"};
+
+struct ProfRecord { int kid; cudaEvent_t a, b; };
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRecord> g_prof;
+int g_prof_launches[K_COUNT];
+double g_prof_ms[K_COUNT];
+
+struct ProfScope {
+    int kid;
+    cudaStream_t s;
+    cudaEvent_t a = nullptr, b = nullptr;
+    ProfScope(int kid_, cudaStream_t s_) : kid(kid_), s(s_) {
+        if (!g_prof_on) return;
+        cudaEventCreate(&a);
+        cudaEventCreate(&b);
+        cudaEventRecord(a, s);
+    }
+    ~ProfScope() {
+        if (!a) return;
+        cudaEventRecord(b, s);
+        std::lock_guard<std::mutex> lock(g_prof_mu);
+        g_prof.push_back({kid, a, b});
+    }
+};
+
+void prof_drain() {
+    std::lock_guard<std::mutex> lock(g_prof_mu);
+    for (auto& r : g_prof) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+            g_prof_ms[r.kid] += ms;
+            g_prof_launches[r.kid] += 1;
+        }
+        cudaEventDestroy(r.a);
+        cudaEventDestroy(r.b);
+    }
+    g_prof.clear();
+}
+
+// Workspace carve-up (byte offsets, each 256-byte aligned).
+struct Plan {
+    int B, H, n, d, m, n_iter, dtype;
+    int BH, splits, keys_per_split;
+    size_t off_ql, off_kl, off_ql16, off_kl16, off_k3v, off_w, off_wt16, off_z, off_pinv;
+    size_t off_po, off_pm, off_pl, total;
+};
+
+int validate(const void* q, const void* k, const void* v, const void* out, int B, int H, int n,
+             int d, int m, int n_iter, int dtype) {
+    if (!q || !k || !v || !out) return NYS_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || n <= 0 || d <= 0 || m <= 0 || n_iter < 0) return NYS_ERR_INVALID_ARG;
+    if (n % m != 0 || m > n) return NYS_ERR_INVALID_ARG;
+    if (dtype != NYS_F32 && dtype != NYS_BF16) return NYS_ERR_UNSUPPORTED;
+    if (d != 32 && d != 64) return NYS_ERR_UNSUPPORTED;
+    if (m > 256) return NYS_ERR_UNSUPPORTED;
+    if (dtype == NYS_BF16 && ((m != 64 && m != 128 && m != 256) || n % 128 != 0))
+        return NYS_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1 << 24) || n / 64 >= 65535) return NYS_ERR_UNSUPPORTED;
+    return NYS_OK;
+}
+
+Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_count) {
+    Plan p{};
+    p.B = B; p.H = H; p.n = n; p.d = d; p.m = m; p.n_iter = n_iter; p.dtype = dtype;
+    p.BH = B * H;
+    // The key split depends on n only (never on B*H or the GPU), so a head's
+    // result is bitwise the same alone or inside any batch.
+    (void)sm_count;
+    const int kps = std::min(((n + 63) / 64) * 64, 1024);
+    const int splits = (n + kps - 1) / kps;
+    p.splits = splits;
+    p.keys_per_split = kps;
+    const size_t BH = p.BH, md = (size_t)m * d, mm = (size_t)m * m;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+    p.off_ql = take(BH * md * 4);
+    p.off_kl = take(BH * md * 4);
+    p.off_ql16 = take(BH * md * 2);
+    p.off_kl16 = take(BH * md * 2);
+    p.off_k3v = take(BH * md * 4);
+    p.off_w = take(BH * md * 4);
+    p.off_wt16 = take(BH * md * 2);
+    p.off_z = take(BH * mm * 4);
+    p.off_pinv = take(BH * 5 * mm * 4);
+    p.off_po = take(BH * splits * md * 4);
+    p.off_pm = take(BH * splits * (size_t)m * 4);
+    p.off_pl = take(BH * splits * (size_t)m * 4);
+    p.total = o;
+    return p;
+}
+
+template <typename T, int D>
+int launch_all(const Plan& p, const DeviceState& st, const T* q, const T* k, const T* v,
+               const uint8_t* mask, const float* conv_w, T* out, char* ws, cudaStream_t s) {
+    float* ql = reinterpret_cast<float*>(ws + p.off_ql);
+    float* kl = reinterpret_cast<float*>(ws + p.off_kl);
+    float* k3v = reinterpret_cast<float*>(ws + p.off_k3v);
+    float* w = reinterpret_cast<float*>(ws + p.off_w);
+    float* z = reinterpret_cast<float*>(ws + p.off_z);
+    float* pinv = reinterpret_cast<float*>(ws + p.off_pinv);
+    float* po = reinterpret_cast<float*>(ws + p.off_po);
+    float* pm = reinterpret_cast<float*>(ws + p.off_pm);
+    float* pl = reinterpret_cast<float*>(ws + p.off_pl);
+    const int BH = p.BH, n = p.n, m = p.m;
+
+    {
+        constexpr int V = Elt<T>::kVec;
+        long long threads = (long long)BH * m * (D / V);
+        dim3 grid((unsigned)((threads + 255) / 256), 2);
+        ProfScope ps(K_LANDMARKS, s);
+        landmarks_kernel<T><<<grid, 256, 0, s>>>(q, k, ql, kl, nullptr, nullptr, BH, n, D, m);
+    }
+    if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
+    if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
+    {
+        ProfScope ps(K_PINV, st.aux);
+        pinv_simt_kernel<<<BH, 256, 0, st.aux>>>(ql, kl, z, pinv, m, D, p.n_iter);
+    }
+    if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
+    {
+        dim3 grid(BH, (m + 63) / 64, p.splits);
+        {
+            ProfScope ps(K_K3V, s);
+            k3v_partial_simt_kernel<T, D><<<grid, 256, k3v_simt_smem_bytes<D>(), s>>>(
+                ql, k, v, mask, po, pm, pl, p.H, n, m, p.splits, p.keys_per_split);
+        }
+        dim3 g2(BH, std::max(1, (m * D) / 1024));
+        ProfScope ps(K_COMBINE, s);
+        k3v_combine_kernel<<<g2, 256, 0, s>>>(po, pm, pl, k3v, m, D, p.splits);
+    }
+    if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;
+    {
+        ProfScope ps(K_W, s);
+        w_kernel<<<dim3(BH, (m + 31) / 32), 256, 0, s>>>(z, k3v, w, nullptr, m, D);
+    }
+    {
+        dim3 grid(BH, (n + 63) / 64);
+        ProfScope ps(K_OUTPUT, s);
+        output_simt_kernel<T, D><<<grid, 256, OutSmem<T, D>::bytes(m), s>>>(q, kl, w, v, conv_w, out,
+                                                                          p.H, n, m);
+    }
+    return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
+
+int run(const void* q, const void* k, const void* v, const uint8_t* mask, const float* conv_w,
+        int B, int H, int n, int d, int m, int n_iter, int dtype, void* out, float* dbg_ql,
+        float* dbg_kl, float* dbg_z, float* dbg_k3v, float* dbg_w, cudaStream_t s) {
+    int rc = validate(q, k, v, out, B, H, n, d, m, n_iter, dtype);
+    if (rc != NYS_OK) return rc;
+    DeviceState* st = nullptr;
+    rc = device_state(&st);
+    if (rc != NYS_OK) return rc;
+    const Plan p = make_plan(B, H, n, d, m, n_iter, dtype, st->sm_count);
+    void* ws = nullptr;
+    if (cudaMallocAsync(&ws, p.total, s) != cudaSuccess) {
+        cudaGetLastError();
+        return NYS_ERR_NOMEM;
+    }
+    char* w = static_cast<char*>(ws);
+    std::unique_lock<std::mutex> launch_lock(st->launch_mu);
+    if (dtype == NYS_F32) {
+        rc = d == 64 ? launch_all<float, 64>(p, *st, (const float*)q, (const float*)k, (const float*)v,
+                                             mask, conv_w, (float*)out, w, s)
+                     : launch_all<float, 32>(p, *st, (const float*)q, (const float*)k, (const float*)v,
+                                             mask, conv_w, (float*)out, w, s);
+    } else {
+        using bf = __nv_bfloat16;
+        rc = d == 64 ? launch_all<bf, 64>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask,
+                                          conv_w, (bf*)out, w, s)
+                     : launch_all<bf, 32>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask,
+                                          conv_w, (bf*)out, w, s);
+    }
+    if (rc == NYS_OK) {
+        const size_t BH = p.BH, md = (size_t)m * d, mm = (size_t)m * m;
+        struct { float* dst; size_t off; size_t bytes; } copies[] = {
+            {dbg_ql, p.off_ql, BH * md * 4}, {dbg_kl, p.off_kl, BH * md * 4},
+            {dbg_z, p.off_z, BH * mm * 4}, {dbg_k3v, p.off_k3v, BH * md * 4},
+            {dbg_w, p.off_w, BH * md * 4}};
+        for (auto& c : copies)
+            if (c.dst && cudaMemcpyAsync(c.dst, w + c.off, c.bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+                rc = NYS_ERR_CUDA;
+    }
+    if (cudaFreeAsync(ws, s) != cudaSuccess && rc == NYS_OK) rc = NYS_ERR_CUDA;
+    return rc;
+}
+
+}  // namespace
+}  // namespace nys
+
+extern "C" {
+
+int nys_attn_forward(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                     const float* conv_w, int B, int H, int n, int d, int m, int n_iter, int dtype,
+                     void* out, void* stream) {
+    return nys::run(q, k, v, key_mask, conv_w, B, H, n, d, m, n_iter, dtype, out, nullptr, nullptr,
+                    nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+int nys_attn_forward_debug(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                           const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
+                           int dtype, void* out, float* q_l, float* k_l, float* z, float* k3v,
+                           float* w, void* stream) {
+    return nys::run(q, k, v, key_mask, conv_w, B, H, n, d, m, n_iter, dtype, out, q_l, k_l, z, k3v,
+                    w, static_cast<cudaStream_t>(stream));
+}
+
+int nys_attn_forward_host(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                          const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
+                          int dtype, void* out, void* stream) {
+    int rc = nys::validate(q, k, v, out, B, H, n, d, m, n_iter, dtype);
+    if (rc != NYS_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t elt = dtype == NYS_F32 ? 4 : 2;
+    const size_t tensor = (size_t)B * H * n * d * elt;
+    const size_t mask_bytes = key_mask ? (size_t)B * n : 0;
+    const size_t w_bytes = conv_w ? (size_t)H * NYS_CONV_TAPS * sizeof(float) : 0;
+    const size_t o_q = 0, o_k = nys::align_up(tensor), o_v = 2 * o_k, o_o = 3 * o_k;
+    const size_t o_mask = 4 * o_k, o_w = o_mask + nys::align_up(mask_bytes);
+    const size_t total = o_w + nys::align_up(w_bytes);
+    void* buf = nullptr;
+    if (cudaMallocAsync(&buf, total, s) != cudaSuccess) {
+        cudaGetLastError();
+        return NYS_ERR_NOMEM;
+    }
+    char* b = static_cast<char*>(buf);
+    bool ok = cudaMemcpyAsync(b + o_q, q, tensor, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+              cudaMemcpyAsync(b + o_k, k, tensor, cudaMemcpyHostToDevice, s) == cudaSuccess &&
+              cudaMemcpyAsync(b + o_v, v, tensor, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    if (ok && key_mask) ok = cudaMemcpyAsync(b + o_mask, key_mask, mask_bytes, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    if (ok && conv_w) ok = cudaMemcpyAsync(b + o_w, conv_w, w_bytes, cudaMemcpyHostToDevice, s) == cudaSuccess;
+    rc = ok ? NYS_OK : NYS_ERR_CUDA;
+    if (rc == NYS_OK)
+        rc = nys_attn_forward(b + o_q, b + o_k, b + o_v, key_mask ? (const uint8_t*)(b + o_mask) : nullptr,
+                              conv_w ? (const float*)(b + o_w) : nullptr, B, H, n, d, m, n_iter, dtype,
+                              b + o_o, stream);
+    if (rc == NYS_OK && cudaMemcpyAsync(out, b + o_o, tensor, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        rc = NYS_ERR_CUDA;
+    cudaFreeAsync(buf, s);
+    if (cudaStreamSynchronize(s) != cudaSuccess && rc == NYS_OK) rc = NYS_ERR_CUDA;
+    return rc;
+}
+
+int nys_attn_device_status(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return NYS_ERR_CUDA;
+    int val = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&val, nys::g_status, sizeof(int)) != cudaSuccess) return NYS_ERR_CUDA;
+    if (cudaMemcpyToSymbol(nys::g_status, &zero, sizeof(int)) != cudaSuccess) return NYS_ERR_CUDA;
+    return val;
+}
+
+size_t nys_attn_workspace_bytes(int B, int H, int n, int d, int m, int dtype) {
+    const char dummy = 0;
+    if (nys::validate(&dummy, &dummy, &dummy, &dummy, B, H, n, d, m, 0, dtype) != NYS_OK) return 0;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaGetLastError();
+    return nys::make_plan(B, H, n, d, m, 0, dtype, sms).total;
+}
+
+const char* nys_strerror(int status) {
+    switch (status) {
+        case NYS_OK: return "ok";
+        case NYS_ERR_INVALID_ARG: return "invalid argument";
+        case NYS_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case NYS_ERR_CUDA: return "CUDA error";
+        case NYS_ERR_NOMEM: return "device workspace allocation failed";
+        case NYS_ERR_TIMEOUT: return "bounded device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int nys_attn_version(void) { return 100; }
+
+int nys_attn_profile_enable(int on) {
+    nys::prof_drain();
+    std::lock_guard<std::mutex> lock(nys::g_prof_mu);
+    nys::g_prof_on = on != 0;
+    for (int i = 0; i < nys::K_COUNT; ++i) {
+        nys::g_prof_ms[i] = 0.0;
+        nys::g_prof_launches[i] = 0;
+    }
+    return NYS_OK;
+}
+
+int nys_attn_profile_read(int kernel_id, int* launches, double* total_ms) {
+    if (kernel_id < 0 || kernel_id >= nys::K_COUNT || !launches || !total_ms) return NYS_ERR_INVALID_ARG;
+    nys::prof_drain();
+    std::lock_guard<std::mutex> lock(nys::g_prof_mu);
+    *launches = nys::g_prof_launches[kernel_id];
+    *total_ms = nys::g_prof_ms[kernel_id];
+    return NYS_OK;
+}
+
+int nys_attn_kernel_count(void) { return nys::K_COUNT; }
+
+const char* nys_attn_kernel_name(int kernel_id) {
+    if (kernel_id < 0 || kernel_id >= nys::K_COUNT) return "";
+    return nys::kKernelNames[kernel_id];
+}
+
+}  // extern "C"

@@ -1,0 +1,482 @@
+// simt.cuh -- float32 CUDA-core kernels of the Nystromformer attention forward.
+//
+// These carry the float32 path (fp32 in, fp32 out, FFMA arithmetic), where
+// tensor-core precision (bf16 / tf32 operands) would not meet a 1e-4 relative
+// error budget, and the m x m stages that are small for every shape.
+// Walkthrough (blog.gitcode.com) section references are given per kernel.
+#pragma once
+
+#include "common.cuh"
+
+namespace nys {
+
+// ------------------------------------------------------------------ block GEMM
+// C = alpha * (A . op(B)) + diag * I over a rows x cols output, by one CTA of
+// 256 threads. A is rows x inner row-major (lda); B is inner x cols row-major
+// (ldb) or, with TRANS_B, cols x inner row-major. 64 x 64 output tiles, each
+// thread owns a 4 x 4 sub-block; the inner dimension is staged 16 at a time
+// through shared memory. Callers synchronise the block around it.
+struct GemmSmem {
+    float a[16][64 + 4];
+    float b[16][64 + 4];
+};
+
+template <bool TRANS_B>
+__device__ void block_gemm(float* __restrict__ C, int ldc, const float* __restrict__ A, int lda,
+                           const float* __restrict__ B, int ldb, int rows, int inner, int cols,
+                           float alpha, float diag, GemmSmem& sm) {
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    for (int r0 = 0; r0 < rows; r0 += 64) {
+        for (int c0 = 0; c0 < cols; c0 += 64) {
+            float acc[4][4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+            for (int k0 = 0; k0 < inner; k0 += 16) {
+                // A tile: 64 rows x 16 k, stored k-major
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int idx = tid + e * 256;
+                    int r = idx >> 4, kk = idx & 15;
+                    int gr = r0 + r, gk = k0 + kk;
+                    sm.a[kk][r] = (gr < rows && gk < inner) ? A[(size_t)gr * lda + gk] : 0.f;
+                }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    int idx = tid + e * 256;
+                    if (TRANS_B) {
+                        int c = idx >> 4, kk = idx & 15;
+                        int gc = c0 + c, gk = k0 + kk;
+                        sm.b[kk][c] = (gc < cols && gk < inner) ? B[(size_t)gc * ldb + gk] : 0.f;
+                    } else {
+                        int kk = idx >> 6, c = idx & 63;
+                        int gc = c0 + c, gk = k0 + kk;
+                        sm.b[kk][c] = (gc < cols && gk < inner) ? B[(size_t)gk * ldb + gc] : 0.f;
+                    }
+                }
+                __syncthreads();
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    float4 av = *reinterpret_cast<const float4*>(&sm.a[kk][ty * 4]);
+                    float4 bv = *reinterpret_cast<const float4*>(&sm.b[kk][tx * 4]);
+                    float a4[4] = {av.x, av.y, av.z, av.w};
+                    float b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+                }
+                __syncthreads();
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                int gr = r0 + ty * 4 + i;
+                if (gr >= rows) continue;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    int gc = c0 + tx * 4 + j;
+                    if (gc >= cols) continue;
+                    C[(size_t)gr * ldc + gc] = alpha * acc[i][j] + (gr == gc ? diag : 0.f);
+                }
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ kernel_2 + iterative inverse
+// Walkthrough 2.4 (kernel_2 = softmax(Q_l K_l^T)) and 2.5 (iterative inverse):
+//   Z_0 = c k2^T, c = 1 / (max column sum * max row sum)
+//   repeat: X = k2 Z; T = 7I - X; U = 15I - X T; T = 13I - X U; Z = Z T / 4
+// One CTA per (batch, head); the m x m matrices live in global scratch
+// (L2-resident), 5 per head: k2, X, T, U, and the second Z buffer.
+__global__ void __launch_bounds__(256)
+pinv_simt_kernel(const float* __restrict__ ql, const float* __restrict__ kl, float* __restrict__ z_out,
+                 float* __restrict__ scratch, int m, int d, int n_iter) {
+    __shared__ GemmSmem sm;
+    __shared__ float red[2][8];
+    const int bh = blockIdx.x;
+    const size_t mm = (size_t)m * m;
+    float* A = scratch + (size_t)bh * 5 * mm;
+    float* X = A + mm;
+    float* T = X + mm;
+    float* U = T + mm;
+    float* Zb = U + mm;
+    float* Z = z_out + (size_t)bh * mm;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    block_gemm<true>(A, m, ql + (size_t)bh * m * d, d, kl + (size_t)bh * m * d, d, m, d, m, 1.f, 0.f, sm);
+    __syncthreads();
+    for (int r = warp; r < m; r += 8) {
+        float* row = A + (size_t)r * m;
+        float mx = -INFINITY;
+        for (int c = lane; c < m; c += 32) mx = fmaxf(mx, row[c]);
+        mx = warp_max(mx);
+        float s = 0.f;
+        for (int c = lane; c < m; c += 32) {
+            float e = __expf(row[c] - mx);
+            row[c] = e;
+            s += e;
+        }
+        s = warp_sum(s);
+        const float inv = 1.f / s;
+        for (int c = lane; c < m; c += 32) row[c] *= inv;
+    }
+    __syncthreads();
+    float mcol = -INFINITY, mrow = -INFINITY;
+    for (int i = tid; i < m; i += 256) {
+        float cs = 0.f, rs = 0.f;
+        for (int j = 0; j < m; ++j) {
+            cs += A[(size_t)j * m + i];
+            rs += A[(size_t)i * m + j];
+        }
+        mcol = fmaxf(mcol, cs);
+        mrow = fmaxf(mrow, rs);
+    }
+    mcol = warp_max(mcol);
+    mrow = warp_max(mrow);
+    if (lane == 0) { red[0][warp] = mcol; red[1][warp] = mrow; }
+    __syncthreads();
+    float c_mc = red[0][0], c_mr = red[1][0];
+    for (int w = 1; w < 8; ++w) { c_mc = fmaxf(c_mc, red[0][w]); c_mr = fmaxf(c_mr, red[1][w]); }
+    const float coeff = 1.f / (c_mc * c_mr);
+    for (size_t e = tid; e < mm; e += 256) {
+        size_t r = e / m, c = e % m;
+        Z[e] = coeff * A[c * m + r];
+    }
+    __syncthreads();
+    float* zc = Z;
+    float* zn = Zb;
+    for (int it = 0; it < n_iter; ++it) {
+        block_gemm<false>(X, m, A, m, zc, m, m, m, m, 1.f, 0.f, sm);       // X = A Z
+        __syncthreads();
+        for (size_t e = tid; e < mm; e += 256) {
+            size_t r = e / m, c = e % m;
+            T[e] = (r == c ? 7.f : 0.f) - X[e];                             // T = 7I - X
+        }
+        __syncthreads();
+        block_gemm<false>(U, m, X, m, T, m, m, m, m, -1.f, 15.f, sm);      // U = 15I - X T
+        __syncthreads();
+        block_gemm<false>(T, m, X, m, U, m, m, m, m, -1.f, 13.f, sm);      // T = 13I - X U
+        __syncthreads();
+        block_gemm<false>(zn, m, zc, m, T, m, m, m, m, 0.25f, 0.f, sm);    // Z = Z T / 4
+        __syncthreads();
+        float* t = zc; zc = zn; zn = t;
+    }
+    if (zc != Z) {
+        for (size_t e = tid; e < mm; e += 256) Z[e] = zc[e];
+    }
+}
+
+// ------------------------------------------------------------------ kernel_3 V, split over keys
+// Walkthrough 2.4: k3 = softmax_row(Q_l Ks^T + mask), new_value = k3 V.
+// CTA (bh, 64-landmark block, key split) runs an online softmax over its key
+// range in 64-key chunks and writes unnormalised partials: O (64 x D), the
+// running max M and the running sum l per landmark row.
+template <int D>
+constexpr size_t k3v_simt_smem_bytes() { return sizeof(float) * (2 * D * 68 + 64 * (D + 4) + 64 * 68); }
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+k3v_partial_simt_kernel(const float* __restrict__ ql, const T* __restrict__ k, const T* __restrict__ v,
+                        const uint8_t* __restrict__ mask, float* __restrict__ part_o,
+                        float* __restrict__ part_m, float* __restrict__ part_l, int H, int n, int m,
+                        int splits, int keys_per_split) {
+    constexpr int CW = D / 16;  // output columns per thread
+    extern __shared__ float smem[];
+    float (*sQ)[68] = reinterpret_cast<float (*)[68]>(smem);                  // [D][68]
+    float (*sK)[68] = reinterpret_cast<float (*)[68]>(smem + D * 68);         // [D][68]
+    float (*sV)[D + 4] = reinterpret_cast<float (*)[D + 4]>(smem + 2 * D * 68);  // [64][D+4]
+    float (*sP)[68] = reinterpret_cast<float (*)[68]>(smem + 2 * D * 68 + 64 * (D + 4));  // [64][68]
+    const int bh = blockIdx.x, lb = blockIdx.y, sp = blockIdx.z;
+    const int b = bh / H;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const int j0 = lb * 64;
+    const float s = split_scale(D);
+    for (int e = tid; e < 64 * D; e += 256) {
+        int r = e / D, c = e % D;
+        sQ[c][r] = (j0 + r < m) ? ql[((size_t)bh * m + j0 + r) * D + c] : 0.f;
+    }
+    float o[4][CW], mrun[4], lrun[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        mrun[i] = -INFINITY;
+        lrun[i] = 0.f;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) o[i][j] = 0.f;
+    }
+    const int kbeg = sp * keys_per_split;
+    const int kend = min(n, kbeg + keys_per_split);
+    const T* kb = k + (size_t)bh * n * D;
+    const T* vb = v + (size_t)bh * n * D;
+    for (int c0 = kbeg; c0 < kend; c0 += 64) {
+        __syncthreads();
+        for (int e = tid; e < 64 * D; e += 256) {
+            int r = e / D, c = e % D;
+            int key = c0 + r;
+            bool ok = key < kend;
+            sK[c][r] = ok ? s * Elt<T>::to_f(kb[(size_t)key * D + c]) : 0.f;
+            sV[r][c] = ok ? Elt<T>::to_f(vb[(size_t)key * D + c]) : 0.f;
+        }
+        __syncthreads();
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < D; ++e) {
+            float4 av = *reinterpret_cast<const float4*>(&sQ[e][ty * 4]);
+            float4 bv = *reinterpret_cast<const float4*>(&sK[e][tx * 4]);
+            float a4[4] = {av.x, av.y, av.z, av.w};
+            float b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+        }
+        bool valid[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            int key = c0 + tx * 4 + j;
+            valid[j] = key < kend && (mask == nullptr || mask[(size_t)b * n + key] != 0);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float cm = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (!valid[j]) acc[i][j] = -INFINITY;
+                cm = fmaxf(cm, acc[i][j]);
+            }
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+            const float mnew = fmaxf(mrun[i], cm);
+            const float alpha = (mnew == -INFINITY) ? 1.f : __expf(mrun[i] - mnew);
+            float rs = 0.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float p = (mnew == -INFINITY) ? 0.f : __expf(acc[i][j] - mnew);
+                sP[ty * 4 + i][tx * 4 + j] = p;
+                rs += p;
+            }
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) rs += __shfl_xor_sync(0xffffffffu, rs, off);
+            lrun[i] = lrun[i] * alpha + rs;
+            mrun[i] = mnew;
+#pragma unroll
+            for (int j = 0; j < CW; ++j) o[i][j] *= alpha;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int kk = 0; kk < 64; ++kk) {
+            float pv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pv[i] = sP[ty * 4 + i][kk];
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+                float vv = sV[kk][tx * CW + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[i][j] = fmaf(pv[i], vv, o[i][j]);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int j = j0 + ty * 4 + i;
+        if (j >= m) continue;
+        size_t row = ((size_t)bh * splits + sp) * m + j;
+#pragma unroll
+        for (int c = 0; c < CW; ++c) part_o[row * D + tx * CW + c] = o[i][c];
+        if (tx == 0) {
+            part_m[row] = mrun[i];
+            part_l[row] = lrun[i];
+        }
+    }
+}
+
+// Merge the key-split partials: k3v[j] = sum_s e^{M_s - M} O_s / sum_s e^{M_s - M} l_s.
+// The split order is fixed, so the result is deterministic.
+__global__ void __launch_bounds__(256)
+k3v_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_m,
+                   const float* __restrict__ part_l, float* __restrict__ k3v, int m, int d, int splits) {
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x;
+    for (int e = blockIdx.y * 256 + tid; e < m * d; e += gridDim.y * 256) {
+        const int j = e / d, c = e % d;
+        float M = -INFINITY;
+        for (int s = 0; s < splits; ++s) M = fmaxf(M, part_m[((size_t)bh * splits + s) * m + j]);
+        float num = 0.f, den = 0.f;
+        for (int s = 0; s < splits; ++s) {
+            size_t row = ((size_t)bh * splits + s) * m + j;
+            float ms = part_m[row];
+            float f = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+            num = fmaf(f, part_o[row * d + c], num);
+            den = fmaf(f, part_l[row], den);
+        }
+        k3v[((size_t)bh * m + j) * d + c] = num / den;
+    }
+}
+
+// W = Z (k3 V): 32 rows of W per CTA (walkthrough 2.4, reassociated as k1 (Z (k3 V))).
+// Also writes W^T in bf16 ([d, m] per head) when wt16 is given.
+__global__ void __launch_bounds__(256)
+w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __restrict__ w,
+         __nv_bfloat16* __restrict__ wt16, int m, int d) {
+    __shared__ float sZ[32][256 + 1];
+    const int bh = blockIdx.x, r0 = blockIdx.y * 32;
+    const int tid = threadIdx.x;
+    const int rows = min(32, m - r0);
+    for (int e = tid; e < 32 * m; e += 256) {
+        int r = e / m, c = e % m;
+        sZ[r][c] = r < rows ? z[((size_t)bh * m + r0 + r) * m + c] : 0.f;
+    }
+    __syncthreads();
+    const float* kv = k3v + (size_t)bh * m * d;
+    for (int e = tid; e < 32 * d; e += 256) {
+        int r = e / d, c = e % d;
+        if (r >= rows) continue;
+        float acc = 0.f;
+        for (int kk = 0; kk < m; ++kk) acc = fmaf(sZ[r][kk], kv[(size_t)kk * d + c], acc);
+        w[((size_t)bh * m + r0 + r) * d + c] = acc;
+        if (wt16) wt16[((size_t)bh * d + c) * m + r0 + r] = __float2bfloat16_rn(acc);
+    }
+}
+
+// ------------------------------------------------------------------ output pass
+// Walkthrough 2.4 and 2.6: out = softmax_row(Qs K_l^T) W + dwconv65(V).
+// CTA (64 query rows, bh). Scores for all m landmarks stay in shared memory,
+// so the row softmax is exact (no online rescaling).
+template <typename T, int D>
+struct OutSmem {
+    static constexpr size_t bytes(int m) {
+        return sizeof(float) * ((size_t)D * 68 * 2 + (size_t)64 * (m + 1) + (size_t)128 * (D + 4) + 72);
+    }
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+output_simt_kernel(const T* __restrict__ q, const float* __restrict__ kl, const float* __restrict__ w,
+                   const T* __restrict__ v, const float* __restrict__ conv_w, T* __restrict__ out,
+                   int H, int n, int m) {
+    constexpr int CW = D / 16;
+    extern __shared__ float smem[];
+    float (*sQ)[68] = reinterpret_cast<float (*)[68]>(smem);              // [D][68]
+    float (*sB)[68] = reinterpret_cast<float (*)[68]>(smem + D * 68);     // [D][68] K_l chunk / W chunk
+    float* sS = smem + 2 * D * 68;                                        // [64][m+1]
+    float (*sV)[D + 4] = reinterpret_cast<float (*)[D + 4]>(sS + 64 * (m + 1));  // [128][D+4]
+    float* sw = reinterpret_cast<float*>(sV + 128);                       // [65]
+    const int ldS = m + 1;
+    const int bh = blockIdx.x, tile = blockIdx.y, h = bh % H;
+    const int i0 = tile * 64;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4, lane = tid & 31, warp = tid >> 5;
+    const float s = split_scale(D);
+    const T* qb = q + (size_t)bh * n * D;
+    for (int e = tid; e < 64 * D; e += 256) {
+        int r = e / D, c = e % D;
+        sQ[c][r] = (i0 + r < n) ? s * Elt<T>::to_f(qb[(size_t)(i0 + r) * D + c]) : 0.f;
+    }
+    const float* klb = kl + (size_t)bh * m * D;
+    for (int j0 = 0; j0 < m; j0 += 64) {
+        __syncthreads();
+        for (int e = tid; e < 64 * D; e += 256) {
+            int r = e / D, c = e % D;
+            sB[c][r] = (j0 + r < m) ? klb[(size_t)(j0 + r) * D + c] : 0.f;
+        }
+        __syncthreads();
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < D; ++e) {
+            float4 av = *reinterpret_cast<const float4*>(&sQ[e][ty * 4]);
+            float4 bv = *reinterpret_cast<const float4*>(&sB[e][tx * 4]);
+            float a4[4] = {av.x, av.y, av.z, av.w};
+            float b4[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a4[i], b4[j], acc[i][j]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                int c = j0 + tx * 4 + j;
+                if (c < m) sS[(ty * 4 + i) * ldS + c] = acc[i][j];
+            }
+    }
+    __syncthreads();
+    for (int r = warp; r < 64; r += 8) {
+        float* row = sS + r * ldS;
+        float mx = -INFINITY;
+        for (int c = lane; c < m; c += 32) mx = fmaxf(mx, row[c]);
+        mx = warp_max(mx);
+        float sum = 0.f;
+        for (int c = lane; c < m; c += 32) {
+            float e = __expf(row[c] - mx);
+            row[c] = e;
+            sum += e;
+        }
+        sum = warp_sum(sum);
+        const float inv = 1.f / sum;
+        for (int c = lane; c < m; c += 32) row[c] *= inv;
+    }
+    float o[4][CW];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < CW; ++j) o[i][j] = 0.f;
+    const float* wb = w + (size_t)bh * m * D;
+    for (int j0 = 0; j0 < m; j0 += 64) {
+        __syncthreads();
+        for (int e = tid; e < 64 * D; e += 256) {
+            int r = e / D, c = e % D;
+            sB[0][r * D + c] = (j0 + r < m) ? wb[(size_t)(j0 + r) * D + c] : 0.f;  // [64][D] row-major
+        }
+        __syncthreads();
+        const float* sW = &sB[0][0];
+        const int jn = min(64, m - j0);
+        for (int kk = 0; kk < jn; ++kk) {
+            float pv[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) pv[i] = sS[(ty * 4 + i) * ldS + j0 + kk];
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+                float wv = sW[kk * D + tx * CW + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[i][j] = fmaf(pv[i], wv, o[i][j]);
+            }
+        }
+    }
+    if (conv_w != nullptr) {
+        const T* vb = v + (size_t)bh * n * D;
+        for (int e = tid; e < 128 * D; e += 256) {
+            int r = e / D, c = e % D;
+            int src = i0 - kHalfTaps + r;
+            sV[r][c] = (src >= 0 && src < n) ? Elt<T>::to_f(vb[(size_t)src * D + c]) : 0.f;
+        }
+        if (tid < kTaps) sw[tid] = conv_w[(size_t)h * kTaps + tid];
+        __syncthreads();
+        for (int t = 0; t < kTaps; ++t) {
+            const float wt = sw[t];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < CW; ++j) o[i][j] = fmaf(wt, sV[ty * 4 + i + t][tx * CW + j], o[i][j]);
+        }
+    }
+    T* ob = out + (size_t)bh * n * D;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        int r = i0 + ty * 4 + i;
+        if (r >= n) continue;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) ob[(size_t)r * D + tx * CW + j] = Elt<T>::from_f(o[i][j]);
+    }
+}
+
+}  // namespace nys

@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI library (no GPU needed).
+
+The shared library must build for sm_100a, load, export every function that
+include/nys_attn.h declares, and reject bad arguments before touching the
+device. No compute call is made here.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include"))
+           if f.endswith(".h")]
+
+
+def _declared():
+    names = set()
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for mt in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(nys_\w+)\s*\(", text, re.M):
+            names.add(mt.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import nystr_self_attention_scale_b200 as nys
+    return nys.lib
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for required in ("nys_attn_forward", "nys_attn_forward_host", "nys_attn_forward_debug",
+                     "nys_strerror", "nys_attn_device_status"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    import nystr_self_attention_scale_b200 as nys
+    out = subprocess.run(["nm", "-D", "--defined-only", nys.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    missing = [n for n in _declared() if n not in exported]
+    assert not missing, missing
+    for n in _declared():
+        getattr(lib, n)
+
+
+def test_library_is_sm100a():
+    import nystr_self_attention_scale_b200 as nys
+    log = open(os.path.join(os.path.dirname(nys.LIB_PATH), "build.log")).read()
+    assert "arch=compute_100a,code=sm_100a" in log
+
+
+def test_strerror_texts(lib):
+    import nystr_self_attention_scale_b200 as nys
+    assert nys.strerror(0) == "ok"
+    assert "invalid" in nys.strerror(-1)
+    assert "unsupported" in nys.strerror(-2)
+    assert nys.strerror(12345) == "unknown status"
+
+
+def _call(lib, B=1, H=1, n=512, d=64, m=64, n_iter=6, dtype=0, null=False):
+    p = None if null else ctypes.c_void_p(16)  # never dereferenced: checks fail first
+    return lib.nys_attn_forward(p, p, p, None, None, B, H, n, d, m, n_iter, dtype, p, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(null=True), -1),
+    (dict(B=0), -1), (dict(H=-1), -1), (dict(n=0), -1), (dict(d=0), -1), (dict(m=0), -1),
+    (dict(n=500, m=64), -1),          # n % m != 0
+    (dict(n=64, m=128), -1),          # m > n
+    (dict(n_iter=-1), -1),
+    (dict(d=48), -2), (dict(d=128), -2),
+    (dict(m=512, n=1024), -2),
+    (dict(dtype=7), -2),
+    (dict(dtype=1, m=32), -2),        # bf16 tensor path: m in {64, 128, 256}
+    (dict(dtype=1, n=192, m=64), -2), # bf16 tensor path: n % 128 == 0
+])
+def test_rejects_before_launch(lib, kw, code):
+    assert _call(lib, **kw) == code
+
+
+def test_host_entry_validates_too(lib):
+    p = ctypes.c_void_p(16)
+    assert lib.nys_attn_forward_host(p, p, p, None, None, 1, 1, 100, 64, 64, 6, 0, p, None) == -1
+
+
+def test_workspace_bytes(lib):
+    import nystr_self_attention_scale_b200 as nys
+    assert nys.workspace_bytes(1, 1, 100, 64, 64) == 0
+    small = nys.workspace_bytes(1, 1, 512, 64, 64, 0)
+    big = nys.workspace_bytes(4, 8, 16384, 64, 256)
+    assert 0 < small < big
+
+
+def test_defaults_match_the_pages():
+    """Defaults printed by the pages (see tests/golden/config_defaults.txt)."""
+    import nystr_self_attention_scale_b200 as nys
+    rows = {}
+    for line in open(os.path.join(ROOT, "tests", "golden", "config_defaults.txt")):
+        line = line.split("#", 1)[0].strip()
+        if line:
+            key, val = line.split("=", 1)
+            rows[key.strip()] = val.strip()
+    assert int(rows["num_landmarks"]) == nys.DEFAULT_NUM_LANDMARKS
+    assert int(rows["conv_kernel_size"]) == nys.CONV_TAPS
+    assert int(rows["iterative_inv_n_iter"]) == nys.DEFAULT_N_ITER
+    hdr = open(os.path.join(ROOT, "include", "nys_attn.h")).read()
+    assert f"#define NYS_CONV_TAPS {rows['conv_kernel_size']}" in hdr
+    assert f"#define NYS_DEFAULT_N_ITER {rows['iterative_inv_n_iter']}" in hdr

@@ -1,0 +1,259 @@
+"""GPU parity: the CUDA path against the fp64 oracle on the same seeded inputs.
+
+Every call goes through the C ABI (via the thin ctypes binding). Full-size
+workloads run on the GPU exactly as the benchmark launches them; the oracle
+then recomputes a sample of heads and query rows (the sampled rows of the
+oracle are exact, not approximations: every output row depends on the whole
+head, which the oracle processes in full).
+"""
+import numpy as np
+import pytest
+
+from parity import assert_close, errors, gpu_forward, oracle_heads, sample_rows
+from workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def nys():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import nystr_self_attention_scale_b200 as nys_mod
+    return nys_mod
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _status_clean(nys):
+    yield
+    assert nys.device_status() == 0
+
+
+def _full_check(nys, oracle_mod, x, what):
+    out = gpu_forward(x, nys, torch)
+    ref = oracle_mod.forward(x["q"], x["k"], x["v"], x["mask"], x["conv_w"], m=x["m"],
+                             n_iter=x["n_iter"])
+    return assert_close(out.double().cpu().numpy(), ref, x["dtype"], what)
+
+
+def _sampled_check(nys, oracle_mod, x, heads, rows, what):
+    out = gpu_forward(x, nys, torch)
+    got = np.stack([out[b, h, rows].double().cpu().numpy() for b, h in heads])
+    ref = oracle_heads(x, oracle_mod, heads, rows=rows)
+    return assert_close(got, ref, x["dtype"], what)
+
+
+# ------------------------------------------------------------------ the workloads, full size
+
+def test_tiny_f32(nys, oracle_mod):
+    x = make_inputs(WORKLOADS["tiny_f32"])
+    _full_check(nys, oracle_mod, x, "tiny_f32")
+
+
+def test_default_f32_masked(nys, oracle_mod):
+    x = make_inputs(WORKLOADS["default_f32_masked"])
+    _full_check(nys, oracle_mod, x, "default_f32_masked")
+
+
+def test_longcls_bf16_masked_full_size_sampled(nys, oracle_mod):
+    w = WORKLOADS["longcls_bf16_masked"]
+    x = make_inputs(w)
+    heads = [(0, 0), (5, 1), (17, 0), (31, 1)]
+    rows = sample_rows(w.n, lengths=[x["lengths"][b] for b, _ in heads])
+    _sampled_check(nys, oracle_mod, x, heads, rows, "longcls_bf16_masked")
+
+
+def test_longcls_bf16_masked_small_full(nys, oracle_mod):
+    """Same recipe at B=3, every row compared."""
+    x = make_inputs(WORKLOADS["longcls_bf16_masked"], seed=1, B=3)
+    _full_check(nys, oracle_mod, x, "longcls_bf16_masked B=3")
+
+
+def test_n16384_bf16_corr_full_size_sampled(nys, oracle_mod):
+    w = WORKLOADS["n16384_bf16_corr"]
+    x = make_inputs(w)
+    heads = [(0, 0), (2, 5), (3, 7)]
+    _sampled_check(nys, oracle_mod, x, heads, sample_rows(w.n), "n16384_bf16_corr")
+
+
+def test_n16384_bf16_corr_small_full(nys, oracle_mod):
+    """The correlated-token recipe at n=2048 (m=256, segment length 8), every row compared."""
+    x = make_inputs(WORKLOADS["n16384_bf16_corr"], seed=2, B=1, H=2, n=2048)
+    _full_check(nys, oracle_mod, x, "corr n=2048")
+
+
+@pytest.mark.parametrize("n", [1024, 4096, 16384, 65536])
+@pytest.mark.parametrize("conv", [True, False])
+def test_sweep_full_size_sampled(nys, oracle_mod, n, conv):
+    w = WORKLOADS[f"sweep_n{n}_{'conv' if conv else 'noconv'}"]
+    x = make_inputs(w)
+    heads = [(0, 0), (7, 7)] if n >= 16384 else [(0, 0), (3, 4), (7, 7)]
+    _sampled_check(nys, oracle_mod, x, heads, sample_rows(n), w.name)
+
+
+def test_sweep_n1024_full(nys, oracle_mod):
+    x = make_inputs(WORKLOADS["sweep_n1024_conv"], B=2, H=2)
+    _full_check(nys, oracle_mod, x, "sweep n=1024 B=2 H=2")
+
+
+# ------------------------------------------------------------------ degenerate m = n
+
+def test_degenerate_m_equals_n_24_iterations_is_exact_attention(nys, oracle_mod):
+    w = WORKLOADS["degenerate_f32_it24"]
+    x = make_inputs(w)
+    out = gpu_forward(x, nys, torch).double().cpu().numpy()[0, 0]
+    ref = oracle_mod.forward(x["q"], x["k"], x["v"], None, None, m=256, n_iter=24)[0, 0]
+    assert_close(out, ref, "f32", "m=n, 24 iterations vs oracle")
+    q, k, v = (x[t][0, 0].astype(np.float64) for t in ("q", "k", "v"))
+    s = q @ k.T / 8.0
+    p = np.exp(s - s.max(1, keepdims=True))
+    exact = (p / p.sum(1, keepdims=True)) @ v
+    assert_close(out, exact, "f32", "m=n, 24 iterations vs exact softmax attention")
+
+
+def test_degenerate_m_equals_n_6_iterations(nys, oracle_mod):
+    x = make_inputs(WORKLOADS["degenerate_f32_it6"])
+    _full_check(nys, oracle_mod, x, "m=n, 6 iterations")
+
+
+# ------------------------------------------------------------------ stages and indexing
+
+@pytest.mark.parametrize("dtype,n,m,d", [("f32", 512, 64, 64), ("bf16", 4096, 128, 32),
+                                         ("bf16", 16384, 256, 64), ("f32", 200, 40, 32)])
+def test_landmarks_one_hot_bit_exact(nys, dtype, n, m, d):
+    """A one-hot token t lands in landmark floor(t/L) only, equal to fl32(d^-1/4) / L."""
+    L = n // m
+    tokens = [0, L - 1, L, n // 2 + 1, n - 1]
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    q = torch.zeros(1, len(tokens), n, d, dtype=dt)
+    for h, t in enumerate(tokens):
+        q[0, h, t, (3 * h) % d] = 1.0
+    q = q.cuda()
+    _, st = nys.forward_debug(q, q, q, m=m)
+    s32 = np.float32(d ** -0.25)
+    for name in ("q_l", "k_l"):
+        got = st[name].cpu().numpy()
+        for h, t in enumerate(tokens):
+            nz = np.argwhere(got[0, h] != 0).tolist()
+            assert nz == [[t // L, (3 * h) % d]], (name, t, nz)
+            assert got[0, h, t // L, (3 * h) % d] == np.float32(s32 / np.float32(L))
+
+
+def test_landmarks_ramp_within_one_ulp(nys):
+    n, m, d = 512, 64, 64
+    i = torch.arange(n, dtype=torch.float64)[:, None]
+    c = torch.arange(d, dtype=torch.float64)[None, :]
+    q = (i + 1000 * c).float()[None, None].cuda()
+    _, st = nys.forward_debug(q, q, q, m=m)
+    L = n // m
+    j = np.arange(m)[:, None]
+    expect = (j * L + (L - 1) / 2.0 + 1000.0 * np.arange(d)[None, :]) * d ** -0.25
+    got = st["q_l"][0, 0].cpu().numpy().astype(np.float64)
+    ulp = np.spacing(np.abs(expect).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(got - expect) <= 2 * ulp)
+
+
+@pytest.mark.parametrize("name", ["default_f32_masked", "longcls_bf16_masked", "n16384_bf16_corr"])
+def test_stages_against_oracle(nys, oracle_mod, name):
+    w = WORKLOADS[name]
+    x = make_inputs(w, seed=3, B=2, H=1, n=min(w.n, 4096))
+    _, st = gpu_forward(x, nys, torch, debug=True)
+    heads = [(0, 0), (1, 0)]
+    _, ost = oracle_heads(x, oracle_mod, heads, rows=[0], stages=True)
+    for idx, (b, h) in enumerate(heads):
+        for g, o in (("q_l", "ql"), ("k_l", "kl")):
+            _, rel = errors(st[g][b, h], ost[idx][o])
+            assert rel < 1e-6, (g, rel)
+        _, rel = errors(st["k3v"][b, h], ost[idx]["k3v"])
+        assert rel < (1e-5 if w.dtype == "f32" else 2e-2), ("k3v", rel)
+        _, rel = errors(st["z"][b, h], ost[idx]["z"])
+        assert rel < (1e-4 if w.dtype == "f32" else 2e-2), ("z", rel)
+
+
+def test_mask_padded_keys_do_not_contribute(nys):
+    """Changing K and V at padded keys, with the segment sums of K kept (a zero-sum
+    perturbation), leaves kernel_3 V unchanged up to the landmark rounding."""
+    x = make_inputs(WORKLOADS["default_f32_masked"], seed=4, B=2, H=2)
+    _, st1 = gpu_forward(x, nys, torch, debug=True)
+    k2, v2 = x["k"].copy(), x["v"].copy()
+    L = x["n"] // x["m"]
+    rng = np.random.default_rng(40)
+    changed = 0
+    for b in range(2):
+        start = ((int(x["lengths"][b]) + L - 1) // L) * L  # first whole padded segment
+        for s0 in range(start, x["n"], L):
+            pert = rng.standard_normal((2, L, x["d"]))
+            pert -= pert.mean(axis=1, keepdims=True)
+            k2[b, :, s0:s0 + L] += pert.astype(np.float32)
+            v2[b, :, s0:s0 + L] = 7.0
+            changed += 1
+    assert changed > 0
+    x2 = dict(x)
+    x2["k"], x2["v"] = k2, v2
+    _, st2 = gpu_forward(x2, nys, torch, debug=True)
+    np.testing.assert_allclose(st2["k3v"], st1["k3v"], rtol=1e-5, atol=1e-6)
+
+
+# ------------------------------------------------------------------ edge cases
+
+@pytest.mark.parametrize("dtype,B,H,n,d,m", [
+    ("f32", 2, 3, 200, 32, 40),     # ragged: segment length 5, n not a tile multiple
+    ("f32", 1, 2, 96, 64, 96),      # m = n (L = 1), fp32
+    ("f32", 3, 1, 64, 64, 1),       # a single landmark
+    ("bf16", 2, 2, 128, 64, 128),   # m = n on the bf16 path
+    ("bf16", 1, 1, 256, 64, 256),   # m = n = 256 on the bf16 path
+    ("bf16", 1, 3, 384, 32, 64),    # n = 3 tiles of 128
+])
+def test_edge_shapes(nys, oracle_mod, dtype, B, H, n, d, m):
+    w = WORKLOADS["tiny_f32"]
+    import dataclasses
+    w = dataclasses.replace(w, dtype=dtype, d=d, m=m, lengths=(max(1, n // 3), n), zero_pad=True)
+    x = make_inputs(w, seed=5, B=B, H=H, n=n)
+    _full_check(nys, oracle_mod, x, f"edge {dtype} B{B} H{H} n{n} d{d} m{m}")
+
+
+def test_single_valid_key(nys, oracle_mod):
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS["default_f32_masked"], lengths=(1, 1))
+    x = make_inputs(w, seed=6, B=2, H=2, n=512)
+    _full_check(nys, oracle_mod, x, "one valid key per sequence")
+
+
+# ------------------------------------------------------------------ determinism and boundary
+
+def test_deterministic_and_heads_independent(nys):
+    x = make_inputs(WORKLOADS["longcls_bf16_masked"], seed=7, B=4)
+    a = gpu_forward(x, nys, torch)
+    b = gpu_forward(x, nys, torch)
+    assert torch.equal(a, b)
+    one = dict(x)
+    for key in ("q", "k", "v"):
+        one[key] = x[key][2:3, 1:2].copy()
+    one["mask"] = x["mask"][2:3].copy()
+    one["conv_w"] = x["conv_w"][1:2].copy()
+    c = gpu_forward(one, nys, torch)
+    assert torch.equal(c[0, 0], a[2, 1])
+
+
+def test_host_entry_matches_device_entry(nys):
+    x = make_inputs(WORKLOADS["longcls_bf16_masked"], seed=8, B=2)
+    dev = gpu_forward(x, nys, torch).cpu()
+    q = torch.from_numpy(x["q"]).to(torch.bfloat16).pin_memory()
+    k = torch.from_numpy(x["k"]).to(torch.bfloat16).pin_memory()
+    v = torch.from_numpy(x["v"]).to(torch.bfloat16).pin_memory()
+    out = nys.forward_host(q, k, v, mask=torch.from_numpy(x["mask"]),
+                           conv_w=torch.from_numpy(x["conv_w"]), m=x["m"])
+    assert torch.equal(out, dev)
+
+
+def test_invalid_arguments_raise(nys):
+    q = torch.zeros(1, 1, 100, 64, device="cuda")
+    with pytest.raises(nys.NysError) as e:
+        nys.forward(q, q, q, m=64)
+    assert e.value.status == -1
+    q = torch.zeros(1, 1, 128, 48, device="cuda")
+    with pytest.raises(nys.NysError) as e:
+        nys.forward(q, q, q, m=64)
+    assert e.value.status == -2
