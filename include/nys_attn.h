@@ -60,7 +60,8 @@ typedef enum {
     NYS_ERR_UNSUPPORTED = -2,  /* shape or dtype outside what the kernels implement            */
     NYS_ERR_CUDA = -3,         /* a CUDA call failed                                           */
     NYS_ERR_NOMEM = -4,        /* workspace allocation failed                                  */
-    NYS_ERR_TIMEOUT = -5       /* a bounded device-side wait ran out                           */
+    NYS_ERR_TIMEOUT = -5,      /* a bounded device-side wait ran out                           */
+    NYS_ERR_SCRATCH_LIMIT = -6 /* needs more than the fixed static scratch (nys_attn_pinv_static) */
 } nys_status_t;
 
 /*
@@ -111,6 +112,45 @@ int nys_attn_forward_debug(const void* q, const void* k, const void* v, const ui
                            const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
                            int dtype, void* out, float* q_l, float* k_l, float* z, float* k3v,
                            float* w, void* stream);
+
+/*
+ * nys_attn_pinv_static -- kernel_2 and its iterative inverse for a batch of
+ * heads, using no memory allocation at all. (The pages have no counterpart
+ * of this entry point; it exists for callers, not for the method.)
+ *
+ * Who needs it: callers that cannot call cudaMalloc / cudaMallocAsync --
+ * for example a host application that reserves all device memory up front
+ * and forbids any later allocation, or a latency-critical loop that cannot
+ * afford an allocation's cost or its failure. nys_attn_forward takes its
+ * scratch from cudaMallocAsync; this entry point takes it from a fixed 8 MiB
+ * array in the library's device memory instead.
+ *
+ *   q_l, k_l  device float32 [BH, m, d]: landmarks of the scaled Q and K
+ *             (as nys_attn_forward_debug returns them)
+ *   z         device float32 [BH, m, m] output: Z = iterative inverse of
+ *             kernel_2 = softmax_row(Q_l K_l^T), n_iter iterations,
+ *             Z_0 = k2^T / (max column sum * max row sum)
+ *   stream    a cudaStream_t (NULL = legacy default stream)
+ * Supported: d in {32, 64}, 1 <= m <= 256, any BH >= 1 (heads run in
+ * batches that fit the array; one head needs 5 m^2 floats). A head that
+ * would need more than the array returns NYS_ERR_SCRATCH_LIMIT; bad
+ * arguments return NYS_ERR_INVALID_ARG / NYS_ERR_UNSUPPORTED before any
+ * launch. The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine).
+ *
+ * Set-up: the first call on a device (with that device current) looks up
+ * the array's device address once; make that first call before any stream
+ * capture begins. The array is held by every GPU that loads the library
+ * until the process exits.
+ *
+ * Sharing: every call uses the same array, which keeps the previous call's
+ * contents (nothing in it needs to start at zero: each launch writes every
+ * scratch element before reading it). Calls whose work overlaps on the GPU
+ * -- on different streams, or from different host threads -- race on the
+ * array and corrupt each other's results; order them on one stream.
+ */
+int nys_attn_pinv_static(const float* q_l, const float* k_l, float* z, int BH, int m, int d,
+                         int n_iter, void* stream);
 
 /* Synchronises the current device, then returns and clears the device status
  * word (NYS_OK or NYS_ERR_TIMEOUT); NYS_ERR_CUDA if the synchronisation fails. */

@@ -27,7 +27,8 @@ DEFAULT_NUM_LANDMARKS = 64
 
 F32, BF16 = 0, 1
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape or dtype", -3: "CUDA error",
-           -4: "device workspace allocation failed", -5: "bounded device wait timed out"}
+           -4: "device workspace allocation failed", -5: "bounded device wait timed out",
+           -6: "problem exceeds the library's fixed static scratch"}
 
 
 class NysError(RuntimeError):
@@ -60,6 +61,8 @@ def _load() -> ctypes.CDLL:
     lib.nys_attn_kernel_count.restype = i
     lib.nys_attn_kernel_name.argtypes = [i]
     lib.nys_attn_kernel_name.restype = ctypes.c_char_p
+    lib.nys_attn_pinv_static.argtypes = [vp, vp, vp, i, i, i, i, vp]
+    lib.nys_attn_pinv_static.restype = i
     lib.nys_strerror.argtypes = [i]
     lib.nys_strerror.restype = ctypes.c_char_p
     return lib
@@ -199,4 +202,22 @@ def profile_read() -> dict:
         ms = ctypes.c_double(0.0)
         _check(lib.nys_attn_profile_read(kid, ctypes.byref(n), ctypes.byref(ms)), "profile_read")
         out[lib.nys_attn_kernel_name(kid).decode()] = (n.value, ms.value)
+    return out
+
+
+def pinv_static(q_l, k_l, n_iter: int = DEFAULT_N_ITER, out=None, stream=None):
+    """kernel_2 + iterative inverse from float32 landmarks [B, H, m, d] -> Z [B, H, m, m],
+    through the allocation-free entry point (scratch is a fixed array inside the library)."""
+    import torch
+    if q_l.shape != k_l.shape or q_l.dim() != 4 or q_l.dtype != torch.float32 or not q_l.is_cuda:
+        raise ValueError("q_l, k_l must be float32 CUDA tensors of one [B, H, m, d] shape")
+    B, H, m, d = (int(t) for t in q_l.shape)
+    q_l, k_l = q_l.contiguous(), k_l.contiguous()
+    if out is None:
+        out = torch.empty(B, H, m, m, device=q_l.device, dtype=torch.float32)
+    s = stream if stream is not None else torch.cuda.current_stream(q_l.device)
+    with torch.cuda.device(q_l.device):
+        rc = lib.nys_attn_pinv_static(_ptr(q_l), _ptr(k_l), _ptr(out), B * H, m, d, int(n_iter),
+                                      s.cuda_stream)
+    _check(rc, "nys_attn_pinv_static")
     return out

@@ -262,6 +262,35 @@ int run(const void* q, const void* k, const void* v, const uint8_t* mask, const 
     return rc;
 }
 
+// ---------------------------------------------------------------- allocation-free inverse
+// Scratch of nys_attn_pinv_static(): a fixed 8 MiB array in device memory.
+// Each head of the iterative inverse needs 5 m x m float32 matrices; heads
+// are processed in batches that fit. Every GPU that loads this library holds
+// the array until the process exits. In host code the name below is only a
+// host-side stand-in: its device address comes from cudaGetSymbolAddress().
+constexpr size_t kStaticScratchFloats = (8u << 20) / sizeof(float);
+static __device__ __align__(256) float g_static_scratch[kStaticScratchFloats];
+
+std::mutex g_static_mu;
+float* g_static_ptr[kMaxDevices];   // device address of g_static_scratch, per device
+
+// Once per device, with that device current: look up the array's address.
+int static_scratch(float** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NYS_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
+            cudaGetLastError();
+            return NYS_ERR_CUDA;
+        }
+        g_static_ptr[dev] = static_cast<float*>(p);
+    }
+    *out = g_static_ptr[dev];
+    return NYS_OK;
+}
+
 }  // namespace
 }  // namespace nys
 
@@ -343,11 +372,32 @@ const char* nys_strerror(int status) {
         case NYS_ERR_CUDA: return "CUDA error";
         case NYS_ERR_NOMEM: return "device workspace allocation failed";
         case NYS_ERR_TIMEOUT: return "bounded device wait timed out";
+        case NYS_ERR_SCRATCH_LIMIT: return "problem exceeds the library's fixed static scratch";
         default: return "unknown status";
     }
 }
 
 int nys_attn_version(void) { return 100; }
+
+int nys_attn_pinv_static(const float* q_l, const float* k_l, float* z, int BH, int m, int d,
+                         int n_iter, void* stream) {
+    if (!q_l || !k_l || !z) return NYS_ERR_INVALID_ARG;
+    if (BH <= 0 || m <= 0 || d <= 0 || n_iter < 0) return NYS_ERR_INVALID_ARG;
+    if ((d != 32 && d != 64) || m > 256) return NYS_ERR_UNSUPPORTED;
+    const size_t per_head = (size_t)5 * m * m;   // k2, X, T, U and the second Z buffer
+    if (per_head > nys::kStaticScratchFloats) return NYS_ERR_SCRATCH_LIMIT;
+    float* scratch = nullptr;
+    int rc = nys::static_scratch(&scratch);
+    if (rc != NYS_OK) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int per_launch = (int)(nys::kStaticScratchFloats / per_head);
+    for (int h0 = 0; h0 < BH; h0 += per_launch) {
+        const int nh = BH - h0 < per_launch ? BH - h0 : per_launch;
+        const size_t md = (size_t)h0 * m * d, mm = (size_t)h0 * m * m;
+        nys::pinv_simt_kernel<<<nh, 256, 0, s>>>(q_l + md, k_l + md, z + mm, scratch, m, d, n_iter);
+    }
+    return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
 
 int nys_attn_profile_enable(int on) {
     nys::prof_drain();
