@@ -17,6 +17,8 @@
 #include "common.cuh"
 #include "landmarks.cuh"
 #include "simt.cuh"
+#include "tc_k3v.cuh"
+#include "tc_output.cuh"
 
 namespace nys {
 namespace {
@@ -54,12 +56,8 @@ int device_state(DeviceState** out) {
         const size_t big = 200 * 1024;
         cudaFuncSetAttribute(k3v_partial_simt_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
         cudaFuncSetAttribute(k3v_partial_simt_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
-        cudaFuncSetAttribute(k3v_partial_simt_kernel<__nv_bfloat16, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
-        cudaFuncSetAttribute(k3v_partial_simt_kernel<__nv_bfloat16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
         cudaFuncSetAttribute(output_simt_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
         cudaFuncSetAttribute(output_simt_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
-        cudaFuncSetAttribute(output_simt_kernel<__nv_bfloat16, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
-        cudaFuncSetAttribute(output_simt_kernel<__nv_bfloat16, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
         if (cudaGetLastError() != cudaSuccess) return NYS_ERR_CUDA;
         st.ready = true;
     }
@@ -69,12 +67,65 @@ int device_state(DeviceState** out) {
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
 
+// [B, n] uint8 key mask -> [B, n / 32] validity bits (bit i of word w = key 32 w + i).
+__global__ void mask_bits_kernel(const uint8_t* __restrict__ mask, uint32_t* __restrict__ bits, int B, int n) {
+    const int words = n / 32;
+    const int w = blockIdx.x * blockDim.x + threadIdx.x;
+    if (w >= B * words) return;
+    const int b = w / words, wi = w % words;
+    const uint4* src = reinterpret_cast<const uint4*>(mask + (size_t)b * n + (size_t)wi * 32);
+    uint32_t v = 0;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const uint4 u = src[q];
+        const uint32_t x[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            v |= (((x[e >> 2] >> ((e & 3) * 8)) & 0xFFu) != 0u ? 1u : 0u) << (q * 16 + e);
+    }
+    bits[w] = v;
+}
+
+// ---------------------------------------------------------------- TMA tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// 3-D bf16 tensor map over a row-major [d2][d1][d0] array, box b0 x b1 x 1,
+// out-of-bounds elements read as zero.
+bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
+                 uint32_t b1, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    const cuuint32_t box[3] = {b0, b1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- per-kernel timing
 // When enabled, every launch is bracketed by two CUDA events on the stream it
 // runs on; nys_attn_profile_read() sums their elapsed times per kernel.
-enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_COUNT };
+enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_MASKBITS, K_COUNT };
 const char* const kKernelNames[K_COUNT] = {"landmarks", "pinv", "k3v_partial", "k3v_combine",
-                                           "w_product", "output"};
+                                           "w_product", "output", "mask_bits"};
 
 struct ProfRecord { int kid; cudaEvent_t a, b; };
 std::mutex g_prof_mu;
@@ -120,7 +171,8 @@ struct Plan {
     int B, H, n, d, m, n_iter, dtype;
     int BH, splits, keys_per_split;
     size_t off_ql, off_kl, off_ql16, off_kl16, off_k3v, off_w, off_wt16, off_z, off_pinv;
-    size_t off_po, off_pm, off_pl, total;
+    size_t off_po, off_pm, off_pl, off_mbits, total;
+    int tc_cps, tc_splits;  // tensor-core kernel_3 V: 128-key chunks per split, splits
 };
 
 int validate(const void* q, const void* k, const void* v, const void* out, int B, int H, int n,
@@ -144,8 +196,15 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
     // The key split depends on n only (never on B*H or the GPU), so a head's
     // result is bitwise the same alone or inside any batch.
     (void)sm_count;
-    const int kps = std::min(((n + 63) / 64) * 64, 1024);
-    const int splits = (n + kps - 1) / kps;
+    int kps = std::min(((n + 63) / 64) * 64, 1024);
+    int splits = (n + kps - 1) / kps;
+    if (dtype == NYS_BF16) {
+        const int chunks = n / 128;
+        p.tc_cps = std::min(chunks, n >= 16384 ? 16 : 8);
+        p.tc_splits = (chunks + p.tc_cps - 1) / p.tc_cps;
+        splits = p.tc_splits;
+        kps = p.tc_cps * 128;
+    }
     p.splits = splits;
     p.keys_per_split = kps;
     const size_t BH = p.BH, md = (size_t)m * d, mm = (size_t)m * m;
@@ -163,12 +222,13 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
     p.off_po = take(BH * splits * md * 4);
     p.off_pm = take(BH * splits * (size_t)m * 4);
     p.off_pl = take(BH * splits * (size_t)m * 4);
+    p.off_mbits = take((size_t)B * ((n + 31) / 32) * 4);
     p.total = o;
     return p;
 }
 
 template <typename T, int D>
-int launch_all(const Plan& p, const DeviceState& st, const T* q, const T* k, const T* v,
+int launch_simt(const Plan& p, const DeviceState& st, const T* q, const T* k, const T* v,
                const uint8_t* mask, const float* conv_w, T* out, char* ws, cudaStream_t s) {
     float* ql = reinterpret_cast<float*>(ws + p.off_ql);
     float* kl = reinterpret_cast<float*>(ws + p.off_kl);
@@ -220,6 +280,122 @@ int launch_all(const Plan& p, const DeviceState& st, const T* q, const T* k, con
     return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
 }
 
+template <int D, int M>
+int launch_output_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, const __nv_bfloat16* v,
+                     const float* conv_w, __nv_bfloat16* out, const __nv_bfloat16* kl16,
+                     const __nv_bfloat16* wt16, cudaStream_t s) {
+    using C = OutTc<D, M>;
+    CUtensorMap mq, mv, mo, mkl, mwt;
+    const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const uint64_t BH = p.BH, n = p.n;
+    if (!map_bf16_3d(&mq, q, D, n, BH, D, 128, sw) || !map_bf16_3d(&mv, v, D, n, BH, D, 192, sw) ||
+        !map_bf16_3d(&mo, out, D, n, BH, D, 128, sw) || !map_bf16_3d(&mkl, kl16, D, M, BH, D, M, sw) ||
+        !map_bf16_3d(&mwt, wt16, M, D, BH, 64, D, CU_TENSOR_MAP_SWIZZLE_128B))
+        return NYS_ERR_CUDA;
+    OutTcParams prm{conv_w, p.H, p.n, p.n / 128, p.BH * (p.n / 128)};
+    const int grid = std::min(prm.total_tiles, st.sm_count);
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(output_tc_kernel<D, M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess)
+            return NYS_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    ProfScope ps(K_OUTPUT, s);
+    output_tc_kernel<D, M><<<grid, 384, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
+    return NYS_OK;
+}
+
+template <int D>
+int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql16, const __nv_bfloat16* k,
+                  const __nv_bfloat16* v, const uint32_t* mbits, float* po, float* pm, float* pl, cudaStream_t s) {
+    using C = K3vTc<D>;
+    CUtensorMap mql, mk, mv;
+    const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const uint64_t BH = p.BH, n = p.n, m = p.m;
+    if (!map_bf16_3d(&mql, ql16, D, m, BH, D, 128, sw) || !map_bf16_3d(&mk, k, D, n, BH, D, 128, sw) ||
+        !map_bf16_3d(&mv, v, D, n, BH, D, 128, sw))
+        return NYS_ERR_CUDA;
+    const int halves = (p.m + 127) / 128;
+    K3vTcParams prm{mbits, po, pm, pl, p.H, p.n, p.m, halves, p.tc_splits, p.tc_cps,
+                    p.BH * halves * p.tc_splits};
+    const int grid = std::min(prm.total_items, st.sm_count);
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(k3v_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess)
+            return NYS_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    ProfScope ps(K_K3V, s);
+    k3v_tc_kernel<D><<<grid, 256, C::kSmemBytes, s>>>(mql, mk, mv, prm);
+    return NYS_OK;
+}
+
+template <int D>
+int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                const __nv_bfloat16* v, const uint8_t* mask, const float* conv_w, __nv_bfloat16* out, char* ws,
+                cudaStream_t s) {
+    using bf = __nv_bfloat16;
+    float* ql = reinterpret_cast<float*>(ws + p.off_ql);
+    float* kl = reinterpret_cast<float*>(ws + p.off_kl);
+    bf* ql16 = reinterpret_cast<bf*>(ws + p.off_ql16);
+    bf* kl16 = reinterpret_cast<bf*>(ws + p.off_kl16);
+    float* k3v = reinterpret_cast<float*>(ws + p.off_k3v);
+    float* w = reinterpret_cast<float*>(ws + p.off_w);
+    bf* wt16 = reinterpret_cast<bf*>(ws + p.off_wt16);
+    float* z = reinterpret_cast<float*>(ws + p.off_z);
+    float* pinv = reinterpret_cast<float*>(ws + p.off_pinv);
+    float* po = reinterpret_cast<float*>(ws + p.off_po);
+    float* pm = reinterpret_cast<float*>(ws + p.off_pm);
+    float* pl = reinterpret_cast<float*>(ws + p.off_pl);
+    uint32_t* mbits = mask ? reinterpret_cast<uint32_t*>(ws + p.off_mbits) : nullptr;
+    const int BH = p.BH, n = p.n, m = p.m;
+    int rc = NYS_OK;
+    {
+        long long threads = (long long)BH * m * (D / 8);
+        dim3 grid((unsigned)((threads + 255) / 256), 2);
+        ProfScope ps(K_LANDMARKS, s);
+        landmarks_kernel<bf><<<grid, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, D, m);
+    }
+    if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
+    if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
+    {
+        ProfScope ps(K_PINV, st.aux);
+        pinv_simt_kernel<<<BH, 256, 0, st.aux>>>(ql, kl, z, pinv, m, D, p.n_iter);
+    }
+    if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
+    if (mask) {
+        const int words = p.B * (n / 32);
+        ProfScope ps(K_MASKBITS, s);
+        mask_bits_kernel<<<(words + 255) / 256, 256, 0, s>>>(mask, mbits, p.B, n);
+    }
+    rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, s);
+    if (rc != NYS_OK) return rc;
+    {
+        dim3 g2(BH, std::max(1, (m * D) / 1024));
+        ProfScope ps(K_COMBINE, s);
+        k3v_combine_kernel<<<g2, 256, 0, s>>>(po, pm, pl, k3v, m, D, p.splits);
+    }
+    if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;
+    {
+        ProfScope ps(K_W, s);
+        w_kernel<<<dim3(BH, (m + 31) / 32), 256, 0, s>>>(z, k3v, w, wt16, m, D);
+    }
+    switch (m) {
+        case 64: rc = launch_output_tc<D, 64>(p, st, q, v, conv_w, out, kl16, wt16, s); break;
+        case 128: rc = launch_output_tc<D, 128>(p, st, q, v, conv_w, out, kl16, wt16, s); break;
+        case 256: rc = launch_output_tc<D, 256>(p, st, q, v, conv_w, out, kl16, wt16, s); break;
+        default: return NYS_ERR_UNSUPPORTED;
+    }
+    if (rc != NYS_OK) return rc;
+    return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
+
 int run(const void* q, const void* k, const void* v, const uint8_t* mask, const float* conv_w,
         int B, int H, int n, int d, int m, int n_iter, int dtype, void* out, float* dbg_ql,
         float* dbg_kl, float* dbg_z, float* dbg_k3v, float* dbg_w, cudaStream_t s) {
@@ -237,16 +413,16 @@ int run(const void* q, const void* k, const void* v, const uint8_t* mask, const 
     char* w = static_cast<char*>(ws);
     std::unique_lock<std::mutex> launch_lock(st->launch_mu);
     if (dtype == NYS_F32) {
-        rc = d == 64 ? launch_all<float, 64>(p, *st, (const float*)q, (const float*)k, (const float*)v,
-                                             mask, conv_w, (float*)out, w, s)
-                     : launch_all<float, 32>(p, *st, (const float*)q, (const float*)k, (const float*)v,
-                                             mask, conv_w, (float*)out, w, s);
+        rc = d == 64 ? launch_simt<float, 64>(p, *st, (const float*)q, (const float*)k, (const float*)v,
+                                              mask, conv_w, (float*)out, w, s)
+                     : launch_simt<float, 32>(p, *st, (const float*)q, (const float*)k, (const float*)v,
+                                              mask, conv_w, (float*)out, w, s);
     } else {
         using bf = __nv_bfloat16;
-        rc = d == 64 ? launch_all<bf, 64>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask,
-                                          conv_w, (bf*)out, w, s)
-                     : launch_all<bf, 32>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask,
-                                          conv_w, (bf*)out, w, s);
+        rc = d == 64 ? launch_bf16<64>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask, conv_w,
+                                       (bf*)out, w, s)
+                     : launch_bf16<32>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask, conv_w,
+                                       (bf*)out, w, s);
     }
     if (rc == NYS_OK) {
         const size_t BH = p.BH, md = (size_t)m * d, mm = (size_t)m * m;

@@ -1,0 +1,375 @@
+// tc_output.cuh -- bf16 output pass on the 5th-generation tensor cores.
+//
+// Walkthrough (blog.gitcode.com) 2.4 and 2.6:
+//   out = softmax_row(Qs K_l^T) W + dwconv65(V),   W = Z (kernel_3 V)
+// per 128-query tile of one (batch, head):
+//   S      = Q_tile . K_l^T          tcgen05 bf16 MMA, fp32 accumulator in TMEM
+//   P      = exp(s (S - rowmax))     thread-per-row softmax read from TMEM, bf16 P
+//                                    written back into the S columns of TMEM
+//   O_att  = P . W                   MMA with A = P straight from TMEM
+//   O_conv = T . V_halo              the 65-tap conv as a 128 x 192 banded Toeplitz
+//                                    matrix T (built once per head) times the 192
+//                                    V rows around the tile (zero outside [0, n),
+//                                    supplied by the TMA out-of-bounds fill)
+//   out    = O_att / rowsum(P) + O_conv, bf16, TMA store
+//
+// Warp roles (384 threads, one persistent CTA per SM over a contiguous range of
+// tiles): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM allocator,
+// warps 4-7 softmax, warps 8-11 epilogue (and the Toeplitz build).
+// Two TMEM slots alternate between consecutive tiles so the softmax of one
+// tile overlaps the MMAs and the epilogue of the other. Every wait is bounded.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace nys {
+
+template <int D, int M>
+struct OutTc {
+    static constexpr int kRows = 128;
+    static constexpr int kHalo = 192;                 // 32 + 128 + 32 V rows per tile
+    static constexpr int kSpan = D * 2;               // row pitch of Q/V/out tiles (bytes)
+    static constexpr uint32_t kLayout = D == 64 ? sm100::kLayoutSw128 : sm100::kLayoutSw64;
+    static constexpr uint32_t kSbo = 8 * kSpan;       // 8-row group stride
+    static constexpr int kStages = 2;
+    static constexpr uint32_t kQBytes = kRows * kSpan;
+    static constexpr uint32_t kVBytes = kHalo * kSpan;
+    static constexpr uint32_t kKlBytes = M * kSpan;
+    static constexpr uint32_t kWtBlock = D * 128;     // [D][64] bf16 K-block of W^T
+    static constexpr uint32_t kWtBytes = (M / 64) * kWtBlock;
+    static constexpr uint32_t kTBlock = 128 * 128;    // [128][64] bf16 K-block of T
+    static constexpr uint32_t kTBytes = 3 * kTBlock;
+    static constexpr uint32_t kOutBytes = kRows * kSpan;
+    static constexpr int kSlotNeed = (M > M / 2 + 2 * D) ? M : (M / 2 + 2 * D);
+    static constexpr int kSlot = kSlotNeed <= 64 ? 64 : (kSlotNeed <= 128 ? 128 : 256);
+    static constexpr int kTmemCols = 2 * kSlot;
+    static constexpr int kColP = 0, kColOatt = M / 2, kColOconv = M / 2 + D;
+    static constexpr uint32_t kOffQ = 0;
+    static constexpr uint32_t kOffV = kOffQ + kStages * kQBytes;
+    static constexpr uint32_t kOffKl = kOffV + kStages * kVBytes;
+    static constexpr uint32_t kOffWt = kOffKl + kKlBytes;
+    static constexpr uint32_t kOffT = kOffWt + kWtBytes;
+    static constexpr uint32_t kOffOut = kOffT + kTBytes;
+    static constexpr uint32_t kOffLinv = kOffOut + kOutBytes;   // [2][128] float
+    static constexpr uint32_t kOffBar = kOffLinv + 2 * 128 * 4;
+    static constexpr int kNumBars = 16;
+    static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
+    static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    static_assert(kSmemBytes <= 232448, "shared memory budget");
+    static_assert(kTmemCols <= 512, "TMEM budget");
+    static constexpr uint32_t kIdS = sm100::make_idesc(128, M, sm100::kFmtBf16, sm100::kFmtBf16, 0, 0);
+    static constexpr uint32_t kIdPW = sm100::make_idesc(128, D, sm100::kFmtBf16, sm100::kFmtBf16, 0, 0);
+    static constexpr uint32_t kIdConv = sm100::make_idesc(128, D, sm100::kFmtBf16, sm100::kFmtBf16, 0, 1);
+};
+
+struct OutTcParams {
+    const float* conv_w;   // [H, 65] or null
+    int H, n, tiles_per_head, total_tiles;
+};
+
+template <int D, int M>
+__global__ void __launch_bounds__(384, 1)
+output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
+                 const __grid_constant__ CUtensorMap map_out, const __grid_constant__ CUtensorMap map_kl,
+                 const __grid_constant__ CUtensorMap map_wt, const OutTcParams prm) {
+    using C = OutTc<D, M>;
+    using namespace sm100;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
+    uint64_t* q_full = bars + 0;     // [2] TMA Q+V landed
+    uint64_t* q_empty = bars + 2;    // [2] stage reusable
+    uint64_t* s_full = bars + 4;     // [2] S in TMEM
+    uint64_t* p_full = bars + 6;     // [2] P in TMEM, S fully read (128 arrivals)
+    uint64_t* o_full = bars + 8;     // [2] O_att, O_conv ready
+    uint64_t* slot_free = bars + 10; // [2] epilogue done with the slot (128 arrivals)
+    uint64_t* const_full = bars + 12;
+    uint64_t* const_empty = bars + 13;
+    uint64_t* mma_done = bars + 14;
+    uint64_t* t_full = bars + 15;    // Toeplitz matrix built (128 arrivals)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
+    float* linv = reinterpret_cast<float*>(sm + C::kOffLinv);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // contiguous tile range of this CTA
+    const int per = prm.total_tiles / gridDim.x, extra = prm.total_tiles % gridDim.x;
+    const int t0 = blockIdx.x * per + min((int)blockIdx.x, extra);
+    const int count = per + ((int)blockIdx.x < extra ? 1 : 0);
+    const int tph = prm.tiles_per_head;
+    auto head_start = [&](int i) { return i == 0 || ((t0 + i) % tph) == 0; };
+
+    if (threadIdx.x == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&q_full[b], 1);
+            mbar_init(&q_empty[b], 1);
+            mbar_init(&s_full[b], 1);
+            mbar_init(&p_full[b], 128);
+            mbar_init(&o_full[b], 1);
+            mbar_init(&slot_free[b], 128);
+        }
+        mbar_init(const_full, 1);
+        mbar_init(t_full, 128);
+        mbar_init(const_empty, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&map_q);
+        prefetch_tmap(&map_v);
+        prefetch_tmap(&map_out);
+        prefetch_tmap(&map_kl);
+        prefetch_tmap(&map_wt);
+    }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t ce_phase = 0;
+            int last_use[2] = {-1, -1};
+            int const_loads = 0;
+            for (int i = 0; i < count && !*abort_flag; ++i) {
+                const int t = t0 + i, bh = t / tph, row0 = (t % tph) * C::kRows;
+                if (head_start(i)) {
+                    if (i > 0) {
+                        if (!mbar_wait(const_empty, ce_phase)) { *abort_flag = 1; break; }
+                        ce_phase ^= 1;
+                    }
+                    mbar_arrive_expect_tx(const_full, C::kKlBytes + C::kWtBytes);
+                    tma_load_3d(sm + C::kOffKl, &map_kl, const_full, 0, 0, bh);
+                    for (int kb = 0; kb < M / 64; ++kb)
+                        tma_load_3d(sm + C::kOffWt + kb * C::kWtBlock, &map_wt, const_full, kb * 64, 0, bh);
+                    ++const_loads;
+                }
+                const int st = i % C::kStages, use = i / C::kStages;
+                if (!mbar_wait(&q_empty[st], (use & 1) ^ 1)) { *abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&q_full[st], C::kQBytes + C::kVBytes);
+                tma_load_3d(sm + C::kOffQ + st * C::kQBytes, &map_q, &q_full[st], 0, row0, bh);
+                tma_load_3d(sm + C::kOffV + st * C::kVBytes, &map_v, &q_full[st], 0, row0 - 32, bh);
+                last_use[st] = use;
+            }
+            if (*abort_flag) {
+                // let every copy already issued land before the CTA exits
+                for (int st = 0; st < 2; ++st)
+                    if (last_use[st] >= 0) mbar_wait(&q_full[st], last_use[st] & 1);
+                if (const_loads > 0) mbar_wait(const_full, (const_loads - 1) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            uint32_t cf_phase = 0;
+            bool ok = true;
+            auto descQ = [&](int st, int k) {
+                return smem_desc(sbase + C::kOffQ + st * C::kQBytes + k * 32, 16, C::kSbo, C::kLayout);
+            };
+            auto descKl = [&](int k) { return smem_desc(sbase + C::kOffKl + k * 32, 16, C::kSbo, C::kLayout); };
+            auto descWt = [&](int k) {
+                return smem_desc(sbase + C::kOffWt + (k >> 2) * C::kWtBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
+            };
+            auto descT = [&](int k) {
+                return smem_desc(sbase + C::kOffT + (k >> 2) * C::kTBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
+            };
+            auto descV = [&](int st, int k) {
+                return smem_desc(sbase + C::kOffV + st * C::kVBytes + k * 16 * C::kSpan, C::kVBytes, C::kSbo,
+                                 C::kLayout);
+            };
+            auto issue_S = [&](int j) -> bool {
+                const int s = j & 1, st = j % C::kStages;
+                if (!mbar_wait(&slot_free[s], ((j >> 1) & 1) ^ 1)) return false;
+                if (!mbar_wait(&q_full[st], (j / C::kStages) & 1)) return false;
+                tc_fence_after();
+                const uint32_t slot = tmem + s * C::kSlot;
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) mma_bf16_ss(slot, descQ(st, k), descKl(k), C::kIdS, k > 0);
+                mma_commit(&s_full[s]);
+                return true;
+            };
+            auto issue_O = [&](int j) -> bool {
+                const int s = j & 1, st = j % C::kStages;
+                if (!mbar_wait(&p_full[s], (j >> 1) & 1)) return false;
+                tc_fence_after();
+                const uint32_t slot = tmem + s * C::kSlot;
+#pragma unroll
+                for (int k = 0; k < M / 16; ++k)
+                    mma_bf16_ts(slot + C::kColOatt, slot + C::kColP + k * 8, descWt(k), C::kIdPW, k > 0);
+                if (prm.conv_w != nullptr) {
+#pragma unroll
+                    for (int k = 0; k < 12; ++k)
+                        mma_bf16_ss(slot + C::kColOconv, descT(k), descV(st, k), C::kIdConv, k > 0);
+                }
+                mma_commit(&o_full[s]);
+                mma_commit(&q_empty[st]);
+                return true;
+            };
+            if (count > 0) {
+                ok = mbar_wait(const_full, cf_phase) && mbar_wait(t_full, cf_phase);
+                cf_phase ^= 1;
+                tc_fence_after();
+                if (ok) ok = issue_S(0);
+            }
+            for (int i = 0; i < count && ok && !*abort_flag; ++i) {
+                const bool has_next = i + 1 < count;
+                const bool next_new_head = has_next && head_start(i + 1);
+                if (has_next && !next_new_head) ok = issue_S(i + 1);
+                if (ok) ok = issue_O(i);
+                if (ok && next_new_head) {
+                    mma_commit(const_empty);
+                    ok = mbar_wait(const_full, cf_phase) && mbar_wait(t_full, cf_phase);
+                    cf_phase ^= 1;
+                    tc_fence_after();
+                    if (ok) ok = issue_S(i + 1);
+                }
+            }
+            if (!ok) *abort_flag = 1;
+            // every MMA issued has completed before TMEM can be released
+            mma_commit(mma_done);
+            mbar_wait(mma_done, 0);
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------ softmax warpgroup
+        const int q4 = warp & 3;
+        const int r = 32 * q4 + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        const float sc = split_scale(D) * kLog2e;  // S holds Q . K_l^T with K_l already scaled
+        for (int i = 0; i < count && !warp_any(*abort_flag != 0); ++i) {
+            const int s = i & 1;
+            if (!warp_all(mbar_wait(&s_full[s], (i >> 1) & 1))) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const uint32_t slot = tmem + s * C::kSlot + lane_base;
+            uint32_t v[32];
+            float mx = -INFINITY;
+#pragma unroll 1
+            for (int c = 0; c < M / 32; ++c) {
+                tmem_ld32(slot + c * 32, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+            }
+            const float mo = mx * sc;
+            float sum = 0.f;
+#pragma unroll 1
+            for (int c = 0; c < M / 32; ++c) {
+                tmem_ld32(slot + c * 32, v);
+                tmem_ld_wait();
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float p0 = ex2(fmaf(__uint_as_float(v[2 * j]), sc, -mo));
+                    const float p1 = ex2(fmaf(__uint_as_float(v[2 * j + 1]), sc, -mo));
+                    sum += p0 + p1;
+                    pk[j] = pack_bf16(p0, p1);
+                }
+                tmem_st16(slot + C::kColP + c * 16, pk);
+            }
+            tmem_st_wait();
+            linv[s * 128 + r] = 1.f / sum;
+            tc_fence_before();
+            mbar_arrive(&p_full[s]);
+        }
+    } else if (warp >= 8) {
+        // ------------------------------------------------ epilogue warpgroup (+ Toeplitz build)
+        const int q4 = warp & 3;
+        const int r = 32 * q4 + lane;
+        const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
+        const bool conv = prm.conv_w != nullptr;
+        const bool leader = (warp == 8 && lane == 0);
+        uint32_t ce_phase = 0;
+        for (int i = 0; i < count; ++i) {
+            if (group_any(*abort_flag != 0, 2, 128)) break;
+            const int t = t0 + i, bh = t / tph, row0 = (t % tph) * C::kRows;
+            if (head_start(i)) {
+                if (i > 0) {
+                    const bool ok = mbar_wait(const_empty, ce_phase);
+                    if (group_any(!ok, 2, 128)) { *abort_flag = 1; break; }
+                    ce_phase ^= 1;
+                }
+                if (conv) {
+                    // T[r][j] = w[j - r] for 0 <= j - r < 65: row r of the banded Toeplitz matrix
+                    const float* wh = prm.conv_w + (size_t)(bh % prm.H) * kTaps;
+#pragma unroll 1
+                    for (int blk = 0; blk < 3; ++blk) {
+#pragma unroll 1
+                        for (int ch = 0; ch < 8; ++ch) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int j0 = blk * 64 + ch * 8 + 2 * e;
+                                const int d0 = j0 - r, d1 = j0 + 1 - r;
+                                const float w0 = (d0 >= 0 && d0 < kTaps) ? __ldg(wh + d0) : 0.f;
+                                const float w1 = (d1 >= 0 && d1 < kTaps) ? __ldg(wh + d1) : 0.f;
+                                pk[e] = pack_bf16(w0, w1);
+                            }
+                            *reinterpret_cast<uint4*>(sm + C::kOffT + blk * C::kTBlock + swz<128>(r, ch)) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                    fence_proxy_async_shared();
+                }
+                mbar_arrive(t_full);
+            }
+            const int s = i & 1;
+            const bool ok = mbar_wait(&p_full[s], (i >> 1) & 1) && mbar_wait(&o_full[s], (i >> 1) & 1);
+            if (group_any(!ok, 2, 128)) {
+                *abort_flag = 1;
+                break;
+            }
+            tc_fence_after();
+            const float li = linv[s * 128 + r];
+            const uint32_t slot = tmem + s * C::kSlot + lane_base;
+            uint32_t outp[D / 2];
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32], b[32];
+                tmem_ld32(slot + C::kColOatt + c * 32, a);
+                if (conv) tmem_ld32(slot + C::kColOconv + c * 32, b);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    float o0 = __uint_as_float(a[2 * j]) * li;
+                    float o1 = __uint_as_float(a[2 * j + 1]) * li;
+                    if (conv) {
+                        o0 += __uint_as_float(b[2 * j]);
+                        o1 += __uint_as_float(b[2 * j + 1]);
+                    }
+                    outp[c * 16 + j] = pack_bf16(o0, o1);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&slot_free[s]);
+            if (leader) tma_store_wait_read<0>();
+            named_barrier(1, 128);
+            uint8_t* stage = sm + C::kOffOut;
+#pragma unroll
+            for (int ch = 0; ch < D / 8; ++ch)
+                *reinterpret_cast<uint4*>(stage + swz<C::kSpan>(r, ch)) =
+                    make_uint4(outp[4 * ch], outp[4 * ch + 1], outp[4 * ch + 2], outp[4 * ch + 3]);
+            fence_proxy_async_shared();
+            named_barrier(1, 128);
+            if (leader) {
+                tma_store_3d(&map_out, stage, 0, row0, bh);
+                tma_store_commit();
+            }
+        }
+        if (leader) tma_store_wait_all<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+}  // namespace nys
