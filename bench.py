@@ -82,10 +82,14 @@ def kernel_work(w, kernel):
     if kernel == "landmarks":
         return 2 * tensor + 2 * BH * m * d * 4, 0, "alu"
     if kernel == "pinv":
-        return BH * 2 * m * d * 4 + BH * m * m * 4, BH * (2 * m * m * d + w.n_iter * 8 * m ** 3), \
+        return BH * 2 * m * d * 4 + BH * m * m * 4, BH * w.n_iter * 8 * m ** 3, \
             "alu" if w.dtype == "f32" else "tensor_tf32"
     if kernel == "k3v_partial":
         return 2 * tensor + BH * m * d * 4, BH * 4 * n * m * d, unit
+    if kernel == "kernel2":
+        return BH * (2 * m * d * 4 + 2 * m * m * 4), BH * 2 * m * m * d, "alu"
+    if kernel == "mask_bits":
+        return w.B * n + w.B * n // 8, 0, "alu"
     if kernel == "k3v_combine":
         return BH * m * d * 8, 0, "alu"
     if kernel == "w_product":
@@ -104,7 +108,7 @@ def compute_peak_tflops(unit, peaks, kernel_impl_simt):
     return peaks["bf16_tflops"]
 
 
-SIMT_KERNELS = {"landmarks", "k3v_combine", "w_product"}
+SIMT_KERNELS = {"landmarks", "k3v_combine", "w_product", "kernel2", "mask_bits"}
 
 
 def roofline_for(w, kernel, avg_ms, peaks, simt_set, traffic):
@@ -395,7 +399,7 @@ def main():
         if ent and ent.get("source_digest") == source_digest() and ent.get("workload") == w.name:
             traffic = ent.get("bytes_per_launch")
     simt = set(SIMT_KERNELS)
-    if w.dtype == "f32" or True:  # the first CUDA path runs every stage on CUDA cores
+    if w.dtype == "f32":  # the float32 path runs every stage on CUDA cores
         simt |= {"pinv", "k3v_partial", "output"}
     roof = roofline_for(w, dom, prof[dom][1] / max(1, prof[dom][0]), peaks, simt, traffic)
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"

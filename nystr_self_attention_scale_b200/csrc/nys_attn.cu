@@ -19,6 +19,7 @@
 #include "simt.cuh"
 #include "tc_k3v.cuh"
 #include "tc_output.cuh"
+#include "tc_pinv.cuh"
 
 namespace nys {
 namespace {
@@ -123,9 +124,9 @@ bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
 // ---------------------------------------------------------------- per-kernel timing
 // When enabled, every launch is bracketed by two CUDA events on the stream it
 // runs on; nys_attn_profile_read() sums their elapsed times per kernel.
-enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_MASKBITS, K_COUNT };
+enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_MASKBITS, K_KERNEL2, K_COUNT };
 const char* const kKernelNames[K_COUNT] = {"landmarks", "pinv", "k3v_partial", "k3v_combine",
-                                           "w_product", "output", "mask_bits"};
+                                           "w_product", "output", "mask_bits", "kernel2"};
 
 struct ProfRecord { int kid; cudaEvent_t a, b; };
 std::mutex g_prof_mu;
@@ -172,6 +173,7 @@ struct Plan {
     int BH, splits, keys_per_split;
     size_t off_ql, off_kl, off_ql16, off_kl16, off_k3v, off_w, off_wt16, off_z, off_pinv;
     size_t off_po, off_pm, off_pl, off_mbits, total;
+    size_t off_k2b, off_k2tb, off_zb, off_ztb, off_ta, off_tb, off_colsum, off_rowsum;  // tensor-core inverse
     int tc_cps, tc_splits;  // tensor-core kernel_3 V: 128-key chunks per split, splits
 };
 
@@ -218,11 +220,21 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
     p.off_w = take(BH * md * 4);
     p.off_wt16 = take(BH * md * 2);
     p.off_z = take(BH * mm * 4);
-    p.off_pinv = take(BH * 5 * mm * 4);
+    p.off_pinv = take(dtype == NYS_F32 ? BH * 5 * mm * 4 : 0);
     p.off_po = take(BH * splits * md * 4);
     p.off_pm = take(BH * splits * (size_t)m * 4);
     p.off_pl = take(BH * splits * (size_t)m * 4);
     p.off_mbits = take((size_t)B * ((n + 31) / 32) * 4);
+    if (dtype == NYS_BF16) {
+        p.off_k2b = take(BH * mm * 4);
+        p.off_k2tb = take(BH * mm * 4);
+        p.off_zb = take(BH * mm * 4);
+        p.off_ztb = take(BH * mm * 4);
+        p.off_ta = take(BH * mm * 4);
+        p.off_tb = take(BH * mm * 4);
+        p.off_colsum = take(BH * ((m + 31) / 32) * (size_t)m * 4);
+        p.off_rowsum = take(BH * (size_t)m * 4);
+    }
     p.total = o;
     return p;
 }
@@ -336,6 +348,50 @@ int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql1
     return NYS_OK;
 }
 
+template <int M>
+int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const float* kl, float* z, char* ws,
+                   cudaStream_t s) {
+    using C = PinvTc<M>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const size_t smem2 = (size_t)(32 + M) * (p.d + 1) * sizeof(float);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(pinv_tc_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(kernel2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+                cudaSuccess)
+            return NYS_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    uint8_t* k2b = reinterpret_cast<uint8_t*>(ws + p.off_k2b);
+    uint8_t* k2tb = reinterpret_cast<uint8_t*>(ws + p.off_k2tb);
+    float* colsum = reinterpret_cast<float*>(ws + p.off_colsum);
+    float* rowsum = reinterpret_cast<float*>(ws + p.off_rowsum);
+    {
+        ProfScope ps(K_KERNEL2, s);
+        kernel2_kernel<<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M, p.d);
+    }
+    PinvTcParams prm{k2b, k2tb, reinterpret_cast<uint8_t*>(ws + p.off_zb), reinterpret_cast<uint8_t*>(ws + p.off_ztb),
+                     reinterpret_cast<uint8_t*>(ws + p.off_ta),
+                     reinterpret_cast<uint8_t*>(ws + p.off_tb), colsum, rowsum, z, p.n_iter};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.BH * C::kClusterSize);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C::kClusterSize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ProfScope ps(K_PINV, s);
+    if (cudaLaunchKernelEx(&cfg, pinv_tc_kernel<M>, prm) != cudaSuccess) return NYS_ERR_CUDA;
+    return NYS_OK;
+}
+
 template <int D>
 int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, const __nv_bfloat16* k,
                 const __nv_bfloat16* v, const uint8_t* mask, const float* conv_w, __nv_bfloat16* out, char* ws,
@@ -349,7 +405,6 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     float* w = reinterpret_cast<float*>(ws + p.off_w);
     bf* wt16 = reinterpret_cast<bf*>(ws + p.off_wt16);
     float* z = reinterpret_cast<float*>(ws + p.off_z);
-    float* pinv = reinterpret_cast<float*>(ws + p.off_pinv);
     float* po = reinterpret_cast<float*>(ws + p.off_po);
     float* pm = reinterpret_cast<float*>(ws + p.off_pm);
     float* pl = reinterpret_cast<float*>(ws + p.off_pl);
@@ -364,10 +419,13 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     }
     if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
     if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
-    {
-        ProfScope ps(K_PINV, st.aux);
-        pinv_simt_kernel<<<BH, 256, 0, st.aux>>>(ql, kl, z, pinv, m, D, p.n_iter);
+    switch (m) {
+        case 64: rc = launch_pinv_tc<64>(p, st, ql, kl, z, ws, st.aux); break;
+        case 128: rc = launch_pinv_tc<128>(p, st, ql, kl, z, ws, st.aux); break;
+        case 256: rc = launch_pinv_tc<256>(p, st, ql, kl, z, ws, st.aux); break;
+        default: return NYS_ERR_UNSUPPORTED;
     }
+    if (rc != NYS_OK) return rc;
     if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
     if (mask) {
         const int words = p.B * (n / 32);

@@ -44,13 +44,19 @@ def _call_static(nys, q_l, k_l, n_iter):
     return z
 
 
+# float32 workloads: there the regular entry point runs the same float32 inverse that
+# nys_attn_pinv_static runs (the bf16 path uses a tf32 tensor-core inverse instead).
 @pytest.mark.parametrize("name,kw", [
     ("default_f32_masked", dict(B=2, H=3)),                 # m = 64, one launch
-    ("n16384_bf16_corr", dict(B=2, H=8, n=4096)),          # m = 256, 16 heads: several batches
+    ("corr_f32", dict(B=2, H=8, n=4096)),                   # m = 256, 16 heads: several batches
     ("degenerate_f32_it24", dict()),                         # m = n = 256, 24 iterations
 ])
 def test_static_scratch_matches_regular_entry_point(nys, name, kw):
-    w = WORKLOADS[name]
+    import dataclasses
+    if name == "corr_f32":
+        w = dataclasses.replace(WORKLOADS["n16384_bf16_corr"], name=name, dtype="f32")
+    else:
+        w = WORKLOADS[name]
     x = make_inputs(w, seed=11, **kw)
     dev = to_device(x, torch)
     _, st = nys.forward_debug(dev["q"], dev["k"], dev["v"], mask=dev["mask"], conv_w=dev["conv_w"],
