@@ -12,6 +12,7 @@ namespace nys {
 constexpr int kTaps = NYS_CONV_TAPS;
 constexpr int kHalfTaps = NYS_CONV_TAPS / 2;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
 
 // Device status word: bounded waits that run out record NYS_ERR_TIMEOUT here.
 __device__ int g_status;

@@ -274,14 +274,14 @@ int launch_simt(const Plan& p, const DeviceState& st, const T* q, const T* k, co
             k3v_partial_simt_kernel<T, D><<<grid, 256, k3v_simt_smem_bytes<D>(), s>>>(
                 ql, k, v, mask, po, pm, pl, p.H, n, m, p.splits, p.keys_per_split);
         }
-        dim3 g2(BH, std::max(1, (m * D) / 1024));
+        const long long threads = (long long)BH * m * (D / 4);
         ProfScope ps(K_COMBINE, s);
-        k3v_combine_kernel<<<g2, 256, 0, s>>>(po, pm, pl, k3v, m, D, p.splits);
+        k3v_combine_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(po, pm, pl, k3v, BH, m, D, p.splits);
     }
     if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;
     {
         ProfScope ps(K_W, s);
-        w_kernel<<<dim3(BH, (m + 31) / 32), 256, 0, s>>>(z, k3v, w, nullptr, m, D);
+        w_kernel<D><<<dim3(BH, (m + 63) / 64), 256, 0, s>>>(z, k3v, w, nullptr, m);
     }
     {
         dim3 grid(BH, (n + 63) / 64);
@@ -316,13 +316,14 @@ int launch_output_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* 
         attr_set[dev] = true;
     }
     ProfScope ps(K_OUTPUT, s);
-    output_tc_kernel<D, M><<<grid, 384, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
+    output_tc_kernel<D, M><<<grid, 320, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
     return NYS_OK;
 }
 
 template <int D>
 int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql16, const __nv_bfloat16* k,
-                  const __nv_bfloat16* v, const uint32_t* mbits, float* po, float* pm, float* pl, cudaStream_t s) {
+                  const __nv_bfloat16* v, const uint32_t* mbits, float* po, float* pm, float* pl, int sms,
+                  cudaStream_t s) {
     using C = K3vTc<D>;
     CUtensorMap mql, mk, mv;
     const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -333,7 +334,7 @@ int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql1
     const int halves = (p.m + 127) / 128;
     K3vTcParams prm{mbits, po, pm, pl, p.H, p.n, p.m, halves, p.tc_splits, p.tc_cps,
                     p.BH * halves * p.tc_splits};
-    const int grid = std::min(prm.total_items, st.sm_count);
+    const int grid = std::min(prm.total_items, sms);
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -359,7 +360,9 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(pinv_tc_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)C::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(kernel2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+            cudaFuncSetAttribute(kernel2_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(kernel2_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
                 cudaSuccess)
             return NYS_ERR_CUDA;
         attr_set[dev] = true;
@@ -370,7 +373,10 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     float* rowsum = reinterpret_cast<float*>(ws + p.off_rowsum);
     {
         ProfScope ps(K_KERNEL2, s);
-        kernel2_kernel<<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M, p.d);
+        if (p.d == 64)
+            kernel2_kernel<64><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
+        else
+            kernel2_kernel<32><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
     }
     PinvTcParams prm{k2b, k2tb, reinterpret_cast<uint8_t*>(ws + p.off_zb), reinterpret_cast<uint8_t*>(ws + p.off_ztb),
                      reinterpret_cast<uint8_t*>(ws + p.off_ta),
@@ -432,17 +438,21 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
         ProfScope ps(K_MASKBITS, s);
         mask_bits_kernel<<<(words + 255) / 256, 256, 0, s>>>(mask, mbits, p.B, n);
     }
-    rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, s);
+    // the inverse runs concurrently on its own SMs (one CTA per SM, one per 128 landmark
+    // rows of each head); the persistent kernel_3 V grid takes the rest
+    const int pinv_ctas = BH * ((m + 127) / 128);
+    const int k3v_sms = std::max(st.sm_count / 4, st.sm_count - pinv_ctas);
+    rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, k3v_sms, s);
     if (rc != NYS_OK) return rc;
     {
-        dim3 g2(BH, std::max(1, (m * D) / 1024));
+        const long long threads = (long long)BH * m * (D / 4);
         ProfScope ps(K_COMBINE, s);
-        k3v_combine_kernel<<<g2, 256, 0, s>>>(po, pm, pl, k3v, m, D, p.splits);
+        k3v_combine_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(po, pm, pl, k3v, BH, m, D, p.splits);
     }
     if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;
     {
         ProfScope ps(K_W, s);
-        w_kernel<<<dim3(BH, (m + 31) / 32), 256, 0, s>>>(z, k3v, w, wt16, m, D);
+        w_kernel<D><<<dim3(BH, (m + 63) / 64), 256, 0, s>>>(z, k3v, w, wt16, m);
     }
     switch (m) {
         case 64: rc = launch_output_tc<D, 64>(p, st, q, v, conv_w, out, kl16, wt16, s); break;

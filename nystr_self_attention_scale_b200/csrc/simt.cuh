@@ -297,50 +297,118 @@ k3v_partial_simt_kernel(const float* __restrict__ ql, const T* __restrict__ k, c
 }
 
 // Merge the key-split partials: k3v[j] = sum_s e^{M_s - M} O_s / sum_s e^{M_s - M} l_s.
-// The split order is fixed, so the result is deterministic.
+// One thread per (head, landmark row, 4 columns); the split order is fixed, so the
+// result is deterministic. All loads of a thread are independent of each other.
 __global__ void __launch_bounds__(256)
 k3v_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_m,
-                   const float* __restrict__ part_l, float* __restrict__ k3v, int m, int d, int splits) {
-    const int bh = blockIdx.x;
-    const int tid = threadIdx.x;
-    for (int e = blockIdx.y * 256 + tid; e < m * d; e += gridDim.y * 256) {
-        const int j = e / d, c = e % d;
-        float M = -INFINITY;
-        for (int s = 0; s < splits; ++s) M = fmaxf(M, part_m[((size_t)bh * splits + s) * m + j]);
-        float num = 0.f, den = 0.f;
-        for (int s = 0; s < splits; ++s) {
-            size_t row = ((size_t)bh * splits + s) * m + j;
-            float ms = part_m[row];
-            float f = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-            num = fmaf(f, part_o[row * d + c], num);
-            den = fmaf(f, part_l[row], den);
-        }
-        k3v[((size_t)bh * m + j) * d + c] = num / den;
+                   const float* __restrict__ part_l, float* __restrict__ k3v, int BH, int m, int d, int splits) {
+    const int q = d / 4;
+    const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)BH * m * q) return;
+    const int c4 = (int)(gid % q);
+    const long long bj = gid / q;           // bh * m + j
+    const int j = (int)(bj % m);
+    const long long bh = bj / m;
+    const size_t row0 = (size_t)bh * splits * m + j;   // row of split 0; split s adds s * m
+    float M = -INFINITY;
+#pragma unroll 8
+    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldg(part_m + row0 + (size_t)s * m));
+    float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
+    float den = 0.f;
+#pragma unroll 8
+    for (int s = 0; s < splits; ++s) {
+        const size_t row = row0 + (size_t)s * m;
+        const float ms = __ldg(part_m + row);
+        const float f = (ms == -INFINITY) ? 0.f : __expf(ms - M);
+        const float4 o = __ldg(reinterpret_cast<const float4*>(part_o + row * d) + c4);
+        num.x = fmaf(f, o.x, num.x);
+        num.y = fmaf(f, o.y, num.y);
+        num.z = fmaf(f, o.z, num.z);
+        num.w = fmaf(f, o.w, num.w);
+        den = fmaf(f, __ldg(part_l + row), den);
     }
+    const float inv = 1.f / den;
+    reinterpret_cast<float4*>(k3v + (size_t)bj * d)[c4] =
+        make_float4(num.x * inv, num.y * inv, num.z * inv, num.w * inv);
 }
 
-// W = Z (k3 V): 32 rows of W per CTA (walkthrough 2.4, reassociated as k1 (Z (k3 V))).
-// Also writes W^T in bf16 ([d, m] per head) when wt16 is given.
+// W = Z (k3 V) (walkthrough 2.4, reassociated as k1 (Z (k3 V))): one CTA per
+// 64-row tile of one head; the inner dimension is staged 64 at a time through
+// shared memory with all of a thread's loads issued before its stores. Also
+// writes W^T in bf16 ([d, m] per head) when wt16 is given.
+template <int D>
 __global__ void __launch_bounds__(256)
 w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __restrict__ w,
-         __nv_bfloat16* __restrict__ wt16, int m, int d) {
-    __shared__ float sZ[32][256 + 1];
-    const int bh = blockIdx.x, r0 = blockIdx.y * 32;
-    const int tid = threadIdx.x;
-    const int rows = min(32, m - r0);
-    for (int e = tid; e < 32 * m; e += 256) {
-        int r = e / m, c = e % m;
-        sZ[r][c] = r < rows ? z[((size_t)bh * m + r0 + r) * m + c] : 0.f;
+         __nv_bfloat16* __restrict__ wt16, int m) {
+    constexpr int CW = D / 16;                       // columns per thread
+    __shared__ __align__(16) float sZ[64][64 + 4];   // [row][k]
+    __shared__ __align__(16) float sK[64][D + 4];    // [k][col]
+    const int bh = blockIdx.x, r0 = blockIdx.y * 64;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    const float* zb = z + (size_t)bh * m * m;
+    const float* kb = k3v + (size_t)bh * m * D;
+    float acc[4][CW];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < CW; ++j) acc[i][j] = 0.f;
+    for (int k0 = 0; k0 < m; k0 += 64) {
+        float za[16];   // scalar loads: m need not be a multiple of 4 on the float32 path
+        float4 ka[D / 16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int idx = tid + e * 256, r = idx >> 6, c = idx & 63;
+            za[e] = (r0 + r < m && k0 + c < m) ? __ldg(zb + (size_t)(r0 + r) * m + k0 + c) : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < D / 16; ++e) {
+            const int idx = tid + e * 256, r = idx / (D / 4), c4 = idx % (D / 4);
+            ka[e] = (k0 + r < m) ? __ldg(reinterpret_cast<const float4*>(kb + (size_t)(k0 + r) * D) + c4)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int idx = tid + e * 256, r = idx >> 6, c = idx & 63;
+            sZ[r][c] = za[e];
+        }
+#pragma unroll
+        for (int e = 0; e < D / 16; ++e) {
+            const int idx = tid + e * 256, r = idx / (D / 4), c4 = idx % (D / 4);
+            *reinterpret_cast<float4*>(&sK[r][4 * c4]) = ka[e];
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int kk = 0; kk < 64; ++kk) {
+            float a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = sZ[ty * 4 + i][kk];
+#pragma unroll
+            for (int j = 0; j < CW; ++j) {
+                const float bv = sK[kk][tx * CW + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(a[i], bv, acc[i][j]);
+            }
+        }
     }
-    __syncthreads();
-    const float* kv = k3v + (size_t)bh * m * d;
-    for (int e = tid; e < 32 * d; e += 256) {
-        int r = e / d, c = e % d;
-        if (r >= rows) continue;
-        float acc = 0.f;
-        for (int kk = 0; kk < m; ++kk) acc = fmaf(sZ[r][kk], kv[(size_t)kk * d + c], acc);
-        w[((size_t)bh * m + r0 + r) * d + c] = acc;
-        if (wt16) wt16[((size_t)bh * d + c) * m + r0 + r] = __float2bfloat16_rn(acc);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = r0 + ty * 4 + i;
+        if (r >= m) continue;
+#pragma unroll
+        for (int j = 0; j < CW; ++j) w[((size_t)bh * m + r) * D + tx * CW + j] = acc[i][j];
+    }
+    if (wt16 != nullptr && r0 + ty * 4 + 3 < m) {
+#pragma unroll
+        for (int j = 0; j < CW; ++j) {
+            const int c = tx * CW + j;
+            __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0][j], acc[1][j]);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2][j], acc[3][j]);
+            uint2 pk;
+            pk.x = *reinterpret_cast<uint32_t*>(&lo);
+            pk.y = *reinterpret_cast<uint32_t*>(&hi);
+            *reinterpret_cast<uint2*>(wt16 + ((size_t)bh * D + c) * m + r0 + ty * 4) = pk;
+        }
     }
 }
 

@@ -7,16 +7,19 @@
 //                                      the d^-1/4 of K is applied in the exponent)
 //   online softmax per landmark row    one thread per row reads S from TMEM,
 //                                      masks padded keys, writes bf16 P back
-//   O_chunk = P . V_chunk              MMA with A = P from TMEM, V as an MN-major
-//                                      operand (keys x d straight from the TMA tile)
-//   O += alpha O + O_chunk             fp32 running sum in registers (one chunk behind,
-//                                      so the P.V MMA latency is hidden)
-// and writes the unnormalised partial (O, running max, running sum) of the
-// split; a deterministic combine over splits follows.
+//   O += P . V_chunk                   MMA with A = P from TMEM, V as an MN-major
+//                                      operand (keys x d straight from the TMA tile),
+//                                      accumulating in TMEM across the chunks
+// The exponentials use a per-row reference max that only moves when a chunk's
+// max exceeds it by more than 2^8 (log2 units); then O and the running sum are
+// rescaled once. Every exponential of a row uses the same reference, so the
+// result is the exact softmax; P stays below 256, well inside bf16 range.
+// Each item writes the unnormalised partial (O, reference max, running sum) of
+// its split; a deterministic combine over splits follows.
 //
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
-// TMEM allocator, warps 4-7 softmax + accumulation. S and O are double
-// buffered in TMEM; K/V chunks use a 3-stage shared-memory ring.
+// Warp roles (256 threads): warp 0 TMA producer and TMEM allocator, warp 1 MMA
+// issuer, warps 4-7 softmax. S is double buffered in TMEM; K/V chunks use a
+// 3-stage shared-memory ring.
 #pragma once
 
 #include "sm100.cuh"
@@ -35,7 +38,7 @@ struct K3vTc {
     static constexpr uint32_t kOffK = kOffQl + kTileBytes;
     static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
     static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
-    static constexpr int kNumBars = 2 + 2 * kStages + 8 + 1;
+    static constexpr int kNumBars = 2 + 2 * kStages + 7 + 1;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
     // at least 116 KB so that only one CTA (and one 512-column TMEM allocation) fits per SM
     static constexpr uint32_t kSmemNeed = kOffMisc + 16 + 1024;
@@ -68,11 +71,11 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
     uint64_t* ql_empty = bars + 1;
     uint64_t* kv_full = bars + 2;                  // [kStages]
     uint64_t* kv_empty = bars + 2 + C::kStages;    // [kStages]
-    uint64_t* s_full = bars + 2 + 2 * C::kStages;  // [2]
-    uint64_t* p_full = s_full + 2;                 // [2] (128 arrivals)
-    uint64_t* o_full = s_full + 4;                 // [2]
-    uint64_t* o_free = s_full + 6;                 // [2] (128 arrivals)
-    uint64_t* mma_done = s_full + 8;
+    uint64_t* s_full = bars + 2 + 2 * C::kStages;  // [2] S(j) in TMEM
+    uint64_t* p_full = s_full + 2;                 // [2] P(j) in TMEM (128 arrivals)
+    uint64_t* pv_done = s_full + 4;                // [2] P(j) V(j) accumulated into O
+    uint64_t* o_free = s_full + 6;                 // the item's O has been read (128 arrivals)
+    uint64_t* mma_done = s_full + 7;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
 
@@ -96,9 +99,9 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
             mbar_init(&p_full[b], 128);
-            mbar_init(&o_full[b], 1);
-            mbar_init(&o_free[b], 128);
+            mbar_init(&pv_done[b], 1);
         }
+        mbar_init(o_free, 128);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -108,7 +111,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         prefetch_tmap(&map_k);
         prefetch_tmap(&map_v);
     }
-    if (warp == 2) {
+    if (warp == 0) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -161,7 +164,8 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             };
             auto issue_S = [&](int j) -> bool {
                 const int b = j & 1, st = j % C::kStages;
-                if (j >= 2 && !mbar_wait(&o_full[b], ((j - 2) >> 1) & 1)) return false;  // P(j-2) consumed
+                // S buffer b last held S(j - 2); P(j - 2) V was accumulated once PV(j - 2) completed
+                if (j >= 2 && !mbar_wait(&pv_done[b], ((j - 2) >> 1) & 1)) return false;
                 if (!mbar_wait(&kv_full[st], (j / C::kStages) & 1)) return false;
                 tc_fence_after();
 #pragma unroll
@@ -170,16 +174,17 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 mma_commit(&s_full[b]);
                 return true;
             };
-            auto issue_PV = [&](int j) -> bool {
+            auto issue_PV = [&](int j, bool first, int item_it) -> bool {
                 const int b = j & 1, st = j % C::kStages;
                 if (!mbar_wait(&p_full[b], (j >> 1) & 1)) return false;
-                if (!mbar_wait(&o_free[b], ((j >> 1) & 1) ^ 1)) return false;
+                // the previous item's O must have been read before it is overwritten
+                if (first && !mbar_wait(o_free, (item_it & 1) ^ 1)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C::kChunk / 16; ++k)
-                    mma_bf16_ts(tmem + C::kColO + b * D, tmem + C::kColS + b * 128 + k * 8, descV(st, k), C::kIdPV,
-                                k > 0);
-                mma_commit(&o_full[b]);
+                    mma_bf16_ts(tmem + C::kColO, tmem + C::kColS + b * 128 + k * 8, descV(st, k), C::kIdPV,
+                                (first && k == 0) ? 0u : 1u);
+                mma_commit(&pv_done[b]);
                 mma_commit(&kv_empty[st]);
                 return true;
             };
@@ -194,7 +199,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                     const int j = g + c;
                     if (c + 1 < nch) ok = issue_S(j + 1);
                     else mma_commit(ql_empty);   // every S MMA of this item is issued
-                    if (ok) ok = issue_PV(j);
+                    if (ok) ok = issue_PV(j, c == 0, it);
                 }
                 g += nch;
             }
@@ -206,84 +211,76 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-        const float s_d = split_scale(D);
-        const float sc = s_d * kLog2e;
-        int g = 0;
-        for (int item = blockIdx.x; item < prm.total_items && !warp_any(*abort_flag != 0); item += gridDim.x) {
+        const float sc = split_scale(D) * kLog2e;   // exponent scale of the raw S = Q_l . K^T
+        constexpr float kSlack = 8.f;               // log2 units: P stays below 2^8
+        int g = 0, it = 0;
+        for (int item = blockIdx.x; item < prm.total_items && !warp_any(*abort_flag != 0);
+             item += gridDim.x, ++it) {
             const int bh = item / per_bh, half = (item / prm.splits) % prm.halves;
             const int split = item % prm.splits;
             const int b_idx = bh / prm.H;
             int c0;
             const int nch = item_chunks(item, &c0);
-            float o[D];
-#pragma unroll
-            for (int e = 0; e < D; ++e) o[e] = 0.f;
-            float m_run = -INFINITY, l_run = 0.f, alpha_prev = 1.f;
+            float m_ref = -INFINITY, l_run = 0.f;   // reference max (log2 units) and running sum
             bool ok = true;
-            auto accumulate = [&](int j, float alpha) -> bool {
-                const int b = j & 1;
-                if (!warp_all(mbar_wait(&o_full[b], (j >> 1) & 1))) return false;
-                tc_fence_after();
-                uint32_t v[32];
-#pragma unroll
-                for (int h = 0; h < D / 32; ++h) {
-                    tmem_ld32(tmem + lane_base + C::kColO + b * D + h * 32, v);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) o[h * 32 + e] = fmaf(o[h * 32 + e], alpha, __uint_as_float(v[e]));
-                }
-                tc_fence_before();
-                mbar_arrive(&o_free[b]);
-                return true;
-            };
             for (int c = 0; c < nch && ok; ++c) {
                 const int j = g + c, b = j & 1;
                 const int key0 = (c0 + c) * C::kChunk;
                 // key-validity bits of this chunk (bit k = key key0 + k is valid)
                 uint32_t mb[4] = {~0u, ~0u, ~0u, ~0u};
                 if (prm.mask_bits != nullptr) {
-                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(prm.mask_bits + (size_t)b_idx * (prm.n / 32) + key0 / 32));
+                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(prm.mask_bits + (size_t)b_idx * (prm.n / 32) +
+                                                                          key0 / 32));
                     mb[0] = u.x; mb[1] = u.y; mb[2] = u.z; mb[3] = u.w;
                 }
                 const bool full = (mb[0] & mb[1] & mb[2] & mb[3]) == ~0u;
                 if (!warp_all(mbar_wait(&s_full[b], (j >> 1) & 1))) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sbuf = tmem + lane_base + C::kColS + b * 128;
-                uint32_t v[32];
-                float cmax = -INFINITY;
-#pragma unroll 1
-                for (int h = 0; h < 4; ++h) {
-                    tmem_ld32(sbuf + h * 32, v);
-                    tmem_ld_wait();
-                    if (full) {
+                uint32_t v[4][32];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) cmax = fmaxf(cmax, __uint_as_float(v[e]));
-                    } else {
+                for (int h = 0; h < 4; ++h) tmem_ld32(sbuf + h * 32, v[h]);
+                tmem_ld_wait();
+                if (!full) {
+#pragma unroll
+                    for (int h = 0; h < 4; ++h)
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
-                            if ((mb[h] >> e) & 1u) cmax = fmaxf(cmax, __uint_as_float(v[e]));
+                            if (!((mb[h] >> e) & 1u)) v[h][e] = __float_as_uint(-INFINITY);
+                }
+                float cmax = -INFINITY;
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) cmax = fmaxf(cmax, __uint_as_float(v[h][e]));
+                const float cm = cmax * sc;
+                // move the reference only when this chunk's max exceeds it by more than the slack
+                const bool move = cm > m_ref + kSlack;
+                const float m_new = move ? cm : m_ref;
+                const float alpha = move ? ex2(m_ref - m_new) : 1.f;   // m_ref = -inf gives 0
+                if (c > 0 && warp_any(move && m_ref != -INFINITY)) {
+                    // rescale this warp's rows of O once P(j - 1) V has been accumulated
+                    if (!warp_all(mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) { ok = false; break; }
+                    tc_fence_after();
+                    uint32_t o[32];
+#pragma unroll
+                    for (int h = 0; h < D / 32; ++h) {
+                        tmem_ld32(tmem + lane_base + C::kColO + h * 32, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tmem + lane_base + C::kColO + h * 32, o);
                     }
                 }
-                const float m_new = fmaxf(m_run, cmax);
-                // a row whose keys so far are all padded keeps P = 0 (no branch around the
-                // warp-collective TMEM accesses below)
-                const bool live = m_new != -INFINITY;
-                const float mo = live ? m_new * sc : 0.f;
-                const float alpha = live ? ex2(fmaf(m_run, sc, -mo)) : 1.f;   // m_run = -inf gives 0
+                const float mo = m_new == -INFINITY ? 0.f : m_new;   // rows with every key padded so far: P = 0
                 float sum = 0.f;
-#pragma unroll 1
+#pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    tmem_ld32(sbuf + h * 32, v);
-                    tmem_ld_wait();
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        float p0 = ex2(fmaf(__uint_as_float(v[2 * e]), sc, -mo));
-                        float p1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), sc, -mo));
-                        const bool k0 = live && (full || ((mb[h] >> (2 * e)) & 1u));
-                        const bool k1 = live && (full || ((mb[h] >> (2 * e + 1)) & 1u));
-                        p0 = k0 ? p0 : 0.f;
-                        p1 = k1 ? p1 : 0.f;
+                        const float p0 = ex2(fmaf(__uint_as_float(v[h][2 * e]), sc, -mo));
+                        const float p1 = ex2(fmaf(__uint_as_float(v[h][2 * e + 1]), sc, -mo));
                         sum += p0 + p1;
                         pk[e] = pack_bf16(p0, p1);
                     }
@@ -293,20 +290,37 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 tc_fence_before();
                 mbar_arrive(&p_full[b]);
                 l_run = fmaf(l_run, alpha, sum);
-                m_run = m_new;
-                if (c > 0 && !accumulate(j - 1, alpha_prev)) { ok = false; break; }
-                alpha_prev = alpha;
+                m_ref = m_new;
             }
-            if (ok && nch > 0) ok = accumulate(g + nch - 1, alpha_prev);
+            // the item's O is complete once its last P V has been accumulated; stream it out
+            const int row = half * C::kRows + r;
+            const size_t prow = ((size_t)bh * prm.splits + split) * prm.m + row;
+            if (ok && nch > 0) {
+                const int jl = g + nch - 1;
+                ok = warp_all(mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1));
+                if (ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int h = 0; h < D / 32; ++h) {
+                        uint32_t t[32];
+                        tmem_ld32(tmem + lane_base + C::kColO + h * 32, t);
+                        tmem_ld_wait();
+                        if (row < prm.m) {
+                            float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D + h * 32);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                dst[e] = make_float4(__uint_as_float(t[4 * e]), __uint_as_float(t[4 * e + 1]),
+                                                     __uint_as_float(t[4 * e + 2]), __uint_as_float(t[4 * e + 3]));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(o_free);
             if (!ok) { *abort_flag = 1; break; }
             g += nch;
-            const int row = half * C::kRows + r;
             if (row < prm.m) {
-                const size_t prow = ((size_t)bh * prm.splits + split) * prm.m + row;
-                float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D);
-#pragma unroll
-                for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-                prm.part_m[prow] = m_run == -INFINITY ? -INFINITY : m_run * s_d;
+                prm.part_m[prow] = m_ref == -INFINITY ? -INFINITY : m_ref * kLn2;
                 prm.part_l[prow] = l_run;
             }
         }
@@ -314,7 +328,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }

@@ -13,9 +13,10 @@
 //                                    supplied by the TMA out-of-bounds fill)
 //   out    = O_att / rowsum(P) + O_conv, bf16, TMA store
 //
-// Warp roles (384 threads, one persistent CTA per SM over a contiguous range of
-// tiles): warp 0 TMA producer, warp 1 MMA issuer, warp 2 TMEM allocator,
-// warps 4-7 softmax, warps 8-11 epilogue (and the Toeplitz build).
+// Warp roles (320 threads, one persistent CTA per SM over a contiguous range of
+// tiles): warp 0 TMA producer and TMEM allocator, warp 1 MMA issuer, warps 2-5
+// softmax, warps 6-9 epilogue (and the Toeplitz build). A warp w reaches TMEM
+// lanes 32 (w % 4) .. +31, so each group of four warps covers all 128 rows.
 // Two TMEM slots alternate between consecutive tiles so the softmax of one
 // tile overlaps the MMAs and the epilogue of the other. Every wait is bounded.
 #pragma once
@@ -68,7 +69,7 @@ struct OutTcParams {
 };
 
 template <int D, int M>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(320, 1)
 output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
                  const __grid_constant__ CUtensorMap map_out, const __grid_constant__ CUtensorMap map_kl,
                  const __grid_constant__ CUtensorMap map_wt, const OutTcParams prm) {
@@ -123,7 +124,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         prefetch_tmap(&map_kl);
         prefetch_tmap(&map_wt);
     }
-    if (warp == 2) {
+    if (warp == 0) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -236,7 +237,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mma_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 2 && warp < 6) {
         // ------------------------------------------------ softmax warpgroup
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
@@ -247,43 +248,53 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             if (!warp_all(mbar_wait(&s_full[s], (i >> 1) & 1))) { *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
-            uint32_t v[32];
+            // pass 1: row max; up to four 32-column loads in flight per wait
+            constexpr int kNB1 = M >= 128 ? 4 : M / 32;
             float mx = -INFINITY;
 #pragma unroll 1
-            for (int c = 0; c < M / 32; ++c) {
-                tmem_ld32(slot + c * 32, v);
+            for (int c0 = 0; c0 < M; c0 += 32 * kNB1) {
+                uint32_t v[kNB1][32];
+#pragma unroll
+                for (int bq = 0; bq < kNB1; ++bq) tmem_ld32(slot + c0 + bq * 32, v[bq]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[j]));
+                for (int bq = 0; bq < kNB1; ++bq)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[bq][j]));
             }
             const float mo = mx * sc;
+            // pass 2: exponentials, 64 columns per wait, packed bf16 P into columns [c0/2, c0/2 + 32)
             float sum = 0.f;
 #pragma unroll 1
-            for (int c = 0; c < M / 32; ++c) {
-                tmem_ld32(slot + c * 32, v);
+            for (int c0 = 0; c0 < M; c0 += 64) {
+                uint32_t v[2][32];
+                tmem_ld32(slot + c0, v[0]);
+                tmem_ld32(slot + c0 + 32, v[1]);
                 tmem_ld_wait();
-                uint32_t pk[16];
+                uint32_t pk[32];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const float p0 = ex2(fmaf(__uint_as_float(v[2 * j]), sc, -mo));
-                    const float p1 = ex2(fmaf(__uint_as_float(v[2 * j + 1]), sc, -mo));
-                    sum += p0 + p1;
-                    pk[j] = pack_bf16(p0, p1);
-                }
-                tmem_st16(slot + C::kColP + c * 16, pk);
+                for (int bq = 0; bq < 2; ++bq)
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const float p0 = ex2(fmaf(__uint_as_float(v[bq][2 * j]), sc, -mo));
+                        const float p1 = ex2(fmaf(__uint_as_float(v[bq][2 * j + 1]), sc, -mo));
+                        sum += p0 + p1;
+                        pk[bq * 16 + j] = pack_bf16(p0, p1);
+                    }
+                tmem_st32(slot + C::kColP + c0 / 2, pk);
             }
             tmem_st_wait();
             linv[s * 128 + r] = 1.f / sum;
             tc_fence_before();
             mbar_arrive(&p_full[s]);
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 6) {
         // ------------------------------------------------ epilogue warpgroup (+ Toeplitz build)
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const bool conv = prm.conv_w != nullptr;
-        const bool leader = (warp == 8 && lane == 0);
+        const bool leader = (warp == 6 && lane == 0);
         uint32_t ce_phase = 0;
         for (int i = 0; i < count; ++i) {
             if (group_any(*abort_flag != 0, 2, 128)) break;
@@ -366,7 +377,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }

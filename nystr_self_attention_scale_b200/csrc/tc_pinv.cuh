@@ -48,22 +48,52 @@ __device__ __forceinline__ float tf32_rna(float x) {
 }
 
 // ------------------------------------------------------------------ kernel_2 rows
-// grid (BH, m / 32), 256 threads. Dynamic shared memory: (32 + m) * (d + 1) floats.
+// grid (BH, m / 32), 256 threads. Dynamic shared memory: (32 + m) * (D + 1) floats.
+template <int D>
 __global__ void __launch_bounds__(256)
 kernel2_kernel(const float* __restrict__ ql, const float* __restrict__ kl, uint8_t* __restrict__ k2b,
                uint8_t* __restrict__ k2tb, float* __restrict__ colsum_part, float* __restrict__ rowsum,
-               int m, int d) {
+               int m) {
     extern __shared__ float sm2[];
+    constexpr int d = D, ld = D + 1;
     const int bh = blockIdx.x, blk = blockIdx.y, r0 = blk * 32;
-    const int ld = d + 1;
     float* sq = sm2;                 // [32][d+1]
     float* sk = sm2 + 32 * ld;       // [m][d+1]
     float* ss = sk;                  // scores [32][m+1] reuse after the products (see below)
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const float* qb = ql + ((size_t)bh * m + r0) * d;
-    const float* kb = kl + (size_t)bh * m * d;
-    for (int e = tid; e < 32 * d; e += 256) sq[(e / d) * ld + e % d] = qb[e];
-    for (int e = tid; e < m * d; e += 256) sk[(e / d) * ld + e % d] = kb[e];
+    const float4* qb = reinterpret_cast<const float4*>(ql + ((size_t)bh * m + r0) * d);
+    const float4* kb = reinterpret_cast<const float4*>(kl + (size_t)bh * m * d);
+    // stage Q_l rows and all of K_l; every thread issues its loads before its stores
+    {
+        constexpr int kQv = 32 * D / 4 / 256;   // float4 per thread for the 32 Q_l rows
+        float4 qv[kQv];
+#pragma unroll
+        for (int e = 0; e < kQv; ++e) qv[e] = __ldg(qb + tid + e * 256);
+#pragma unroll
+        for (int e = 0; e < kQv; ++e) {
+            const int idx = (tid + e * 256) * 4, r = idx / D, c = idx % D;
+            sq[r * ld + c] = qv[e].x; sq[r * ld + c + 1] = qv[e].y;
+            sq[r * ld + c + 2] = qv[e].z; sq[r * ld + c + 3] = qv[e].w;
+        }
+        const int nkv = m * D / 4;
+        for (int base = 0; base < nkv; base += 256 * 8) {
+            float4 kv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int idx = base + tid + e * 256;
+                kv[e] = idx < nkv ? __ldg(kb + idx) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int idx = base + tid + e * 256;
+                if (idx < nkv) {
+                    const int r = (idx * 4) / D, c = (idx * 4) % D;
+                    sk[r * ld + c] = kv[e].x; sk[r * ld + c + 1] = kv[e].y;
+                    sk[r * ld + c + 2] = kv[e].z; sk[r * ld + c + 3] = kv[e].w;
+                }
+            }
+        }
+    }
     __syncthreads();
     // each thread: rows (warp*4 .. +4), columns lane, lane+32, ...
     constexpr int kMaxCols = 8;   // m <= 256
