@@ -316,7 +316,7 @@ int launch_output_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* 
         attr_set[dev] = true;
     }
     ProfScope ps(K_OUTPUT, s);
-    output_tc_kernel<D, M><<<grid, 320, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
+    output_tc_kernel<D, M><<<grid, 448, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
     return NYS_OK;
 }
 
@@ -345,7 +345,7 @@ int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql1
         attr_set[dev] = true;
     }
     ProfScope ps(K_K3V, s);
-    k3v_tc_kernel<D><<<grid, 256, C::kSmemBytes, s>>>(mql, mk, mv, prm);
+    k3v_tc_kernel<D><<<grid, 384, C::kSmemBytes, s>>>(mql, mk, mv, prm);
     return NYS_OK;
 }
 

@@ -17,9 +17,12 @@
 // Each item writes the unnormalised partial (O, reference max, running sum) of
 // its split; a deterministic combine over splits follows.
 //
-// Warp roles (256 threads): warp 0 TMA producer and TMEM allocator, warp 1 MMA
-// issuer, warps 4-7 softmax. S is double buffered in TMEM; K/V chunks use a
-// 3-stage shared-memory ring.
+// Warp roles (384 threads): warp 0 TMA producer and TMEM allocator, warp 1 MMA
+// issuer, warps 4-7 and 8-11 two softmax warpgroups that split every chunk's
+// 128 keys (64 each), exchanging the chunk max through shared memory. Each
+// group writes its P into its own half of the S columns (the P.V MMA takes its
+// A operand from the two ranges). S is double buffered in TMEM; K/V chunks use
+// a 3-stage shared-memory ring.
 #pragma once
 
 #include "sm100.cuh"
@@ -39,12 +42,14 @@ struct K3vTc {
     static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
     static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
     static constexpr int kNumBars = 2 + 2 * kStages + 7 + 1;
-    static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr uint32_t kOffXch = kOffBar + kNumBars * 8;          // [2][2][128] chunk maxima
+    static constexpr uint32_t kOffLx = kOffXch + 2 * 2 * 128 * 4;        // [128] partial sums
+    static constexpr uint32_t kOffMisc = kOffLx + 128 * 4;
     // at least 116 KB so that only one CTA (and one 512-column TMEM allocation) fits per SM
     static constexpr uint32_t kSmemNeed = kOffMisc + 16 + 1024;
     static constexpr uint32_t kSmemBytes = kSmemNeed > 118784 ? kSmemNeed : 118784;
     static constexpr int kTmemCols = 512;
-    static constexpr int kColS = 0, kColO = 256;
+    static constexpr int kColS = 0, kColO = 256;   // S[b] at 128 b; P halves at 128 b + {0, 64}
     static constexpr uint32_t kIdS = sm100::make_idesc(128, kChunk, sm100::kFmtBf16, sm100::kFmtBf16, 0, 0);
     static constexpr uint32_t kIdPV = sm100::make_idesc(128, D, sm100::kFmtBf16, sm100::kFmtBf16, 0, 1);
 };
@@ -58,7 +63,7 @@ struct K3vTcParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
 k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const K3vTcParams prm) {
     using C = K3vTc<D>;
@@ -98,10 +103,10 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 128);
+            mbar_init(&p_full[b], 256);
             mbar_init(&pv_done[b], 1);
         }
-        mbar_init(o_free, 128);
+        mbar_init(o_free, 256);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -181,9 +186,11 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 if (first && !mbar_wait(o_free, (item_it & 1) ^ 1)) return false;
                 tc_fence_after();
 #pragma unroll
-                for (int k = 0; k < C::kChunk / 16; ++k)
-                    mma_bf16_ts(tmem + C::kColO, tmem + C::kColS + b * 128 + k * 8, descV(st, k), C::kIdPV,
-                                (first && k == 0) ? 0u : 1u);
+                for (int k = 0; k < C::kChunk / 16; ++k) {
+                    // keys 16k .. 16k+15: the first 64 from group 0's P, the rest from group 1's
+                    const uint32_t pa = tmem + C::kColS + b * 128 + (k < 4 ? k * 8 : 64 + (k - 4) * 8);
+                    mma_bf16_ts(tmem + C::kColO, pa, descV(st, k), C::kIdPV, (first && k == 0) ? 0u : 1u);
+                }
                 mma_commit(&pv_done[b]);
                 mma_commit(&kv_empty[st]);
                 return true;
@@ -208,91 +215,105 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             mbar_wait(mma_done, 0);
         }
     } else if (warp >= 4) {
+        const int grp = (warp - 4) >> 2;          // softmax group: keys [64 grp, 64 grp + 64) of a chunk
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const float sc = split_scale(D) * kLog2e;   // exponent scale of the raw S = Q_l . K^T
         constexpr float kSlack = 8.f;               // log2 units: P stays below 2^8
+        float* xch = reinterpret_cast<float*>(sm + C::kOffXch);
+        float* lx = reinterpret_cast<float*>(sm + C::kOffLx);
         int g = 0, it = 0;
-        for (int item = blockIdx.x; item < prm.total_items && !warp_any(*abort_flag != 0);
-             item += gridDim.x, ++it) {
+        for (int item = blockIdx.x; item < prm.total_items; item += gridDim.x, ++it) {
+            if (group_any(*abort_flag != 0, 1, 256)) break;
             const int bh = item / per_bh, half = (item / prm.splits) % prm.halves;
             const int split = item % prm.splits;
             const int b_idx = bh / prm.H;
             int c0;
             const int nch = item_chunks(item, &c0);
-            float m_ref = -INFINITY, l_run = 0.f;   // reference max (log2 units) and running sum
+            float m_ref = -INFINITY, l_run = 0.f;   // reference max (log2 units) and this group's sum
             bool ok = true;
-            for (int c = 0; c < nch && ok; ++c) {
+            for (int c = 0; c < nch; ++c) {
                 const int j = g + c, b = j & 1;
                 const int key0 = (c0 + c) * C::kChunk;
-                // key-validity bits of this chunk (bit k = key key0 + k is valid)
-                uint32_t mb[4] = {~0u, ~0u, ~0u, ~0u};
+                // key-validity bits of this group's 64 keys (bit k = key key0 + 64 grp + k)
+                uint32_t mb0 = ~0u, mb1 = ~0u;
                 if (prm.mask_bits != nullptr) {
-                    const uint4 u = __ldg(reinterpret_cast<const uint4*>(prm.mask_bits + (size_t)b_idx * (prm.n / 32) +
-                                                                          key0 / 32));
-                    mb[0] = u.x; mb[1] = u.y; mb[2] = u.z; mb[3] = u.w;
+                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(prm.mask_bits + (size_t)b_idx * (prm.n / 32) +
+                                                                          key0 / 32 + 2 * grp));
+                    mb0 = u.x; mb1 = u.y;
                 }
-                const bool full = (mb[0] & mb[1] & mb[2] & mb[3]) == ~0u;
-                if (!warp_all(mbar_wait(&s_full[b], (j >> 1) & 1))) { ok = false; break; }
+                const bool full = (mb0 & mb1) == ~0u;
+                ok = warp_all(mbar_wait(&s_full[b], (j >> 1) & 1));
+                if (group_any(!ok, 1, 256)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sbuf = tmem + lane_base + C::kColS + b * 128;
-                uint32_t v[4][32];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) tmem_ld32(sbuf + h * 32, v[h]);
+                uint32_t v[2][32];
+                tmem_ld32(sbuf + 64 * grp, v[0]);
+                tmem_ld32(sbuf + 64 * grp + 32, v[1]);
                 tmem_ld_wait();
                 if (!full) {
 #pragma unroll
-                    for (int h = 0; h < 4; ++h)
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (!((mb[h] >> e) & 1u)) v[h][e] = __float_as_uint(-INFINITY);
+                    for (int e = 0; e < 32; ++e) {
+                        if (!((mb0 >> e) & 1u)) v[0][e] = __float_as_uint(-INFINITY);
+                        if (!((mb1 >> e) & 1u)) v[1][e] = __float_as_uint(-INFINITY);
+                    }
                 }
                 float cmax = -INFINITY;
 #pragma unroll
-                for (int h = 0; h < 4; ++h)
+                for (int h = 0; h < 2; ++h)
 #pragma unroll
                     for (int e = 0; e < 32; ++e) cmax = fmaxf(cmax, __uint_as_float(v[h][e]));
+                xch[(b * 2 + grp) * 128 + r] = cmax;
+                named_barrier(1, 256);
+                cmax = fmaxf(cmax, xch[(b * 2 + (grp ^ 1)) * 128 + r]);
                 const float cm = cmax * sc;
                 // move the reference only when this chunk's max exceeds it by more than the slack
+                // (both groups take the same decision: same maxima, same history)
                 const bool move = cm > m_ref + kSlack;
                 const float m_new = move ? cm : m_ref;
                 const float alpha = move ? ex2(m_ref - m_new) : 1.f;   // m_ref = -inf gives 0
-                if (c > 0 && warp_any(move && m_ref != -INFINITY)) {
+                if (grp == 0 && c > 0 && warp_any(move && m_ref != -INFINITY)) {
                     // rescale this warp's rows of O once P(j - 1) V has been accumulated
-                    if (!warp_all(mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1))) { ok = false; break; }
-                    tc_fence_after();
-                    uint32_t o[32];
+                    ok = warp_all(mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
+                    if (ok) {
+                        tc_fence_after();
+                        uint32_t o[32];
 #pragma unroll
-                    for (int h = 0; h < D / 32; ++h) {
-                        tmem_ld32(tmem + lane_base + C::kColO + h * 32, o);
-                        tmem_ld_wait();
+                        for (int h = 0; h < D / 32; ++h) {
+                            tmem_ld32(tmem + lane_base + C::kColO + h * 32, o);
+                            tmem_ld_wait();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tmem + lane_base + C::kColO + h * 32, o);
+                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                            tmem_st32(tmem + lane_base + C::kColO + h * 32, o);
+                        }
                     }
                 }
                 const float mo = m_new == -INFINITY ? 0.f : m_new;   // rows with every key padded so far: P = 0
                 float sum = 0.f;
+                const uint32_t pcol = sbuf + 64 * grp;   // this group's P: 32 columns at the start of its half
 #pragma unroll
-                for (int h = 0; h < 4; ++h) {
+                for (int h = 0; h < 2; ++h) {
                     uint32_t pk[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        const float p0 = ex2(fmaf(__uint_as_float(v[h][2 * e]), sc, -mo));
-                        const float p1 = ex2(fmaf(__uint_as_float(v[h][2 * e + 1]), sc, -mo));
-                        sum += p0 + p1;
-                        pk[e] = pack_bf16(p0, p1);
+                        // bf16 P by truncation; the running sum adds the same truncated values
+                        const uint32_t u0 = __float_as_uint(ex2(fmaf(__uint_as_float(v[h][2 * e]), sc, -mo))) & 0xFFFF0000u;
+                        const uint32_t u1 = __float_as_uint(ex2(fmaf(__uint_as_float(v[h][2 * e + 1]), sc, -mo))) & 0xFFFF0000u;
+                        sum += __uint_as_float(u0) + __uint_as_float(u1);
+                        pk[e] = __byte_perm(u0, u1, 0x7632);
                     }
-                    tmem_st16(sbuf + h * 16, pk);
+                    tmem_st16(pcol + h * 16, pk);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&p_full[b]);
                 l_run = fmaf(l_run, alpha, sum);
                 m_ref = m_new;
+                if (group_any(!ok, 1, 256)) { ok = false; break; }
             }
-            // the item's O is complete once its last P V has been accumulated; stream it out
+            // the item's O is complete once its last P V has been accumulated; each group streams
+            // out half of the columns, group 0 adds the two partial sums
             const int row = half * C::kRows + r;
             const size_t prow = ((size_t)bh * prm.splits + split) * prm.m + row;
             if (ok && nch > 0) {
@@ -301,7 +322,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 if (ok) {
                     tc_fence_after();
 #pragma unroll
-                    for (int h = 0; h < D / 32; ++h) {
+                    for (int h = grp; h < D / 32; h += 2) {
                         uint32_t t[32];
                         tmem_ld32(tmem + lane_base + C::kColO + h * 32, t);
                         tmem_ld_wait();
@@ -317,12 +338,14 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             }
             tc_fence_before();
             mbar_arrive(o_free);
-            if (!ok) { *abort_flag = 1; break; }
+            if (grp == 1) lx[r] = l_run;
+            if (group_any(!ok, 1, 256)) { *abort_flag = 1; break; }
             g += nch;
-            if (row < prm.m) {
+            if (grp == 0 && row < prm.m) {
                 prm.part_m[prow] = m_ref == -INFINITY ? -INFINITY : m_ref * kLn2;
-                prm.part_l[prow] = l_run;
+                prm.part_l[prow] = l_run + lx[r];
             }
+            named_barrier(1, 256);   // lx is read before the next item overwrites it
         }
     }
 

@@ -13,12 +13,16 @@
 //                                    supplied by the TMA out-of-bounds fill)
 //   out    = O_att / rowsum(P) + O_conv, bf16, TMA store
 //
-// Warp roles (320 threads, one persistent CTA per SM over a contiguous range of
-// tiles): warp 0 TMA producer and TMEM allocator, warp 1 MMA issuer, warps 2-5
-// softmax, warps 6-9 epilogue (and the Toeplitz build). A warp w reaches TMEM
-// lanes 32 (w % 4) .. +31, so each group of four warps covers all 128 rows.
-// Two TMEM slots alternate between consecutive tiles so the softmax of one
-// tile overlaps the MMAs and the epilogue of the other. Every wait is bounded.
+// Warp roles (448 threads, one persistent CTA per SM over a contiguous range of
+// tiles): warp 0 TMA producers and TMEM allocator, warp 1 MMA issuer, warps
+// 2-5 and 6-9 two softmax warpgroups, warps 10-13 epilogue (and the Toeplitz
+// build). A warp w reaches TMEM lanes 32 (w % 4) .. +31, so each group of four
+// warps covers all 128 rows. Two TMEM slots alternate between consecutive
+// tiles. Both softmax warpgroups work on the same tile, each on half of the
+// landmark columns (row maxima are exchanged through shared memory), which
+// halves the time a slot is held by the softmax. Each group writes its P
+// into its own half of the S columns, and the P.W MMA takes its A operand
+// from those two column ranges. Every wait is bounded.
 #pragma once
 
 #include "sm100.cuh"
@@ -38,22 +42,28 @@ struct OutTc {
     static constexpr uint32_t kKlBytes = M * kSpan;
     static constexpr uint32_t kWtBlock = D * 128;     // [D][64] bf16 K-block of W^T
     static constexpr uint32_t kWtBytes = (M / 64) * kWtBlock;
+    static constexpr uint32_t kWtLoadBytes = kWtBytes;
     static constexpr uint32_t kTBlock = 128 * 128;    // [128][64] bf16 K-block of T
     static constexpr uint32_t kTBytes = 3 * kTBlock;
     static constexpr uint32_t kOutBytes = kRows * kSpan;
-    static constexpr int kSlotNeed = (M > M / 2 + 2 * D) ? M : (M / 2 + 2 * D);
-    static constexpr int kSlot = kSlotNeed <= 64 ? 64 : (kSlotNeed <= 128 ? 128 : 256);
+    // TMEM slot (256 columns): S in [0, M); P of the two column halves at [0, M/4) and
+    // [M/2, M/2 + M/4); O_att and O_conv in columns the softmax no longer needs
+    static constexpr int kSlot = 256;
     static constexpr int kTmemCols = 2 * kSlot;
-    static constexpr int kColP = 0, kColOatt = M / 2, kColOconv = M / 2 + D;
+    static constexpr int kColPA = 0, kColPB = M / 2;
+    static constexpr int kColOatt = M == 256 ? M / 4 : M;
+    static constexpr int kColOconv = M == 256 ? 3 * M / 4 : M + D;
+    static_assert(kColOconv + D <= kSlot, "TMEM slot layout");
     static constexpr uint32_t kOffQ = 0;
     static constexpr uint32_t kOffV = kOffQ + kStages * kQBytes;
     static constexpr uint32_t kOffKl = kOffV + kStages * kVBytes;
     static constexpr uint32_t kOffWt = kOffKl + kKlBytes;
     static constexpr uint32_t kOffT = kOffWt + kWtBytes;
     static constexpr uint32_t kOffOut = kOffT + kTBytes;
-    static constexpr uint32_t kOffLinv = kOffOut + kOutBytes;   // [2][128] float
-    static constexpr uint32_t kOffBar = kOffLinv + 2 * 128 * 4;
-    static constexpr int kNumBars = 16;
+    static constexpr uint32_t kOffPmax = kOffOut + kOutBytes;   // [2 slots][2 groups][128] float
+    static constexpr uint32_t kOffPsum = kOffPmax + 2 * 2 * 128 * 4;
+    static constexpr uint32_t kOffBar = kOffPsum + 2 * 2 * 128 * 4;
+    static constexpr int kNumBars = 20;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -69,7 +79,7 @@ struct OutTcParams {
 };
 
 template <int D, int M>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
 output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
                  const __grid_constant__ CUtensorMap map_out, const __grid_constant__ CUtensorMap map_kl,
                  const __grid_constant__ CUtensorMap map_wt, const OutTcParams prm) {
@@ -79,8 +89,8 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(sm);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
-    uint64_t* q_full = bars + 0;     // [2] TMA Q+V landed
-    uint64_t* q_empty = bars + 2;    // [2] stage reusable
+    uint64_t* q_full = bars + 0;     // [2] Q tile landed
+    uint64_t* q_empty = bars + 2;    // [2] Q stage reusable (its S MMA completed)
     uint64_t* s_full = bars + 4;     // [2] S in TMEM
     uint64_t* p_full = bars + 6;     // [2] P in TMEM, S fully read (128 arrivals)
     uint64_t* o_full = bars + 8;     // [2] O_att, O_conv ready
@@ -89,9 +99,12 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint64_t* const_empty = bars + 13;
     uint64_t* mma_done = bars + 14;
     uint64_t* t_full = bars + 15;    // Toeplitz matrix built (128 arrivals)
+    uint64_t* v_full = bars + 16;    // [2] V halo landed
+    uint64_t* v_empty = bars + 18;   // [2] V stage reusable (its conv MMA completed)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
-    float* linv = reinterpret_cast<float*>(sm + C::kOffLinv);
+    float* pmax = reinterpret_cast<float*>(sm + C::kOffPmax);
+    float* psum = reinterpret_cast<float*>(sm + C::kOffPsum);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // contiguous tile range of this CTA
@@ -106,9 +119,11 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mbar_init(&q_full[b], 1);
             mbar_init(&q_empty[b], 1);
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 128);
+            mbar_init(&p_full[b], 256);
             mbar_init(&o_full[b], 1);
             mbar_init(&slot_free[b], 128);
+            mbar_init(&v_full[b], 1);
+            mbar_init(&v_empty[b], 1);
         }
         mbar_init(const_full, 1);
         mbar_init(t_full, 128);
@@ -134,7 +149,9 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+        // ------------------------------------------------ TMA producers: lane 0 streams Q tiles
+        // and the per-head constants, lane 1 streams the V halos (needed only by the conv MMA,
+        // late in a tile), so each Q tile is requested as soon as its stage's S MMA is done.
         if (lane == 0) {
             uint32_t ce_phase = 0;
             int last_use[2] = {-1, -1};
@@ -146,7 +163,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         if (!mbar_wait(const_empty, ce_phase)) { *abort_flag = 1; break; }
                         ce_phase ^= 1;
                     }
-                    mbar_arrive_expect_tx(const_full, C::kKlBytes + C::kWtBytes);
+                    mbar_arrive_expect_tx(const_full, C::kKlBytes + C::kWtLoadBytes);
                     tma_load_3d(sm + C::kOffKl, &map_kl, const_full, 0, 0, bh);
                     for (int kb = 0; kb < M / 64; ++kb)
                         tma_load_3d(sm + C::kOffWt + kb * C::kWtBlock, &map_wt, const_full, kb * 64, 0, bh);
@@ -154,9 +171,8 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 }
                 const int st = i % C::kStages, use = i / C::kStages;
                 if (!mbar_wait(&q_empty[st], (use & 1) ^ 1)) { *abort_flag = 1; break; }
-                mbar_arrive_expect_tx(&q_full[st], C::kQBytes + C::kVBytes);
+                mbar_arrive_expect_tx(&q_full[st], C::kQBytes);
                 tma_load_3d(sm + C::kOffQ + st * C::kQBytes, &map_q, &q_full[st], 0, row0, bh);
-                tma_load_3d(sm + C::kOffV + st * C::kVBytes, &map_v, &q_full[st], 0, row0 - 32, bh);
                 last_use[st] = use;
             }
             if (*abort_flag) {
@@ -165,6 +181,19 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (last_use[st] >= 0) mbar_wait(&q_full[st], last_use[st] & 1);
                 if (const_loads > 0) mbar_wait(const_full, (const_loads - 1) & 1);
             }
+        } else if (lane == 1 && prm.conv_w != nullptr) {
+            int last_use[2] = {-1, -1};
+            for (int i = 0; i < count && !*abort_flag; ++i) {
+                const int t = t0 + i, bh = t / tph, row0 = (t % tph) * C::kRows;
+                const int st = i % C::kStages, use = i / C::kStages;
+                if (!mbar_wait(&v_empty[st], (use & 1) ^ 1)) { *abort_flag = 1; break; }
+                mbar_arrive_expect_tx(&v_full[st], C::kVBytes);
+                tma_load_3d(sm + C::kOffV + st * C::kVBytes, &map_v, &v_full[st], 0, row0 - 32, bh);
+                last_use[st] = use;
+            }
+            if (*abort_flag)
+                for (int st = 0; st < 2; ++st)
+                    if (last_use[st] >= 0) mbar_wait(&v_full[st], last_use[st] & 1);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer
@@ -194,6 +223,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) mma_bf16_ss(slot, descQ(st, k), descKl(k), C::kIdS, k > 0);
                 mma_commit(&s_full[s]);
+                mma_commit(&q_empty[st]);
                 return true;
             };
             auto issue_O = [&](int j) -> bool {
@@ -202,15 +232,20 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 tc_fence_after();
                 const uint32_t slot = tmem + s * C::kSlot;
 #pragma unroll
-                for (int k = 0; k < M / 16; ++k)
-                    mma_bf16_ts(slot + C::kColOatt, slot + C::kColP + k * 8, descWt(k), C::kIdPW, k > 0);
+                for (int k = 0; k < M / 16; ++k) {
+                    // landmarks 16k .. 16k+15: first half from P_A, second half from P_B
+                    const uint32_t pa = k < M / 32 ? slot + C::kColPA + k * 8 : slot + C::kColPB + (k - M / 32) * 8;
+                    mma_bf16_ts(slot + C::kColOatt, pa, descWt(k), C::kIdPW, k > 0);
+                }
                 if (prm.conv_w != nullptr) {
+                    if (!mbar_wait(&v_full[st], (j / C::kStages) & 1)) return false;
+                    tc_fence_after();
 #pragma unroll
                     for (int k = 0; k < 12; ++k)
                         mma_bf16_ss(slot + C::kColOconv, descT(k), descV(st, k), C::kIdConv, k > 0);
                 }
                 mma_commit(&o_full[s]);
-                mma_commit(&q_empty[st]);
+                if (prm.conv_w != nullptr) mma_commit(&v_empty[st]);
                 return true;
             };
             if (count > 0) {
@@ -237,64 +272,78 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mma_commit(mma_done);
             mbar_wait(mma_done, 0);
         }
-    } else if (warp >= 2 && warp < 6) {
-        // ------------------------------------------------ softmax warpgroup
+    } else if (warp >= 2 && warp < 10) {
+        // ------------------------------------------------ softmax: two warpgroups, one tile,
+        // group g reads landmark columns [g M/2, g M/2 + M/2) of its row
+        constexpr int kHalf = M / 2;
+        const int g = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const float sc = split_scale(D) * kLog2e;  // S holds Q . K_l^T with K_l already scaled
         for (int i = 0; i < count && !warp_any(*abort_flag != 0); ++i) {
             const int s = i & 1;
-            if (!warp_all(mbar_wait(&s_full[s], (i >> 1) & 1))) { *abort_flag = 1; break; }
+            const bool ok = warp_all(mbar_wait(&s_full[s], (i >> 1) & 1));
+            // the whole group pair agrees before the exchange barrier below
+            if (group_any(!ok, 3, 256)) { *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
-            // pass 1: row max; up to four 32-column loads in flight per wait
-            constexpr int kNB1 = M >= 128 ? 4 : M / 32;
+            const uint32_t scol = slot + g * kHalf;
+            // pass 1: the max of this half-row, 64 columns per wait
+            constexpr int kB = kHalf < 64 ? kHalf : 64;
             float mx = -INFINITY;
 #pragma unroll 1
-            for (int c0 = 0; c0 < M; c0 += 32 * kNB1) {
-                uint32_t v[kNB1][32];
+            for (int c0 = 0; c0 < kHalf; c0 += kB) {
+                uint32_t v[kB / 32][32];
 #pragma unroll
-                for (int bq = 0; bq < kNB1; ++bq) tmem_ld32(slot + c0 + bq * 32, v[bq]);
+                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(scol + c0 + bq * 32, v[bq]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int bq = 0; bq < kNB1; ++bq)
+                for (int bq = 0; bq < kB / 32; ++bq)
 #pragma unroll
                     for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[bq][j]));
             }
+            pmax[(s * 2 + g) * 128 + r] = mx;
+            named_barrier(3, 256);
+            mx = fmaxf(mx, pmax[(s * 2 + (g ^ 1)) * 128 + r]);
             const float mo = mx * sc;
-            // pass 2: exponentials, 64 columns per wait, packed bf16 P into columns [c0/2, c0/2 + 32)
+            // pass 2: P into this group's own half of the S columns, in increasing column order,
+            // so it only overwrites scores this thread has already read
+            const uint32_t pcol = slot + (g == 0 ? C::kColPA : C::kColPB);
             float sum = 0.f;
 #pragma unroll 1
-            for (int c0 = 0; c0 < M; c0 += 64) {
-                uint32_t v[2][32];
-                tmem_ld32(slot + c0, v[0]);
-                tmem_ld32(slot + c0 + 32, v[1]);
-                tmem_ld_wait();
-                uint32_t pk[32];
+            for (int c0 = 0; c0 < kHalf; c0 += kB) {
+                uint32_t v[kB / 32][32];
 #pragma unroll
-                for (int bq = 0; bq < 2; ++bq)
+                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(scol + c0 + bq * 32, v[bq]);
+                tmem_ld_wait();
+#pragma unroll
+                for (int bq = 0; bq < kB / 32; ++bq) {
+                    uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const float p0 = ex2(fmaf(__uint_as_float(v[bq][2 * j]), sc, -mo));
-                        const float p1 = ex2(fmaf(__uint_as_float(v[bq][2 * j + 1]), sc, -mo));
-                        sum += p0 + p1;
-                        pk[bq * 16 + j] = pack_bf16(p0, p1);
+                        // bf16 P by truncation; the row sum adds the same truncated values, so
+                        // the weights P / sum(P) the MMA applies are normalised exactly
+                        const uint32_t u0 = __float_as_uint(ex2(fmaf(__uint_as_float(v[bq][2 * j]), sc, -mo))) & 0xFFFF0000u;
+                        const uint32_t u1 = __float_as_uint(ex2(fmaf(__uint_as_float(v[bq][2 * j + 1]), sc, -mo))) & 0xFFFF0000u;
+                        sum += __uint_as_float(u0) + __uint_as_float(u1);
+                        pk[j] = __byte_perm(u0, u1, 0x7632);
                     }
-                tmem_st32(slot + C::kColP + c0 / 2, pk);
+                    tmem_st16(pcol + (c0 + bq * 32) / 2, pk);
+                }
             }
             tmem_st_wait();
-            linv[s * 128 + r] = 1.f / sum;
+            psum[(s * 2 + g) * 128 + r] = sum;
             tc_fence_before();
             mbar_arrive(&p_full[s]);
         }
-    } else if (warp >= 6) {
+    } else if (warp >= 10) {
         // ------------------------------------------------ epilogue warpgroup (+ Toeplitz build)
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const bool conv = prm.conv_w != nullptr;
-        const bool leader = (warp == 6 && lane == 0);
+        const bool leader = (warp == 10 && lane == 0);
         uint32_t ce_phase = 0;
         for (int i = 0; i < count; ++i) {
             if (group_any(*abort_flag != 0, 2, 128)) break;
@@ -336,7 +385,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 break;
             }
             tc_fence_after();
-            const float li = linv[s * 128 + r];
+            const float li = 1.f / (psum[(s * 2) * 128 + r] + psum[(s * 2 + 1) * 128 + r]);
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
             uint32_t outp[D / 2];
 #pragma unroll
