@@ -20,6 +20,7 @@
 #include "tc_k3v.cuh"
 #include "tc_output.cuh"
 #include "tc_pinv.cuh"
+#include "tc_pinv_pair.cuh"
 
 namespace nys {
 namespace {
@@ -106,8 +107,20 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D bf16 tensor map over a row-major [d2][d1][d0] array, box b0 x b1 x 1,
-// out-of-bounds elements read as zero.
+// 3-D tensor map over a row-major [d2][d1][d0] array of `elt`-byte elements,
+// box b0 x b1 x 1, out-of-bounds elements read as zero.
+bool map_3d(CUtensorMap* m, CUtensorMapDataType dt, uint32_t elt, const void* base, uint64_t d0, uint64_t d1,
+            uint64_t d2, uint32_t b0, uint32_t b1, CUtensorMapSwizzle sw) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * elt, d0 * d1 * elt};
+    const cuuint32_t box[3] = {b0, b1, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0,
                  uint32_t b1, CUtensorMapSwizzle sw) {
     EncodeTiledFn fn = encode_fn();
@@ -360,10 +373,10 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(pinv_tc_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)C::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(kernel2_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
-                cudaSuccess ||
-            cudaFuncSetAttribute(kernel2_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
-                cudaSuccess)
+            cudaFuncSetAttribute(kernel2_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 96 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(kernel2_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 96 * 1024) != cudaSuccess)
             return NYS_ERR_CUDA;
         attr_set[dev] = true;
     }
@@ -374,9 +387,9 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     {
         ProfScope ps(K_KERNEL2, s);
         if (p.d == 64)
-            kernel2_kernel<64><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
+            kernel2_kernel<64, false><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
         else
-            kernel2_kernel<32><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
+            kernel2_kernel<32, false><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
     }
     PinvTcParams prm{k2b, k2tb, reinterpret_cast<uint8_t*>(ws + p.off_zb), reinterpret_cast<uint8_t*>(ws + p.off_ztb),
                      reinterpret_cast<uint8_t*>(ws + p.off_ta),
@@ -395,6 +408,65 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     cfg.numAttrs = 1;
     ProfScope ps(K_PINV, s);
     if (cudaLaunchKernelEx(&cfg, pinv_tc_kernel<M>, prm) != cudaSuccess) return NYS_ERR_CUDA;
+    return NYS_OK;
+}
+
+// m = 256: kernel_2 (row-major k2 / k2^T) and the CTA-pair inverse.
+int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, const float* kl, float* z, char* ws,
+                     cudaStream_t s) {
+    using C = PinvPair;
+    constexpr int M = 256;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const size_t smem2 = (size_t)(32 + M) * (p.d + 1) * sizeof(float);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(pinv_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess ||
+            cudaFuncSetAttribute(kernel2_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 96 * 1024) != cudaSuccess ||
+            cudaFuncSetAttribute(kernel2_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 96 * 1024) != cudaSuccess)
+            return NYS_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    float* k2 = reinterpret_cast<float*>(ws + p.off_k2b);
+    float* k2t = reinterpret_cast<float*>(ws + p.off_k2tb);
+    float* zs = reinterpret_cast<float*>(ws + p.off_zb);
+    float* colsum = reinterpret_cast<float*>(ws + p.off_colsum);
+    float* rowsum = reinterpret_cast<float*>(ws + p.off_rowsum);
+    {
+        ProfScope ps(K_KERNEL2, s);
+        if (p.d == 64)
+            kernel2_kernel<64, true><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2, k2t, colsum, rowsum, M);
+        else
+            kernel2_kernel<32, true><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2, k2t, colsum, rowsum, M);
+    }
+    PinvPairMaps maps;
+    const uint64_t BH = p.BH;
+    const auto f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    if (!map_3d(&maps.a_k2, f32, 4, k2, M, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.a_k2t, f32, 4, k2t, M, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.a_z, f32, 4, zs, M, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.z_out, f32, 4, z, M, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.b_k2, f32, 4, k2, M, M, BH, 32, 32, sw))
+        return NYS_ERR_CUDA;
+    PinvPairParams prm{colsum, rowsum, k2t, z, p.n_iter};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.BH * 2);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ProfScope ps(K_PINV, s);
+    if (cudaLaunchKernelEx(&cfg, pinv_pair_kernel, maps, prm) != cudaSuccess) return NYS_ERR_CUDA;
     return NYS_OK;
 }
 
@@ -428,7 +500,7 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     switch (m) {
         case 64: rc = launch_pinv_tc<64>(p, st, ql, kl, z, ws, st.aux); break;
         case 128: rc = launch_pinv_tc<128>(p, st, ql, kl, z, ws, st.aux); break;
-        case 256: rc = launch_pinv_tc<256>(p, st, ql, kl, z, ws, st.aux); break;
+        case 256: rc = launch_pinv_pair(p, st, ql, kl, z, ws, st.aux); break;
         default: return NYS_ERR_UNSUPPORTED;
     }
     if (rc != NYS_OK) return rc;

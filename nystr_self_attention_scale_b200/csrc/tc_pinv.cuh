@@ -49,10 +49,12 @@ __device__ __forceinline__ float tf32_rna(float x) {
 
 // ------------------------------------------------------------------ kernel_2 rows
 // grid (BH, m / 32), 256 threads. Dynamic shared memory: (32 + m) * (D + 1) floats.
-template <int D>
+// kPlain: k2 and k2^T are written row-major (for tensor-map loads); otherwise in
+// the blocked swizzled layout above (for plain bulk copies).
+template <int D, bool kPlain>
 __global__ void __launch_bounds__(256)
-kernel2_kernel(const float* __restrict__ ql, const float* __restrict__ kl, uint8_t* __restrict__ k2b,
-               uint8_t* __restrict__ k2tb, float* __restrict__ colsum_part, float* __restrict__ rowsum,
+kernel2_kernel(const float* __restrict__ ql, const float* __restrict__ kl, void* __restrict__ k2out,
+               void* __restrict__ k2tout, float* __restrict__ colsum_part, float* __restrict__ rowsum,
                int m) {
     extern __shared__ float sm2[];
     constexpr int d = D, ld = D + 1;
@@ -149,31 +151,56 @@ kernel2_kernel(const float* __restrict__ ql, const float* __restrict__ kl, uint8
         if (lane == 0) rowsum[(size_t)bh * m + r0 + r] = rs;
     }
     __syncthreads();
-    const size_t mat = (size_t)m * m * 4;
-    uint8_t* k2h = k2b + (size_t)bh * mat;
-    uint8_t* k2th = k2tb + (size_t)bh * mat;
-    // k2 rows r0..r0+31: 16-byte chunks
-    for (int e = tid; e < 32 * (m / 4); e += 256) {
-        const int r = e / (m / 4), c = (e % (m / 4)) * 4;
-        float4 v = make_float4(tf32_rna(ss[r * lds + c]), tf32_rna(ss[r * lds + c + 1]),
-                               tf32_rna(ss[r * lds + c + 2]), tf32_rna(ss[r * lds + c + 3]));
-        *reinterpret_cast<float4*>(k2h + bsw_offset(r0 + r, c, m)) = v;
-    }
-    // k2^T: column c of this block is row c of k2^T, atom blk (32 floats = one line)
-    for (int c = tid; c < m; c += 256) {
-        float cs = 0.f;
-#pragma unroll 4
-        for (int q = 0; q < 8; ++q) {
-            float4 v;
-            v.x = ss[(4 * q + 0) * lds + c];
-            v.y = ss[(4 * q + 1) * lds + c];
-            v.z = ss[(4 * q + 2) * lds + c];
-            v.w = ss[(4 * q + 3) * lds + c];
-            cs += (v.x + v.y) + (v.z + v.w);
-            v = make_float4(tf32_rna(v.x), tf32_rna(v.y), tf32_rna(v.z), tf32_rna(v.w));
-            *reinterpret_cast<float4*>(k2th + bsw_offset(c, r0 + 4 * q, m)) = v;
+    if constexpr (kPlain) {
+        float* k2h = reinterpret_cast<float*>(k2out) + (size_t)bh * m * m;
+        float* k2th = reinterpret_cast<float*>(k2tout) + (size_t)bh * m * m;
+        // k2 rows r0 .. r0+31, 16 bytes per thread and step
+        for (int e = tid; e < 32 * (m / 4); e += 256) {
+            const int r = e / (m / 4), c = (e % (m / 4)) * 4;
+            *reinterpret_cast<float4*>(k2h + (size_t)(r0 + r) * m + c) =
+                make_float4(tf32_rna(ss[r * lds + c]), tf32_rna(ss[r * lds + c + 1]),
+                            tf32_rna(ss[r * lds + c + 2]), tf32_rna(ss[r * lds + c + 3]));
         }
-        colsum_part[((size_t)bh * (m / 32) + blk) * m + c] = cs;
+        // k2^T rows c, columns r0 .. r0+31: eight threads write one 128-byte segment
+        for (int e = tid; e < m * 8; e += 256) {
+            const int c = e >> 3, q = e & 7;
+            *reinterpret_cast<float4*>(k2th + (size_t)c * m + r0 + 4 * q) =
+                make_float4(tf32_rna(ss[(4 * q) * lds + c]), tf32_rna(ss[(4 * q + 1) * lds + c]),
+                            tf32_rna(ss[(4 * q + 2) * lds + c]), tf32_rna(ss[(4 * q + 3) * lds + c]));
+        }
+        for (int c = tid; c < m; c += 256) {
+            float cs = 0.f;
+#pragma unroll 8
+            for (int rr = 0; rr < 32; ++rr) cs += ss[rr * lds + c];
+            colsum_part[((size_t)bh * (m / 32) + blk) * m + c] = cs;
+        }
+    } else {
+        const size_t mat = (size_t)m * m * 4;
+        uint8_t* k2h = reinterpret_cast<uint8_t*>(k2out) + (size_t)bh * mat;
+        uint8_t* k2th = reinterpret_cast<uint8_t*>(k2tout) + (size_t)bh * mat;
+        // k2 rows r0..r0+31: 16-byte chunks
+        for (int e = tid; e < 32 * (m / 4); e += 256) {
+            const int r = e / (m / 4), c = (e % (m / 4)) * 4;
+            float4 v = make_float4(tf32_rna(ss[r * lds + c]), tf32_rna(ss[r * lds + c + 1]),
+                                   tf32_rna(ss[r * lds + c + 2]), tf32_rna(ss[r * lds + c + 3]));
+            *reinterpret_cast<float4*>(k2h + bsw_offset(r0 + r, c, m)) = v;
+        }
+        // k2^T: column c of this block is row c of k2^T, atom blk (32 floats = one line)
+        for (int c = tid; c < m; c += 256) {
+            float cs = 0.f;
+#pragma unroll 4
+            for (int q = 0; q < 8; ++q) {
+                float4 v;
+                v.x = ss[(4 * q + 0) * lds + c];
+                v.y = ss[(4 * q + 1) * lds + c];
+                v.z = ss[(4 * q + 2) * lds + c];
+                v.w = ss[(4 * q + 3) * lds + c];
+                cs += (v.x + v.y) + (v.z + v.w);
+                v = make_float4(tf32_rna(v.x), tf32_rna(v.y), tf32_rna(v.z), tf32_rna(v.w));
+                *reinterpret_cast<float4*>(k2th + bsw_offset(c, r0 + 4 * q, m)) = v;
+            }
+            colsum_part[((size_t)bh * (m / 32) + blk) * m + c] = cs;
+        }
     }
 }
 
