@@ -104,7 +104,7 @@ def compute_peak_tflops(unit, peaks, kernel_impl_simt):
     if unit == "alu" or kernel_impl_simt:
         return N_SMS * FP32_LANES_PER_SM * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
     if unit == "tensor_tf32":
-        return peaks["bf16_tflops"] * 0.5   # nominal tf32 : bf16 dense ratio 1.1 : 2.25
+        return peaks["bf16_tflops"] * 1.1 / 2.25   # nominal dense tf32 : bf16 = 1.1 : 2.25 PFLOP/s
     return peaks["bf16_tflops"]
 
 
