@@ -446,13 +446,11 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
     const uint64_t BH = p.BH;
     const auto f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!map_3d(&maps.a_k2, f32, 4, k2, M, M, BH, 32, 128, sw) ||
-        !map_3d(&maps.a_k2t, f32, 4, k2t, M, M, BH, 32, 128, sw) ||
-        !map_3d(&maps.a_z, f32, 4, zs, M, M, BH, 32, 128, sw) ||
-        !map_3d(&maps.z_out, f32, 4, z, M, M, BH, 32, 128, sw) ||
-        !map_3d(&maps.b_k2, f32, 4, k2, M, M, BH, 32, 32, sw))
+    if (!map_3d(&maps.k2, f32, 4, k2, M, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.k2t, f32, 4, k2t, M, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.wt, f32, 4, zs, M, M, BH, 32, 128, sw))
         return NYS_ERR_CUDA;
-    PinvPairParams prm{colsum, rowsum, k2t, z, p.n_iter};
+    PinvPairParams prm{colsum, rowsum, k2, k2t, zs, z, p.n_iter};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.BH * 2);
     cfg.blockDim = dim3(C::kThreads);

@@ -3,30 +3,36 @@
 // Walkthrough (blog.gitcode.com) 2.5: Z_0 = c k2^T, then n_iter times
 //   X = k2 Z;  T1 = 7I - X;  T3 = 15I - X T1;  T5 = 13I - X T3;  Z = Z T5 / 4.
 //
-// One head per cluster of two CTAs, and every product is one 2-CTA tcgen05 MMA
-// (cta_group::2, M = N = 256, tf32): CTA r supplies rows 128r .. 128r+127 of
-// the left factor A and receives the same rows of the product D in its TMEM,
-// and it holds half of the right factor B in its shared memory: columns
-// 128r .. 128r+127, as 128 K-major lines of 256 tf32 values (128 KB).
+// Two exact identities shape the kernel. (1) T1, T3 and T5 are polynomials in
+// X, so they commute with X. (2) Transposing the update gives W = Z^T with
+// W_0 = c k2, X^T = W k2^T and W <- T5(X^T) W / 4, where T5(X^T) is the same
+// polynomial taken in X^T. The kernel iterates in X^T (called X below)
+//   P1: X = W k2^T    P2: U = T1 X    P3: V = T3 X    P4: W = T5 W / 4
+// (equal to the page's sequence in real arithmetic) and takes every left
+// factor from TMEM: W is the raw accumulator of the previous P4, and each T is
+// written back to TMEM by the epilogue that forms it (tf32-rounded). The right
+// factors live in shared memory as K-major lines: X, written once per
+// iteration by the P1 epilogue column by column into the B half of the CTA
+// that owns the column (its own or, through distributed shared memory, the
+// peer's) -- X is symmetric only in exact arithmetic, and using its rows as
+// its columns loses accuracy on ill-conditioned k2 -- and, streamed from L2 one
+// 32-wide K atom at a time behind the previous product's MMAs, the rows of k2
+// (for P1) and the columns of W (for P4; the P4 epilogue writes W^T row-major
+// to scratch).
 //
-// The right factor of every product is produced by the epilogue of the
-// previous one (T1, T3, T5, and Z for the next X = k2 Z), so it never leaves
-// the chip: each thread owns one row of D, applies the affine step (scale and
-// identity shift), rounds to tf32 and stores the row, column by column, into
-// the B lines of whichever CTA owns that column -- its own shared memory or the
-// peer's through distributed shared memory. X = k2 Z stays in TMEM and is the
-// A operand of the next two products. The A operands that are not products of
-// this iteration -- rows of k2 (for X = k2 Z) and rows of Z (for Z T5) -- are
-// streamed in 32-column chunks by TMA through a 3-stage ring; the new rows of
-// Z go back to L2-resident scratch with TMA stores during the same epilogue.
+// One head per cluster of two CTAs, one 2-CTA tcgen05 MMA per K step
+// (cta_group::2, kind::tf32, M = N = 256): CTA r holds rows 128r .. 128r+127 of
+// A and D in its TMEM and lines (columns) 128r .. 128r+127 of B in its shared
+// memory. TMEM: R0 = columns 0..255, R1 = 256..511; per iteration
+//   P1: A = R0 (W), D -> R1;  P2: A = R1 (T1), D -> R0;
+//   P3: A = R0 (T3), D -> R1; P4: A = R1 (T5), D -> R0 (the next W).
+// Scale factors are folded into the epilogues: the stored W is the raw P4
+// accumulator (sigma = c for W_0 = c k2 loaded unscaled, c/4 after the first
+// P4, 1/4 afterwards).
 //
-// Iteration 0 never forms Z_0 = c k2^T: its B operand is loaded as rows of k2,
-// its A rows come from k2^T, and c is applied in the epilogues (X = c k2 k2^T
-// is kept unscaled in TMEM, so T3 and T5 take the factor c too).
-//
-// Roles (320 threads): warps 0-7 epilogue (warp w reads TMEM lanes 32 (w % 4)
-// and columns of half w / 4), warp 8 lane 0 TMA producer (both CTAs), warp 9
-// TMEM allocation (both CTAs) and, in CTA 0 only, the MMA issuer.
+// Roles (320 threads): warps 0-7 epilogue (warp w: TMEM lanes 32 (w % 4),
+// columns 128 (w / 4) ..), warp 8 lane 0 TMA producer (both CTAs), warp 9 TMEM
+// allocation (both CTAs) and, in CTA 0, the MMA issuer.
 #pragma once
 
 #include "sm100.cuh"
@@ -125,33 +131,31 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
 }  // namespace pair2
 
 struct PinvPairMaps {
-    CUtensorMap a_k2;    // k2  [BH][256][256] fp32, box 32 x 128, 128-byte swizzle: A chunks
-    CUtensorMap a_k2t;   // k2^T, same box: A chunks of Z_0 = c k2^T
-    CUtensorMap a_z;     // Z scratch, same box: A chunks of Z and the TMA stores of new Z rows
-    CUtensorMap z_out;   // the result, same box (stores)
-    CUtensorMap b_k2;    // k2, box 32 x 32, 128-byte swizzle: the first right factor Z_0 (rows of k2)
+    CUtensorMap k2;    // k2   [BH][256][256] fp32, box 32 x 128, 128-byte swizzle: B atoms of P1
+    CUtensorMap k2t;   // k2^T, same box: B atoms of the first P4 (columns of W_0 = c k2)
+    CUtensorMap wt;    // W^T scratch, same box: B atoms of the later P4s
 };
 
 struct PinvPairParams {
     const float* colsum_part;  // [BH][8][256] column sums of k2 per 32-row block
     const float* rowsum;       // [BH][256]
+    const float* k2;           // [BH][256][256] (rows of W_0, loaded into TMEM)
     const float* k2t;          // [BH][256][256] (n_iter = 0 only)
-    float* z_out;              // [BH][256][256] (n_iter = 0 only)
+    float* wt;                 // [BH][256][256] W^T scratch (row g = column g of W)
+    float* z_out;              // [BH][256][256]
     int n_iter;
 };
 
 struct PinvPair {
     static constexpr int M = 256;
-    static constexpr int kStages = 3;
-    static constexpr uint32_t kAtomBytes = 128 * 128;             // 128 lines x 32 tf32
-    static constexpr uint32_t kBBytes = 8 * kAtomBytes;           // 8 K-atoms
-    static constexpr uint32_t kAChunk = 128 * 128;                // 128 rows x 32 tf32
-    static constexpr uint32_t kOffRing = kBBytes;
-    static constexpr uint32_t kOffStage = kOffRing + kStages * kAChunk;   // two 16 KB store-staging tiles
-    static constexpr uint32_t kOffBar = kOffStage + 2 * kAChunk;
-    // barriers: full[3], empty[3], mma_done, b_ready, b_init, z_ready, drain
-    static constexpr uint32_t kOffMisc = kOffBar + 16 * 8;
-    static constexpr uint32_t kSmemBytes = kOffMisc + 64 + 1024;
+    static constexpr uint32_t kAtomBytes = 128 * 128;          // 128 lines x 32 tf32
+    static constexpr uint32_t kBBytes = 8 * kAtomBytes;        // 8 K atoms = 128 KB
+    static constexpr uint32_t kOffBar = kBBytes;
+    // barriers: bfull[8], bfree[8], mma_done, mma4_done, e_ready, wl_ready, drain
+    static constexpr uint32_t kOffMisc = kOffBar + 24 * 8;
+    static constexpr uint32_t kSmemNeed = kOffMisc + 64 + 1024;
+    // more than half of the SM's shared memory: no other CTA (and no other TMEM user) shares the SM
+    static constexpr uint32_t kSmemBytes = kSmemNeed < 200 * 1024 ? 200 * 1024 : kSmemNeed;
     static constexpr int kThreads = 320;
     static constexpr uint32_t kIdesc = sm100::make_idesc(256, 256, sm100::kFmtTf32, sm100::kFmtTf32, 0, 0);
 };
@@ -166,15 +170,13 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* bbuf = sm;
-    uint8_t* ring = sm + C::kOffRing;
-    uint8_t* stage = sm + C::kOffStage;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + C::kOffBar);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* mma_done = empty + C::kStages;
-    uint64_t* b_ready = mma_done + 1;
-    uint64_t* b_init = b_ready + 1;
-    uint64_t* z_ready = b_init + 1;
-    uint64_t* drain = z_ready + 1;
+    uint64_t* bfull = reinterpret_cast<uint64_t*>(sm + C::kOffBar);   // [8], used in CTA 0
+    uint64_t* bfree = bfull + 8;                                       // [8], both CTAs (after P3, P4)
+    uint64_t* mma_done = bfree + 8;      // P1..P3 accumulators complete (both CTAs)
+    uint64_t* mma4_done = mma_done + 1;  // P4 accumulator complete (both CTAs)
+    uint64_t* e_ready = mma4_done + 1;   // epilogue output in place for the next product (CTA 0)
+    uint64_t* wl_ready = e_ready + 1;    // W^T scratch written by both CTAs (each CTA)
+    uint64_t* drain = wl_ready + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     float* red = reinterpret_cast<float*>(sm + C::kOffMisc + 16);   // [8]
 
@@ -185,14 +187,14 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     const int r0 = (int)rank * 128;
 
     if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < 8; ++s) {
+            mbar_init(&bfull[s], 1);
+            mbar_init(&bfree[s], 1);
         }
         mbar_init(mma_done, 1);
-        mbar_init(b_ready, 16);    // one arrival per epilogue warp of either CTA
-        mbar_init(b_init, 1);
-        mbar_init(z_ready, 2);
+        mbar_init(mma4_done, 1);
+        mbar_init(e_ready, 16);    // one arrival per epilogue warp of either CTA
+        mbar_init(wl_ready, 16);
         mbar_init(drain, 1);
         fence_mbar_init();
     }
@@ -224,7 +226,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     const float coeff = 1.f / (fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) *
                                fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
     const uint32_t tmem = *tmem_slot;
-    const uint32_t tA = tmem, tB = tmem + 256;   // X (A operand of two products) / product accumulators
+    const uint32_t R0 = tmem, R1 = tmem + 256;
     const int n_iter = prm.n_iter;
 
     if (n_iter == 0) {
@@ -239,31 +241,28 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     } else if (warp == 8) {
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
-            prefetch_tmap(&maps.a_k2);
-            prefetch_tmap(&maps.a_k2t);
-            prefetch_tmap(&maps.a_z);
-            prefetch_tmap(&maps.b_k2);
-            const uint32_t full0 = mapa(smem_u32(full), 0);
-            // B line n of this CTA is column 128 rank + n of Z_0, i.e. row 128 rank + n of k2
-            mbar_arrive_expect_tx(b_init, C::kBBytes);
-            for (int a = 0; a < 8; ++a)
-                for (int j = 0; j < 4; ++j)
-                    tma_load_3d(bbuf + a * C::kAtomBytes + j * 4096, &maps.b_k2, b_init, 32 * a, r0 + 32 * j, bh);
+            prefetch_tmap(&maps.k2);
+            prefetch_tmap(&maps.k2t);
+            prefetch_tmap(&maps.wt);
+            const uint32_t bfull0 = mapa(smem_u32(bfull), 0);
             bool ok = true;
-            uint32_t g = 0;
             for (int it = 0; it < n_iter && ok; ++it) {
                 for (int part = 0; part < 2 && ok; ++part) {
-                    const CUtensorMap* mp = part == 0 ? &maps.a_k2 : (it == 0 ? &maps.a_k2t : &maps.a_z);
-                    if (part == 1 && it > 0) {
-                        ok = mbar_wait(z_ready, (uint32_t)(it - 1) & 1u);   // this CTA's new Z rows are stored
+                    const int p = part == 0 ? 0 : 3;
+                    const CUtensorMap* mp = p == 0 ? &maps.k2 : (it == 0 ? &maps.k2t : &maps.wt);
+                    if (p == 3 && it > 0) {
+                        ok = wait_acq_cluster(wl_ready, (uint32_t)(it - 1) & 1u);   // W^T of both CTAs stored
                         fence_proxy_async_global();
                     }
-                    for (int kc = 0; kc < 8 && ok; ++kc, ++g) {
-                        const uint32_t st = g % C::kStages;
-                        ok = mbar_wait(&empty[st], ((g / C::kStages) & 1u) ^ 1u);
+                    for (int kc = 0; kc < 8 && ok; ++kc) {
+                        // K atom kc is free once the previous product (P3 before P4, P4 before the
+                        // next P1) has read it. bfree[kc] completes twice per iteration, after
+                        // P3 and after P4, and never runs ahead of these loads by more than one
+                        // phase, so its parity is exact.
+                        if (it > 0 || p == 3) ok = mbar_wait(&bfree[kc], p == 3 ? 0u : 1u);
                         if (!ok) break;
-                        if (leader) mbar_arrive_expect_tx(&full[st], 2 * C::kAChunk);
-                        tma_load_3d_pair(ring + st * C::kAChunk, mp, full0 + 8 * st, 32 * kc, r0, bh);
+                        if (leader) mbar_arrive_expect_tx(&bfull[kc], 2 * C::kAtomBytes);
+                        tma_load_3d_pair(bbuf + kc * C::kAtomBytes, mp, bfull0 + 8 * kc, 32 * kc, r0, bh);
                     }
                 }
             }
@@ -272,42 +271,35 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer (first CTA of the pair)
         if (leader && lane == 0) {
-            const uint32_t bs = smem_u32(bbuf), rs = smem_u32(ring);
+            const uint32_t bs = smem_u32(bbuf);
             bool ok = true;
-            uint32_t g = 0, nb = 0;
+            uint32_t ne = 0, nf = 0;   // e_ready phases waited, streamed products issued
             for (int it = 0; it < n_iter && ok; ++it) {
                 for (int p = 0; p < 4 && ok; ++p) {
-                    ok = wait_acq_cluster(b_ready, nb & 1u);   // B of this product in place, last D read
-                    ++nb;
-                    if (!ok) break;
+                    const uint32_t a_col = (p == 0 || p == 2) ? R0 : R1;
+                    const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
+                    const bool streamed = p == 0 || p == 3;
+                    if (p != 0 || it == 0) {
+                        ok = wait_acq_cluster(e_ready, ne & 1u);   // left factor (and X) in place
+                        ++ne;
+                        if (!ok) break;
+                    }
                     tc_fence_after();
-                    const bool from_ring = p == 0 || p == 3;
-                    const uint32_t d = p == 0 ? tA : tB;
                     for (int kc = 0; kc < 8; ++kc) {
-                        uint32_t sa = 0, st = 0;
-                        if (from_ring) {
-                            st = g % C::kStages;
-                            ok = mbar_wait(&full[st], (g / C::kStages) & 1u);
+                        if (streamed) {
+                            ok = mbar_wait(&bfull[kc], nf & 1u);
                             if (!ok) break;
                             tc_fence_after();
-                            sa = rs + st * C::kAChunk;
                         }
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bdesc =
-                                smem_desc(bs + kc * C::kAtomBytes + kk * 32, 16, 1024, kLayoutSw128);
-                            const uint32_t acc = (kc | kk) != 0 ? 1u : 0u;
-                            if (from_ring)
-                                mma2_ss(d, smem_desc(sa + kk * 32, 16, 1024, kLayoutSw128), bdesc, C::kIdesc, acc);
-                            else
-                                mma2_ts(d, tA + kc * 32 + kk * 8, bdesc, C::kIdesc, acc);
-                        }
-                        if (from_ring) {
-                            commit2(&empty[st], 3);
-                            ++g;
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma2_ts(d_col, a_col + kc * 32 + kk * 8,
+                                    smem_desc(bs + kc * C::kAtomBytes + kk * 32, 16, 1024, kLayoutSw128), C::kIdesc,
+                                    (kc | kk) != 0 ? 1u : 0u);
+                        if (p >= 2) commit2(&bfree[kc], 3);   // the producer refills this atom next
                     }
-                    if (ok) commit2(mma_done, 3);
+                    if (streamed) ++nf;
+                    if (ok) commit2(p == 3 ? mma4_done : mma_done, 3);
                 }
             }
             // every MMA issued here has completed before the pair tears down
@@ -318,107 +310,126 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     } else {
         // ------------------------------------------------ epilogue (warps 0-7, both CTAs)
         const int q = warp & 3, h = warp >> 2;      // TMEM lane quadrant, column half
-        const int lt = tid & 127;                   // thread index within the half
-        const int row = r0 + 32 * q + lane;         // this thread's row of every product
+        const int lrow = 32 * q + lane;             // TMEM lane = this CTA's row = its B line
+        const int row = r0 + lrow;                  // global row of every product
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        const uint32_t b_ready0 = mapa(smem_u32(b_ready), 0);
-        // columns 128 h .. 128 h + 127 of every product belong to the B half of CTA h
-        const bool to_local = (uint32_t)h == rank;
-        const uint32_t b_dst = to_local ? smem_u32(bbuf) : mapa(smem_u32(bbuf), rank ^ 1u);
-        // byte offset of (this row's K position) inside a B line of column i, for i % 8 = 0..7
+        const uint32_t e_ready0 = mapa(smem_u32(e_ready), 0);
+        const uint32_t wl_loc = mapa(smem_u32(wl_ready), rank), wl_rem = mapa(smem_u32(wl_ready), rank ^ 1u);
+        // X lines: columns 128 h .. 128 h + 127 belong to CTA h's B half
+        const bool x_local = (uint32_t)h == rank;
+        const uint32_t x_dst = x_local ? smem_u32(bbuf) : mapa(smem_u32(bbuf), rank ^ 1u);
         const uint32_t k_off = (uint32_t)(4 * (int)rank + q) * C::kAtomBytes + (uint32_t)(lane & 3) * 4u;
         const uint32_t xl = (uint32_t)(lane >> 2);
-        uint8_t* stg = stage + h * C::kAChunk;
-        const int bar_stage = 1 + h;                 // named barrier of this half's 128 threads
-
-        bool failed = !mbar_wait(b_init, 0);
-        failed = group_any(failed, 3, 256);
-        if (!failed) {
+        const bool diag_half = (uint32_t)h == rank;  // this half's columns hold the diagonal element
+        const int diag_atom = 4 * h + q;             // (only when diag_half)
+        auto arrive_e = [&]() {
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) arrive_cluster(b_ready0);
+            if (lane == 0) arrive_cluster(e_ready0);
+        };
+
+        // W_0 = c k2: rows of k2 (unscaled) into R0
+#pragma unroll 1
+        for (int jj = 0; jj < 4; ++jj) {
+            const int a = 4 * h + jj;
+            const float4* src = reinterpret_cast<const float4*>(prm.k2 + ((size_t)bh * M + row) * M + 32 * a);
+            uint32_t v[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 f = __ldg(src + c);
+                v[4 * c] = __float_as_uint(f.x); v[4 * c + 1] = __float_as_uint(f.y);
+                v[4 * c + 2] = __float_as_uint(f.z); v[4 * c + 3] = __float_as_uint(f.w);
+            }
+            tmem_st32(R0 + lane_base + 32 * a, v);
         }
-        uint32_t nprod = 0;
+        tmem_st_wait();
+        arrive_e();
+
+        bool failed = false;
+        uint32_t nd = 0, n4 = 0;   // mma_done / mma4_done phases waited
         for (int it = 0; it < n_iter && !failed; ++it) {
-            const float s_it = it == 0 ? coeff : 1.f;
+            const float sigma = it == 0 ? coeff : (it == 1 ? 0.25f * coeff : 0.25f);
+            const float lambda = it == 0 ? 0.25f * coeff : 0.25f;
+            const bool last_it = it + 1 == n_iter;
             for (int p = 0; p < 4 && !failed; ++p) {
-                const bool ok = mbar_wait(mma_done, nprod & 1u);
-                ++nprod;
+                const bool ok = p == 3 ? mbar_wait(mma4_done, (n4++) & 1u) : mbar_wait(mma_done, (nd++) & 1u);
                 failed = group_any(!ok, 3, 256);
                 if (failed) break;
                 tc_fence_after();
-                const bool last = it + 1 == n_iter && p == 3;
-                const uint32_t d = p == 0 ? tA : tB;
-                const float alpha = p == 3 ? 0.25f * s_it : -s_it;
-                const float diag = p == 0 ? 7.f : (p == 1 ? 15.f : (p == 2 ? 13.f : 0.f));
-                const CUtensorMap* zmap = last ? &maps.z_out : &maps.a_z;
+                const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
+                const float alpha = p == 0 ? -sigma : -1.f;
+                const float diag = p == 0 ? 7.f : (p == 1 ? 15.f : 13.f);
 #pragma unroll 1
                 for (int jj = 0; jj < 4; ++jj) {
-                    const int a = 4 * h + jj;             // 32-column atom of D
+                    const int a = 4 * h + jj;   // 32-column atom
                     uint32_t v[32];
-                    tmem_ld32(d + lane_base + a * 32, v);
+                    tmem_ld32(d_col + lane_base + 32 * a, v);
                     tmem_ld_wait();
-                    float e[32];
+                    if (p == 3) {
+                        // W_next = lambda D: its transpose, row-major (row g = column g of W), is both
+                        // the next P4's right factor and, transposed back, the result Z = W^T
+                        float* dst = last_it ? prm.z_out : prm.wt;
+                        float* col = dst + (size_t)bh * M * M + (size_t)(32 * a) * M + row;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) e[i] = alpha * __uint_as_float(v[i]);
-                    if (a == (row >> 5)) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) e[i] += i == lane ? diag : 0.f;
+                        for (int i = 0; i < 32; ++i) {
+                            const float w = lambda * __uint_as_float(v[i]);
+                            col[(size_t)i * M] = last_it ? w : tf32_rna(w);
+                        }
+                        continue;
                     }
-                    if (!last) {
+                    float e[32];
+                    if (p == 0) {
+                        // X = sigma D is the right factor of P2 and P3 as K-major lines: column
+                        // g = 32 a + i of X is line 32 (a % 4) + i of CTA a / 4 (= h), and this
+                        // thread's row is K position `row` of every line
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) e[i] = tf32_rna(e[i]);
-                        // column 32 a + i is line 32 (a % 4) + i of CTA h's B half
-                        const uint32_t base = b_dst + k_off + (uint32_t)(a & 3) * 4096u;
-                        if (to_local) {
+                        for (int i = 0; i < 32; ++i) e[i] = sigma * __uint_as_float(v[i]);
+                        const uint32_t base = x_dst + k_off + (uint32_t)(a & 3) * 4096u;
+                        if (x_local) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
-                                st_local(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), e[i]);
+                                st_local(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), tf32_rna(e[i]));
                         } else {
 #pragma unroll
                             for (int i = 0; i < 32; ++i)
-                                st_remote(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), e[i]);
+                                st_remote(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), tf32_rna(e[i]));
                         }
-                    }
-                    if (p == 3) {
-                        // this half's staging tile -> TMA store of rows r0.., columns 32 a ..
-                        if (jj > 0) {
-                            if (lt == 0) tma_store_wait_read<0>();
-                            named_barrier(bar_stage, 128);
-                        }
-                        const int srow = 32 * q + lane;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c)
-                            *reinterpret_cast<float4*>(stg + swz<128>(srow, c)) =
-                                make_float4(e[4 * c], e[4 * c + 1], e[4 * c + 2], e[4 * c + 3]);
-                        fence_proxy_async_shared();
-                        named_barrier(bar_stage, 128);
-                        if (lt == 0) {
-                            tma_store_3d(zmap, stg, 32 * a, r0, bh);
-                            tma_store_commit();
+                        for (int i = 0; i < 32; ++i) e[i] = -e[i];
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) e[i] = alpha * __uint_as_float(v[i]);
+                    }
+                    // T = diag I + alpha D, back into TMEM as the next left factor
+                    if (diag_half && a == diag_atom) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) e[i] += i == lane ? diag : 0.f;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(tf32_rna(e[i]));
+                    tmem_st32(d_col + lane_base + 32 * a, v);
+                }
+                if (p == 3) {
+                    if (!last_it) {
+                        fence_proxy_async_global();   // W^T is read next by TMA
+                        __syncwarp();
+                        if (lane == 0) {
+                            arrive_cluster(wl_rem);
+                            arrive_cluster(wl_loc);
                         }
                     }
-                }
-                if (p == 0 && it > 0 && lt == 0) {
-                    // the Z rows stored at the end of the previous iteration are in L2 before the
-                    // producer streams them back as the A operand of Z T5
-                    tma_store_wait_all<0>();
-                    fence_proxy_async_global();
-                    mbar_arrive(z_ready);
-                }
-                if (!last) {
-                    fence_proxy_async_cluster();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) arrive_cluster(b_ready0);
+                } else {
+                    tmem_st_wait();
+                    if (p == 0) fence_proxy_async_cluster();   // X lines (here and in the peer) feed the MMA
+                    arrive_e();
                 }
             }
         }
-        if (lt == 0) tma_store_wait_all<0>();
     }
 
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();   // no remote store, arrive or MMA of either CTA is still pending
+    cluster_sync_all();   // no arrive or MMA of either CTA is still pending
     if (warp == 9) {
         tc_fence_after();
         tmem_dealloc2(tmem, 512);
