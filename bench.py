@@ -9,7 +9,9 @@ the workload, through the C ABI (nys_attn_forward). Default workload: the
 n=16384 bf16 correlated-token shape (B=4, H=8, d=64, m=256, conv on).
 
 Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
-(a 256 MiB device write, outside the timed interval) and bracketed by CUDA
+(a 256 MiB device write followed by a 256 MiB read of another buffer, so that
+no dirty lines are left to be written back during the step; outside the
+timed interval) and bracketed by CUDA
 events on the launching stream; a barrier and a device synchronisation on
 both sides; the maximum over ranks is reported. Per-kernel device times come
 from CUDA events the library records around each launch during the same
@@ -334,14 +336,22 @@ def main():
     conv_w = None if x["conv_w"] is None else torch.from_numpy(x["conv_w"]).cuda()
     out = torch.empty_like(q)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_clean = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush_sink = torch.empty(1, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
+
+    def flush_l2():
+        # evict the step's inputs by writing a buffer larger than L2, then read another one so
+        # that the written lines are written back here, untimed, and not during the next step
+        flush.zero_()
+        torch.sum(flush_clean, dim=0, keepdim=True, out=flush_sink)
 
     def step():
         nys.forward(q, k, v, mask=mask, conv_w=conv_w, m=w.m, n_iter=w.n_iter, out=out)
 
     for _ in range(args.warmup):
         if not args.no_flush:
-            flush.zero_()
+            flush_l2()
         step()
     torch.cuda.synchronize()
     assert nys.device_status() == 0
@@ -361,7 +371,7 @@ def main():
     nys.profile_enable(True)
     for i in range(args.steps):
         if not args.no_flush:
-            flush.zero_()
+            flush_l2()
         starts[i].record(stream)
         step()
         ends[i].record(stream)
@@ -449,7 +459,8 @@ def main():
             "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "m": w.m,
                        "n_iter": w.n_iter, "conv": w.conv, "mask": w.lengths is not None,
                        "inputs": w.dist, "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "not flushed" if args.no_flush else "flushed before every step (256 MiB write, untimed)"},
+                       "l2": "not flushed" if args.no_flush else
+                       "flushed before every step (256 MiB write, then a 256 MiB read of another buffer; untimed)"},
             "roofline": roof,
             "step_roofline": {"t_roof_us": round(t_roof * 1e6, 2), "frac": round(t_roof / (ms_per_step * 1e-3), 4),
                               "ideal_bytes": ideal_bytes, "flops": total_flops},

@@ -166,6 +166,17 @@ const char* nys_strerror(int status);
 int nys_attn_version(void);
 
 /*
+ * Self-test of the FMA-pipe 2^x approximation that the bf16 softmax passes
+ * use for part of their exponentials (the pages fix no exponential; this is
+ * an implementation check, with no counterpart in them). Evaluates it on
+ * 2^20 evenly spaced points of [-125, 8] on the current device and writes
+ * the maximum relative error against CUDA's exp2f to *max_rel_err (host
+ * pointer). Synchronous. NYS_ERR_INVALID_ARG for a null pointer,
+ * NYS_ERR_CUDA on a CUDA failure.
+ */
+int nys_attn_selftest_exp2(float* max_rel_err);
+
+/*
  * Per-kernel timing, for benchmarks. While enabled, each kernel launch of
  * the forward is bracketed by two CUDA events recorded on the stream the
  * kernel runs on. nys_attn_profile_enable() clears the counters (and turns

@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
     lib.nys_attn_kernel_name.restype = ctypes.c_char_p
     lib.nys_attn_pinv_static.argtypes = [vp, vp, vp, i, i, i, i, vp]
     lib.nys_attn_pinv_static.restype = i
+    lib.nys_attn_selftest_exp2.argtypes = [ctypes.POINTER(ctypes.c_float)]
+    lib.nys_attn_selftest_exp2.restype = i
     lib.nys_strerror.argtypes = [i]
     lib.nys_strerror.restype = ctypes.c_char_p
     return lib
@@ -179,6 +181,13 @@ def forward_host(q, k, v, mask=None, conv_w=None, m: int = DEFAULT_NUM_LANDMARKS
 def device_status() -> int:
     """Synchronise and return (and clear) the library's device status word."""
     return int(lib.nys_attn_device_status())
+
+
+def selftest_exp2() -> float:
+    """Maximum relative error of the library's FMA-pipe 2^x against CUDA's exp2f on [-125, 8]."""
+    err = ctypes.c_float(0.0)
+    _check(lib.nys_attn_selftest_exp2(ctypes.byref(err)), "nys_attn_selftest_exp2")
+    return float(err.value)
 
 
 def workspace_bytes(B, H, n, d, m, dtype_code=BF16) -> int:

@@ -11,6 +11,7 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <vector>
 
@@ -329,7 +330,7 @@ int launch_output_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* 
         attr_set[dev] = true;
     }
     ProfScope ps(K_OUTPUT, s);
-    output_tc_kernel<D, M><<<grid, 448, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
+    output_tc_kernel<D, M><<<grid, 480, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
     return NYS_OK;
 }
 
@@ -358,7 +359,7 @@ int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql1
         attr_set[dev] = true;
     }
     ProfScope ps(K_K3V, s);
-    k3v_tc_kernel<D><<<grid, 384, C::kSmemBytes, s>>>(mql, mk, mv, prm);
+    k3v_tc_kernel<D><<<grid, C::kThreads, C::kSmemBytes, s>>>(mql, mk, mv, prm);
     return NYS_OK;
 }
 
@@ -411,7 +412,7 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     return NYS_OK;
 }
 
-// m = 256: kernel_2 (row-major k2 / k2^T) and the CTA-pair inverse.
+// m = 256: kernel_2 and the iterative inverse in one CTA-pair kernel.
 int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, const float* kl, float* z, char* ws,
                      cudaStream_t s) {
     using C = PinvPair;
@@ -419,38 +420,26 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);
-    const size_t smem2 = (size_t)(32 + M) * (p.d + 1) * sizeof(float);
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(pinv_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(kernel2_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 96 * 1024) != cudaSuccess ||
-            cudaFuncSetAttribute(kernel2_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 96 * 1024) != cudaSuccess)
+                                 (int)C::kSmemBytes) != cudaSuccess)
             return NYS_ERR_CUDA;
         attr_set[dev] = true;
     }
     float* k2 = reinterpret_cast<float*>(ws + p.off_k2b);
     float* k2t = reinterpret_cast<float*>(ws + p.off_k2tb);
     float* zs = reinterpret_cast<float*>(ws + p.off_zb);
-    float* colsum = reinterpret_cast<float*>(ws + p.off_colsum);
-    float* rowsum = reinterpret_cast<float*>(ws + p.off_rowsum);
-    {
-        ProfScope ps(K_KERNEL2, s);
-        if (p.d == 64)
-            kernel2_kernel<64, true><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2, k2t, colsum, rowsum, M);
-        else
-            kernel2_kernel<32, true><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2, k2t, colsum, rowsum, M);
-    }
     PinvPairMaps maps;
     const uint64_t BH = p.BH;
     const auto f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-    if (!map_3d(&maps.k2, f32, 4, k2, M, M, BH, 32, 128, sw) ||
+    if (!map_3d(&maps.ql, f32, 4, ql, p.d, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.kl, f32, 4, kl, p.d, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.k2, f32, 4, k2, M, M, BH, 32, 128, sw) ||
         !map_3d(&maps.k2t, f32, 4, k2t, M, M, BH, 32, 128, sw) ||
         !map_3d(&maps.wt, f32, 4, zs, M, M, BH, 32, 128, sw))
         return NYS_ERR_CUDA;
-    PinvPairParams prm{colsum, rowsum, k2, k2t, zs, z, p.n_iter};
+    PinvPairParams prm{k2, k2t, zs, z, p.d, p.n_iter};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.BH * 2);
     cfg.blockDim = dim3(C::kThreads);
@@ -692,6 +681,38 @@ const char* nys_strerror(int status) {
 }
 
 int nys_attn_version(void) { return 100; }
+
+namespace nys {
+__global__ void exp2_selftest_kernel(int n, float lo, float hi, unsigned int* worst) {
+    float w = 0.f;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; 2 * i + 1 < n; i += gridDim.x * blockDim.x) {
+        const float x0 = lo + (hi - lo) * (float)(2 * i) / (float)(n - 1);
+        const float x1 = lo + (hi - lo) * (float)(2 * i + 1) / (float)(n - 1);
+        float e0, e1;
+        sm100::exp2_poly_pair(sm100::f2(x0, x1), e0, e1);
+        const float r0 = exp2f(x0), r1 = exp2f(x1);
+        w = fmaxf(w, fmaxf(fabsf(e0 - r0) / r0, fabsf(e1 - r1) / r1));
+    }
+    atomicMax(worst, __float_as_uint(w));   // non-negative floats order like their bits
+}
+}  // namespace nys
+
+int nys_attn_selftest_exp2(float* max_rel_err) {
+    if (!max_rel_err) return NYS_ERR_INVALID_ARG;
+    unsigned int* d = nullptr;
+    if (cudaMalloc(&d, sizeof(unsigned int)) != cudaSuccess) return NYS_ERR_CUDA;
+    unsigned int h = 0;
+    int rc = NYS_OK;
+    if (cudaMemset(d, 0, sizeof(unsigned int)) != cudaSuccess) rc = NYS_ERR_CUDA;
+    if (rc == NYS_OK) {
+        nys::exp2_selftest_kernel<<<256, 256>>>(1 << 20, -125.f, 8.f, d);
+        if (cudaGetLastError() != cudaSuccess || cudaMemcpy(&h, d, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+            rc = NYS_ERR_CUDA;
+    }
+    cudaFree(d);
+    std::memcpy(max_rel_err, &h, sizeof(float));
+    return rc;
+}
 
 int nys_attn_pinv_static(const float* q_l, const float* k_l, float* z, int BH, int m, int d,
                          int n_iter, void* stream) {

@@ -237,6 +237,63 @@ __device__ __forceinline__ float ex2(float x) {
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
+// ---------------------------------------------------------------- packed fp32 pairs (sm_100a)
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t p, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+// Two floats to bf16 (round to nearest even), `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16_rn(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// 2^x for a pair of floats on the FMA pipe, to offload the MUFU unit. x is
+// clamped to >= -125 (so the result stays a normal float: about 2^-125
+// instead of a smaller value or 0) and must be <= 127. Range reduction: adding 1.5 * 2^23 rounds x to the nearest integer
+// n (held in the low mantissa bits), f = x - n lies in [-1/2, 1/2]; 2^f comes
+// from a degree-3 polynomial fitted for this library (minimax relative error,
+// Lawson iterations on a dense grid; max relative error 7.5e-5 evaluated in
+// fp32 Horner form); n is then added to the exponent field.
+__device__ __forceinline__ void exp2_poly_pair(uint64_t x2, float& e0, float& e1) {
+    constexpr float kShift = 12582912.f;   // 1.5 * 2^23
+    float x0, x1;
+    f2_split(x2, x0, x1);
+    x2 = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = f2_add(x2, f2(kShift, kShift));
+    const uint64_t n = f2_add(t, f2(-kShift, -kShift));
+    const uint64_t f = f2_fma(n, f2(-1.f, -1.f), x2);
+    uint64_t p = f2_fma(f2(0.05517132207751274f, 0.05517132207751274f), f,
+                        f2(0.24261054396629333f, 0.24261054396629333f));
+    p = f2_fma(p, f, f2(0.6932609677314758f, 0.6932609677314758f));
+    p = f2_fma(p, f, f2(0.9999281167984009f, 0.9999281167984009f));
+    float p0, p1, t0, t1;
+    f2_split(p, p0, p1);
+    f2_split(t, t0, t1);
+    // the low bits of t hold n; n << 23 lands in the exponent field (the high bits of t drop out)
+    e0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    e1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

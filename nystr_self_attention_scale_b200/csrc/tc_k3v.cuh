@@ -7,6 +7,8 @@
 //                                      the d^-1/4 of K is applied in the exponent)
 //   online softmax per landmark row    one thread per row reads S from TMEM,
 //                                      masks padded keys, writes bf16 P back
+//                                      (exponentials split between the MUFU unit
+//                                      and a polynomial on the FMA pipe)
 //   O += P . V_chunk                   MMA with A = P from TMEM, V as an MN-major
 //                                      operand (keys x d straight from the TMA tile),
 //                                      accumulating in TMEM across the chunks
@@ -17,11 +19,12 @@
 // Each item writes the unnormalised partial (O, reference max, running sum) of
 // its split; a deterministic combine over splits follows.
 //
-// Warp roles (384 threads): warp 0 TMA producer and TMEM allocator, warp 1 MMA
-// issuer, warps 4-7 and 8-11 two softmax warpgroups that split every chunk's
-// 128 keys (64 each), exchanging the chunk max through shared memory. Each
-// group writes its P into its own half of the S columns (the P.V MMA takes its
-// A operand from the two ranges). S is double buffered in TMEM; K/V chunks use
+// Warp roles (640 threads): warp 0 TMA producer and TMEM allocator, warp 1 MMA
+// issuer, warps 4-19 four softmax warpgroups that split every chunk's 128 keys
+// (32 each), exchanging the chunk max through shared memory; four warps per
+// SM sub-partition hide the TMEM and MUFU latencies. Each group writes its P
+// into the first half of its own 32 S columns (the P.V MMA takes its A
+// operand from the four ranges). S is double buffered in TMEM; K/V chunks use
 // a 3-stage shared-memory ring.
 #pragma once
 
@@ -42,9 +45,12 @@ struct K3vTc {
     static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
     static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
     static constexpr int kNumBars = 2 + 2 * kStages + 7 + 1;
-    static constexpr uint32_t kOffXch = kOffBar + kNumBars * 8;          // [2][2][128] chunk maxima
-    static constexpr uint32_t kOffLx = kOffXch + 2 * 2 * 128 * 4;        // [128] partial sums
-    static constexpr uint32_t kOffMisc = kOffLx + 128 * 4;
+    static constexpr int kGroups = 4;                                     // softmax warpgroups
+    static constexpr int kSoftmaxThreads = kGroups * 128;
+    static constexpr int kThreads = 128 + kSoftmaxThreads;               // warps 0-3 + the groups
+    static constexpr uint32_t kOffXch = kOffBar + kNumBars * 8;          // [2][4][128] chunk maxima
+    static constexpr uint32_t kOffLx = kOffXch + 2 * kGroups * 128 * 4;  // [4][128] partial sums
+    static constexpr uint32_t kOffMisc = kOffLx + kGroups * 128 * 4;
     // at least 116 KB so that only one CTA (and one 512-column TMEM allocation) fits per SM
     static constexpr uint32_t kSmemNeed = kOffMisc + 16 + 1024;
     static constexpr uint32_t kSmemBytes = kSmemNeed > 118784 ? kSmemNeed : 118784;
@@ -63,7 +69,7 @@ struct K3vTcParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(640, 1)
 k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const K3vTcParams prm) {
     using C = K3vTc<D>;
@@ -103,10 +109,10 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 256);
+            mbar_init(&p_full[b], C::kSoftmaxThreads);
             mbar_init(&pv_done[b], 1);
         }
-        mbar_init(o_free, 256);
+        mbar_init(o_free, C::kSoftmaxThreads);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -187,8 +193,8 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < C::kChunk / 16; ++k) {
-                    // keys 16k .. 16k+15: the first 64 from group 0's P, the rest from group 1's
-                    const uint32_t pa = tmem + C::kColS + b * 128 + (k < 4 ? k * 8 : 64 + (k - 4) * 8);
+                    // keys 16k .. 16k+15: P of group k / 2, at the start of its 32 S columns
+                    const uint32_t pa = tmem + C::kColS + b * 128 + 32 * (k >> 1) + 8 * (k & 1);
                     mma_bf16_ts(tmem + C::kColO, pa, descV(st, k), C::kIdPV, (first && k == 0) ? 0u : 1u);
                 }
                 mma_commit(&pv_done[b]);
@@ -215,17 +221,18 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             mbar_wait(mma_done, 0);
         }
     } else if (warp >= 4) {
-        const int grp = (warp - 4) >> 2;          // softmax group: keys [64 grp, 64 grp + 64) of a chunk
+        const int grp = (warp - 4) >> 2;          // softmax group: keys [32 grp, 32 grp + 32) of a chunk
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const float sc = split_scale(D) * kLog2e;   // exponent scale of the raw S = Q_l . K^T
         constexpr float kSlack = 8.f;               // log2 units: P stays below 2^8
-        float* xch = reinterpret_cast<float*>(sm + C::kOffXch);
-        float* lx = reinterpret_cast<float*>(sm + C::kOffLx);
+        constexpr int kT = C::kSoftmaxThreads;
+        float* xch = reinterpret_cast<float*>(sm + C::kOffXch);   // [2 buffers][4 groups][128]
+        float* lx = reinterpret_cast<float*>(sm + C::kOffLx);     // [4 groups][128]
         int g = 0, it = 0;
         for (int item = blockIdx.x; item < prm.total_items; item += gridDim.x, ++it) {
-            if (group_any(*abort_flag != 0, 1, 256)) break;
+            if (group_any(*abort_flag != 0, 1, kT)) break;
             const int bh = item / per_bh, half = (item / prm.splits) % prm.halves;
             const int split = item % prm.splits;
             const int b_idx = bh / prm.H;
@@ -236,116 +243,140 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             for (int c = 0; c < nch; ++c) {
                 const int j = g + c, b = j & 1;
                 const int key0 = (c0 + c) * C::kChunk;
-                // key-validity bits of this group's 64 keys (bit k = key key0 + 64 grp + k)
-                uint32_t mb0 = ~0u, mb1 = ~0u;
-                if (prm.mask_bits != nullptr) {
-                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(prm.mask_bits + (size_t)b_idx * (prm.n / 32) +
-                                                                          key0 / 32 + 2 * grp));
-                    mb0 = u.x; mb1 = u.y;
-                }
-                const bool full = (mb0 & mb1) == ~0u;
+                // key-validity bits of this group's 32 keys (bit k = key key0 + 32 grp + k)
+                const uint32_t mb = prm.mask_bits != nullptr
+                                        ? __ldg(prm.mask_bits + (size_t)b_idx * (prm.n / 32) + key0 / 32 + grp)
+                                        : ~0u;
+                const bool full = mb == ~0u;
+                // a wait that runs out leaves S unread: the group still passes the chunk's one
+                // barrier below (which also ORs the failure across the groups) and then stops
                 ok = warp_all(mbar_wait(&s_full[b], (j >> 1) & 1));
-                if (group_any(!ok, 1, 256)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t sbuf = tmem + lane_base + C::kColS + b * 128;
-                uint32_t v[2][32];
-                tmem_ld32(sbuf + 64 * grp, v[0]);
-                tmem_ld32(sbuf + 64 * grp + 32, v[1]);
-                tmem_ld_wait();
+                uint32_t v[32];
+                if (ok) {
+                    tmem_ld32(sbuf + 32 * grp, v);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = 0u;
+                }
                 if (!full) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        if (!((mb0 >> e) & 1u)) v[0][e] = __float_as_uint(-INFINITY);
-                        if (!((mb1 >> e) & 1u)) v[1][e] = __float_as_uint(-INFINITY);
-                    }
+                    for (int e = 0; e < 32; ++e)
+                        if (!((mb >> e) & 1u)) v[e] = __float_as_uint(-INFINITY);
                 }
-                float cmax = -INFINITY;
+                float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four short max chains
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) cmax = fmaxf(cmax, __uint_as_float(v[h][e]));
-                xch[(b * 2 + grp) * 128 + r] = cmax;
-                named_barrier(1, 256);
-                cmax = fmaxf(cmax, xch[(b * 2 + (grp ^ 1)) * 128 + r]);
+                for (int e = 0; e < 16; ++e)
+                    mq[e & 3] = max3(mq[e & 3], __uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+                xch[(b * 4 + grp) * 128 + r] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+                if (group_any(!ok, 1, kT)) { ok = false; break; }   // also publishes xch
+                const float* xr = xch + b * 4 * 128 + r;
+                const float cmax = fmaxf(fmaxf(xr[0], xr[128]), fmaxf(xr[256], xr[384]));
                 const float cm = cmax * sc;
                 // move the reference only when this chunk's max exceeds it by more than the slack
-                // (both groups take the same decision: same maxima, same history)
+                // (every group takes the same decision: same maxima, same history)
                 const bool move = cm > m_ref + kSlack;
                 const float m_new = move ? cm : m_ref;
                 const float alpha = move ? ex2(m_ref - m_new) : 1.f;   // m_ref = -inf gives 0
-                if (grp == 0 && c > 0 && warp_any(move && m_ref != -INFINITY)) {
-                    // rescale this warp's rows of O once P(j - 1) V has been accumulated
+                if (grp < D / 32 && c > 0 && warp_any(move && m_ref != -INFINITY)) {
+                    // rescale this warp's rows of O (group g: columns 32 g .. 32 g + 31) once
+                    // P(j - 1) V has been accumulated
                     ok = warp_all(mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
                     if (ok) {
                         tc_fence_after();
                         uint32_t o[32];
+                        tmem_ld32(tmem + lane_base + C::kColO + grp * 32, o);
+                        tmem_ld_wait();
 #pragma unroll
-                        for (int h = 0; h < D / 32; ++h) {
-                            tmem_ld32(tmem + lane_base + C::kColO + h * 32, o);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                            tmem_st32(tmem + lane_base + C::kColO + h * 32, o);
-                        }
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tmem + lane_base + C::kColO + grp * 32, o);
                     }
                 }
                 const float mo = m_new == -INFINITY ? 0.f : m_new;   // rows with every key padded so far: P = 0
-                float sum = 0.f;
-                const uint32_t pcol = sbuf + 64 * grp;   // this group's P: 32 columns at the start of its half
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    uint32_t pk[16];
+                // exponentials on packed fp32 pairs: in chunks without padded keys the FMA pipe takes
+                // 6 of every 16 pairs (polynomial 2^x) and the MUFU unit the rest; chunks with padded
+                // keys use the MUFU unit only, so that padded keys get exactly 0. P is rounded to
+                // bf16 (nearest even); the running sum adds the fp32 values.
+                const uint64_t sc2 = f2(sc, sc), nmo2 = f2(-mo, -mo);
+                uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
+                uint32_t pk[16];
+                if (full) {
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
-                        // bf16 P by truncation; the running sum adds the same truncated values
-                        const uint32_t u0 = __float_as_uint(ex2(fmaf(__uint_as_float(v[h][2 * e]), sc, -mo))) & 0xFFFF0000u;
-                        const uint32_t u1 = __float_as_uint(ex2(fmaf(__uint_as_float(v[h][2 * e + 1]), sc, -mo))) & 0xFFFF0000u;
-                        sum += __uint_as_float(u0) + __uint_as_float(u1);
-                        pk[e] = __byte_perm(u0, u1, 0x7632);
+                        const uint64_t x2 =
+                            f2_fma(f2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, nmo2);
+                        float e0, e1;
+                        if ((e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7) {
+                            exp2_poly_pair(x2, e0, e1);
+                        } else {
+                            float x0, x1;
+                            f2_split(x2, x0, x1);
+                            e0 = ex2(x0);
+                            e1 = ex2(x1);
+                        }
+                        pk[e] = pack_bf16_rn(e0, e1);
+                        acc[e & 1] = f2_add(acc[e & 1], f2(e0, e1));
                     }
-                    tmem_st16(pcol + h * 16, pk);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const uint64_t x2 =
+                            f2_fma(f2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, nmo2);
+                        float x0, x1;
+                        f2_split(x2, x0, x1);
+                        const float e0 = ex2(x0), e1 = ex2(x1);
+                        pk[e] = pack_bf16_rn(e0, e1);
+                        acc[e & 1] = f2_add(acc[e & 1], f2(e0, e1));
+                    }
+                }
+                // this group's P: 16 columns at the start of its own (already read) 32 S columns
+                tmem_st16(sbuf + 32 * grp, pk);
+                float sum;
+                {
+                    float a0, a1, b0, b1;
+                    f2_split(acc[0], a0, a1);
+                    f2_split(acc[1], b0, b1);
+                    sum = (a0 + a1) + (b0 + b1);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(&p_full[b]);
                 l_run = fmaf(l_run, alpha, sum);
                 m_ref = m_new;
-                if (group_any(!ok, 1, 256)) { ok = false; break; }
             }
-            // the item's O is complete once its last P V has been accumulated; each group streams
-            // out half of the columns, group 0 adds the two partial sums
+            // the item's O is complete once its last P V has been accumulated; groups 0 .. D/32 - 1
+            // each stream out 32 columns, group 0 adds the four partial sums
             const int row = half * C::kRows + r;
             const size_t prow = ((size_t)bh * prm.splits + split) * prm.m + row;
-            if (ok && nch > 0) {
+            if (ok && nch > 0 && grp < D / 32) {
                 const int jl = g + nch - 1;
                 ok = warp_all(mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1));
                 if (ok) {
                     tc_fence_after();
+                    uint32_t t[32];
+                    tmem_ld32(tmem + lane_base + C::kColO + grp * 32, t);
+                    tmem_ld_wait();
+                    if (row < prm.m) {
+                        float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D + grp * 32);
 #pragma unroll
-                    for (int h = grp; h < D / 32; h += 2) {
-                        uint32_t t[32];
-                        tmem_ld32(tmem + lane_base + C::kColO + h * 32, t);
-                        tmem_ld_wait();
-                        if (row < prm.m) {
-                            float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D + h * 32);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                dst[e] = make_float4(__uint_as_float(t[4 * e]), __uint_as_float(t[4 * e + 1]),
-                                                     __uint_as_float(t[4 * e + 2]), __uint_as_float(t[4 * e + 3]));
-                        }
+                        for (int e = 0; e < 8; ++e)
+                            dst[e] = make_float4(__uint_as_float(t[4 * e]), __uint_as_float(t[4 * e + 1]),
+                                                 __uint_as_float(t[4 * e + 2]), __uint_as_float(t[4 * e + 3]));
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(o_free);
-            if (grp == 1) lx[r] = l_run;
-            if (group_any(!ok, 1, 256)) { *abort_flag = 1; break; }
+            lx[grp * 128 + r] = l_run;
+            if (group_any(!ok, 1, kT)) { *abort_flag = 1; break; }   // also publishes lx
             g += nch;
             if (grp == 0 && row < prm.m) {
                 prm.part_m[prow] = m_ref == -INFINITY ? -INFINITY : m_ref * kLn2;
-                prm.part_l[prow] = l_run + lx[r];
+                prm.part_l[prow] = (lx[r] + lx[128 + r]) + (lx[256 + r] + lx[384 + r]);
             }
-            named_barrier(1, 256);   // lx is read before the next item overwrites it
+            named_barrier(1, kT);   // lx is read before the next item overwrites it
         }
     }
 

@@ -13,10 +13,11 @@
 //                                    supplied by the TMA out-of-bounds fill)
 //   out    = O_att / rowsum(P) + O_conv, bf16, TMA store
 //
-// Warp roles (448 threads, one persistent CTA per SM over a contiguous range of
-// tiles): warp 0 TMA producers and TMEM allocator, warp 1 MMA issuer, warps
-// 2-5 and 6-9 two softmax warpgroups, warps 10-13 epilogue (and the Toeplitz
-// build). A warp w reaches TMEM lanes 32 (w % 4) .. +31, so each group of four
+// Warp roles (480 threads, one persistent CTA per SM over a contiguous range of
+// tiles): warp 0 TMA producer of Q and the per-head constants, and TMEM
+// allocator, warp 1 MMA issuer, warps 2-5 and 6-9 two softmax warpgroups,
+// warps 10-13 epilogue (and the Toeplitz build), warp 14 TMA producer of the
+// V halos. A warp w reaches TMEM lanes 32 (w % 4) .. +31, so each group of four
 // warps covers all 128 rows. Two TMEM slots alternate between consecutive
 // tiles. Both softmax warpgroups work on the same tile, each on half of the
 // landmark columns (row maxima are exchanged through shared memory), which
@@ -79,7 +80,7 @@ struct OutTcParams {
 };
 
 template <int D, int M>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(480, 1)
 output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_v,
                  const __grid_constant__ CUtensorMap map_out, const __grid_constant__ CUtensorMap map_kl,
                  const __grid_constant__ CUtensorMap map_wt, const OutTcParams prm) {
@@ -149,9 +150,8 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------ TMA producers: lane 0 streams Q tiles
-        // and the per-head constants, lane 1 streams the V halos (needed only by the conv MMA,
-        // late in a tile), so each Q tile is requested as soon as its stage's S MMA is done.
+        // ------------------------------------------------ TMA producer: Q tiles and the per-head
+        // constants; each Q tile is requested as soon as its stage's S MMA is done.
         if (lane == 0) {
             uint32_t ce_phase = 0;
             int last_use[2] = {-1, -1};
@@ -181,7 +181,11 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (last_use[st] >= 0) mbar_wait(&q_full[st], last_use[st] & 1);
                 if (const_loads > 0) mbar_wait(const_full, (const_loads - 1) & 1);
             }
-        } else if (lane == 1 && prm.conv_w != nullptr) {
+        }
+    } else if (warp == 14) {
+        // ------------------------------------------------ TMA producer of the V halos (its own warp,
+        // so that its loads are never held back behind the Q producer's waits)
+        if (lane == 0 && prm.conv_w != nullptr) {
             int last_use[2] = {-1, -1};
             for (int i = 0; i < count && !*abort_flag; ++i) {
                 const int t = t0 + i, bh = t / tph, row0 = (t % tph) * C::kRows;
@@ -284,16 +288,15 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         for (int i = 0; i < count && !warp_any(*abort_flag != 0); ++i) {
             const int s = i & 1;
             const bool ok = warp_all(mbar_wait(&s_full[s], (i >> 1) & 1));
-            // the whole group pair agrees before the exchange barrier below
-            if (group_any(!ok, 3, 256)) { *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
             const uint32_t scol = slot + g * kHalf;
-            // pass 1: the max of this half-row, 64 columns per wait
+            // pass 1: the max of this half-row, 64 columns per wait (skipped after a failed wait;
+            // the exchange barrier below ORs the failure over both groups)
             constexpr int kB = kHalf < 64 ? kHalf : 64;
-            float mx = -INFINITY;
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four short max chains
 #pragma unroll 1
-            for (int c0 = 0; c0 < kHalf; c0 += kB) {
+            for (int c0 = 0; c0 < (ok ? kHalf : 0); c0 += kB) {
                 uint32_t v[kB / 32][32];
 #pragma unroll
                 for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(scol + c0 + bq * 32, v[bq]);
@@ -301,16 +304,22 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 #pragma unroll
                 for (int bq = 0; bq < kB / 32; ++bq)
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) mx = fmaxf(mx, __uint_as_float(v[bq][j]));
+                    for (int j = 0; j < 16; ++j)
+                        mq[j & 3] = max3(mq[j & 3], __uint_as_float(v[bq][2 * j]), __uint_as_float(v[bq][2 * j + 1]));
             }
+            float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             pmax[(s * 2 + g) * 128 + r] = mx;
-            named_barrier(3, 256);
+            if (group_any(!ok, 3, 256)) { *abort_flag = 1; break; }   // also publishes pmax
             mx = fmaxf(mx, pmax[(s * 2 + (g ^ 1)) * 128 + r]);
             const float mo = mx * sc;
             // pass 2: P into this group's own half of the S columns, in increasing column order,
             // so it only overwrites scores this thread has already read
             const uint32_t pcol = slot + (g == 0 ? C::kColPA : C::kColPB);
-            float sum = 0.f;
+            // exponentials on packed fp32 pairs: the MUFU unit takes 10 of every 16 pairs, the FMA
+            // pipe the other 6 (polynomial 2^x), so neither pipe alone bounds the loop. P is rounded
+            // to bf16 (nearest even); the row sum adds the fp32 values.
+            const uint64_t sc2 = f2(sc, sc), nmo2 = f2(-mo, -mo);
+            uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll 1
             for (int c0 = 0; c0 < kHalf; c0 += kB) {
                 uint32_t v[kB / 32][32];
@@ -322,18 +331,30 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     uint32_t pk[16];
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        // bf16 P by truncation; the row sum adds the same truncated values, so
-                        // the weights P / sum(P) the MMA applies are normalised exactly
-                        const uint32_t u0 = __float_as_uint(ex2(fmaf(__uint_as_float(v[bq][2 * j]), sc, -mo))) & 0xFFFF0000u;
-                        const uint32_t u1 = __float_as_uint(ex2(fmaf(__uint_as_float(v[bq][2 * j + 1]), sc, -mo))) & 0xFFFF0000u;
-                        sum += __uint_as_float(u0) + __uint_as_float(u1);
-                        pk[j] = __byte_perm(u0, u1, 0x7632);
+                        const uint64_t x2 = f2_fma(f2(__uint_as_float(v[bq][2 * j]), __uint_as_float(v[bq][2 * j + 1])),
+                                                   sc2, nmo2);
+                        float e0, e1;
+                        if ((j & 7) == 2 || (j & 7) == 5 || (j & 7) == 7) {
+                            exp2_poly_pair(x2, e0, e1);
+                        } else {
+                            float x0, x1;
+                            f2_split(x2, x0, x1);
+                            e0 = ex2(x0);
+                            e1 = ex2(x1);
+                        }
+                        pk[j] = pack_bf16_rn(e0, e1);
+                        acc[j & 1] = f2_add(acc[j & 1], f2(e0, e1));
                     }
                     tmem_st16(pcol + (c0 + bq * 32) / 2, pk);
                 }
             }
             tmem_st_wait();
-            psum[(s * 2 + g) * 128 + r] = sum;
+            {
+                float a0, a1, b0, b1;
+                f2_split(acc[0], a0, a1);
+                f2_split(acc[1], b0, b1);
+                psum[(s * 2 + g) * 128 + r] = (a0 + a1) + (b0 + b1);
+            }
             tc_fence_before();
             mbar_arrive(&p_full[s]);
         }

@@ -131,27 +131,33 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
 }  // namespace pair2
 
 struct PinvPairMaps {
-    CUtensorMap k2;    // k2   [BH][256][256] fp32, box 32 x 128, 128-byte swizzle: B atoms of P1
+    CUtensorMap ql;    // Q_l  [BH][256][d] fp32, box 32 x 128, 128-byte swizzle: A of the kernel_2 product
+    CUtensorMap kl;    // K_l, same box: B lines of the kernel_2 product
+    CUtensorMap k2;    // k2   [BH][256][256] fp32, box 32 x 128: B atoms of the later P1s (and its TMA store)
     CUtensorMap k2t;   // k2^T, same box: B atoms of the first P4 (columns of W_0 = c k2)
     CUtensorMap wt;    // W^T scratch, same box: B atoms of the later P4s
 };
 
 struct PinvPairParams {
-    const float* colsum_part;  // [BH][8][256] column sums of k2 per 32-row block
-    const float* rowsum;       // [BH][256]
-    const float* k2;           // [BH][256][256] (rows of W_0, loaded into TMEM)
-    const float* k2t;          // [BH][256][256] (n_iter = 0 only)
-    float* wt;                 // [BH][256][256] W^T scratch (row g = column g of W)
-    float* z_out;              // [BH][256][256]
-    int n_iter;
+    float* k2;         // [BH][256][256] k2 (tf32), written here, read back by TMA
+    float* k2t;        // [BH][256][256] k2^T (tf32), written here, read back by TMA
+    float* wt;         // [BH][256][256] W^T scratch (row g = column g of W)
+    float* z_out;      // [BH][256][256]
+    int d, n_iter;
 };
 
 struct PinvPair {
     static constexpr int M = 256;
     static constexpr uint32_t kAtomBytes = 128 * 128;          // 128 lines x 32 tf32
     static constexpr uint32_t kBBytes = 8 * kAtomBytes;        // 8 K atoms = 128 KB
-    static constexpr uint32_t kOffBar = kBBytes;
-    // barriers: bfull[8], bfree[8], mma_done, mma4_done, e_ready, wl_ready, drain
+    // kernel_2 operands in the B buffer: Q_l hi / lo, K_l hi / lo (d / 32 atoms each)
+    static constexpr uint32_t kOffAhi = 0, kOffAlo = 2 * kAtomBytes, kOffBhi = 4 * kAtomBytes,
+                              kOffBlo = 6 * kAtomBytes;
+    static constexpr uint32_t kOffRed = kBBytes;                // row / column reductions
+    // [2][128] row max / sum halves, [256] own column sums, [256] the peer's, [8] warp maxima,
+    // [2] own and peer max row sum
+    static constexpr uint32_t kOffBar = kOffRed + (2 * 128 + 2 * 128 + 256 + 256 + 8 + 8) * 4;
+    // barriers: bfull[8], bfree[8], mma_done, mma4_done, e_ready, wl_ready, drain, pro_full, cs_ready
     static constexpr uint32_t kOffMisc = kOffBar + 24 * 8;
     static constexpr uint32_t kSmemNeed = kOffMisc + 64 + 1024;
     // more than half of the SM's shared memory: no other CTA (and no other TMEM user) shares the SM
@@ -170,21 +176,30 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* bbuf = sm;
+    float* rx = reinterpret_cast<float*>(sm + C::kOffRed);   // [2][128] row max, later row sum of k2, per half
+    float* sx = rx + 256;                                     // [2][128] row sums of each half
+    float* cs_own = sx + 256;                                 // [256] column sums over this CTA's rows
+    float* cs_peer = cs_own + 256;                            // [256] the same from the peer CTA
+    float* wmax = cs_peer + 256;                              // [8]
+    float* rmax = wmax + 8;                                   // [0] own, [1] peer max row sum
     uint64_t* bfull = reinterpret_cast<uint64_t*>(sm + C::kOffBar);   // [8], used in CTA 0
     uint64_t* bfree = bfull + 8;                                       // [8], both CTAs (after P3, P4)
-    uint64_t* mma_done = bfree + 8;      // P1..P3 accumulators complete (both CTAs)
+    uint64_t* mma_done = bfree + 8;      // kernel_2 and P1..P3 accumulators complete (both CTAs)
     uint64_t* mma4_done = mma_done + 1;  // P4 accumulator complete (both CTAs)
     uint64_t* e_ready = mma4_done + 1;   // epilogue output in place for the next product (CTA 0)
-    uint64_t* wl_ready = e_ready + 1;    // W^T scratch written by both CTAs (each CTA)
+    uint64_t* wl_ready = e_ready + 1;    // k2 / k2^T / W^T scratch written by both CTAs (each CTA)
     uint64_t* drain = wl_ready + 1;
+    uint64_t* pro_full = drain + 1;      // Q_l / K_l tiles landed (each CTA)
+    uint64_t* cs_ready = pro_full + 1;   // the peer's column sums are in cs_peer (each CTA)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
-    float* red = reinterpret_cast<float*>(sm + C::kOffMisc + 16);   // [8]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_rank();
     const bool leader = rank == 0;
     const int bh = blockIdx.x >> 1;
     const int r0 = (int)rank * 128;
+    const int nka = prm.d / 32;          // K atoms of the kernel_2 product
+    const int n_iter = prm.n_iter;
 
     if (tid == 0) {
         for (int s = 0; s < 8; ++s) {
@@ -196,62 +211,45 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         mbar_init(e_ready, 16);    // one arrival per epilogue warp of either CTA
         mbar_init(wl_ready, 16);
         mbar_init(drain, 1);
+        mbar_init(pro_full, 1);
+        mbar_init(cs_ready, 8);    // one arrival per epilogue warp of the peer
         fence_mbar_init();
     }
     if (warp == 9) {
         tmem_alloc2(tmem_slot, 512);
         tmem_relinquish2();
     }
-    // c = 1 / (max column sum * max row sum) of this head's kernel_2
-    if (tid < 128) {
-        float mc = -INFINITY, mr = -INFINITY;
-        for (int c = tid; c < M; c += 128) {
-            float s = 0.f;
-#pragma unroll
-            for (int b = 0; b < M / 32; ++b) s += prm.colsum_part[((size_t)bh * (M / 32) + b) * M + c];
-            mc = fmaxf(mc, s);
-            mr = fmaxf(mr, prm.rowsum[(size_t)bh * M + c]);
-        }
-        mc = warp_max(mc);
-        mr = warp_max(mr);
-        if (lane == 0) {
-            red[warp] = mc;
-            red[4 + warp] = mr;
-        }
-    }
     tc_fence_before();
     __syncthreads();
     cluster_sync_all();   // both CTAs' barriers initialised before any remote arrive or multicast commit
     tc_fence_after();
-    const float coeff = 1.f / (fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) *
-                               fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
     const uint32_t tmem = *tmem_slot;
     const uint32_t R0 = tmem, R1 = tmem + 256;
-    const int n_iter = prm.n_iter;
 
-    if (n_iter == 0) {
-        // Z = c k2^T
-        for (int e = tid; e < 128 * (M / 4); e += C::kThreads) {
-            const int r = r0 + e / (M / 4), c = (e % (M / 4)) * 4;
-            const size_t o = ((size_t)bh * M + r) * M + c;
-            float4 v = *reinterpret_cast<const float4*>(prm.k2t + o);
-            v.x *= coeff; v.y *= coeff; v.z *= coeff; v.w *= coeff;
-            *reinterpret_cast<float4*>(prm.z_out + o) = v;
-        }
-    } else if (warp == 8) {
+    if (warp == 8) {
         // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
+            prefetch_tmap(&maps.ql);
+            prefetch_tmap(&maps.kl);
             prefetch_tmap(&maps.k2);
             prefetch_tmap(&maps.k2t);
             prefetch_tmap(&maps.wt);
+            // kernel_2 operands: this CTA's rows of Q_l (A) and of K_l (its B lines)
+            mbar_arrive_expect_tx(pro_full, 2u * nka * C::kAtomBytes);
+            for (int a = 0; a < nka; ++a) {
+                tma_load_3d(bbuf + C::kOffAhi + a * C::kAtomBytes, &maps.ql, pro_full, 32 * a, r0, bh);
+                tma_load_3d(bbuf + C::kOffBhi + a * C::kAtomBytes, &maps.kl, pro_full, 32 * a, r0, bh);
+            }
             const uint32_t bfull0 = mapa(smem_u32(bfull), 0);
             bool ok = true;
             for (int it = 0; it < n_iter && ok; ++it) {
                 for (int part = 0; part < 2 && ok; ++part) {
                     const int p = part == 0 ? 0 : 3;
+                    if (p == 0 && it == 0) continue;   // the first P1 reads k2 staged by the prologue
                     const CUtensorMap* mp = p == 0 ? &maps.k2 : (it == 0 ? &maps.k2t : &maps.wt);
-                    if (p == 3 && it > 0) {
-                        ok = wait_acq_cluster(wl_ready, (uint32_t)(it - 1) & 1u);   // W^T of both CTAs stored
+                    if (p == 3) {
+                        // k2 / k2^T (prologue) or W^T (previous P4) of both CTAs is in global memory
+                        ok = wait_acq_cluster(wl_ready, (uint32_t)it & 1u);
                         fence_proxy_async_global();
                     }
                     for (int kc = 0; kc < 8 && ok; ++kc) {
@@ -259,7 +257,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                         // next P1) has read it. bfree[kc] completes twice per iteration, after
                         // P3 and after P4, and never runs ahead of these loads by more than one
                         // phase, so its parity is exact.
-                        if (it > 0 || p == 3) ok = mbar_wait(&bfree[kc], p == 3 ? 0u : 1u);
+                        ok = mbar_wait(&bfree[kc], p == 3 ? 0u : 1u);
                         if (!ok) break;
                         if (leader) mbar_arrive_expect_tx(&bfull[kc], 2 * C::kAtomBytes);
                         tma_load_3d_pair(bbuf + kc * C::kAtomBytes, mp, bfull0 + 8 * kc, 32 * kc, r0, bh);
@@ -274,13 +272,32 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             const uint32_t bs = smem_u32(bbuf);
             bool ok = true;
             uint32_t ne = 0, nf = 0;   // e_ready phases waited, streamed products issued
+            // kernel_2: S2 = Q_l K_l^T from split tf32 operands, hi.hi + hi.lo + lo.hi
+            ok = wait_acq_cluster(e_ready, ne & 1u);
+            ++ne;
+            if (ok) {
+                tc_fence_after();
+                const uint32_t aoff[3] = {C::kOffAhi, C::kOffAhi, C::kOffAlo};
+                const uint32_t boff[3] = {C::kOffBhi, C::kOffBlo, C::kOffBhi};
+                uint32_t acc = 0;
+                for (int t = 0; t < 3; ++t)
+                    for (int a = 0; a < nka; ++a)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t ka = a * C::kAtomBytes + kk * 32;
+                            mma2_ss(R1, smem_desc(bs + aoff[t] + ka, 16, 1024, kLayoutSw128),
+                                    smem_desc(bs + boff[t] + ka, 16, 1024, kLayoutSw128), C::kIdesc, acc);
+                            acc = 1;
+                        }
+                commit2(mma_done, 3);
+            }
             for (int it = 0; it < n_iter && ok; ++it) {
                 for (int p = 0; p < 4 && ok; ++p) {
                     const uint32_t a_col = (p == 0 || p == 2) ? R0 : R1;
                     const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
-                    const bool streamed = p == 0 || p == 3;
+                    const bool streamed = p == 3 || (p == 0 && it > 0);
                     if (p != 0 || it == 0) {
-                        ok = wait_acq_cluster(e_ready, ne & 1u);   // left factor (and X) in place
+                        ok = wait_acq_cluster(e_ready, ne & 1u);   // left factor (and X, or k2) in place
                         ++ne;
                         if (!ok) break;
                     }
@@ -312,6 +329,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         const int q = warp & 3, h = warp >> 2;      // TMEM lane quadrant, column half
         const int lrow = 32 * q + lane;             // TMEM lane = this CTA's row = its B line
         const int row = r0 + lrow;                  // global row of every product
+        const int et = tid;                          // 0 .. 255
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         const uint32_t e_ready0 = mapa(smem_u32(e_ready), 0);
         const uint32_t wl_loc = mapa(smem_u32(wl_ready), rank), wl_rem = mapa(smem_u32(wl_ready), rank ^ 1u);
@@ -327,26 +345,167 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             __syncwarp();
             if (lane == 0) arrive_cluster(e_ready0);
         };
-
-        // W_0 = c k2: rows of k2 (unscaled) into R0
-#pragma unroll 1
-        for (int jj = 0; jj < 4; ++jj) {
-            const int a = 4 * h + jj;
-            const float4* src = reinterpret_cast<const float4*>(prm.k2 + ((size_t)bh * M + row) * M + 32 * a);
-            uint32_t v[32];
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                const float4 f = __ldg(src + c);
-                v[4 * c] = __float_as_uint(f.x); v[4 * c + 1] = __float_as_uint(f.y);
-                v[4 * c + 2] = __float_as_uint(f.z); v[4 * c + 3] = __float_as_uint(f.w);
+        auto arrive_wl = [&]() {
+            fence_proxy_async_global();   // read next by TMA
+            __syncwarp();
+            if (lane == 0) {
+                arrive_cluster(wl_rem);
+                arrive_cluster(wl_loc);
             }
-            tmem_st32(R0 + lane_base + 32 * a, v);
-        }
-        tmem_st_wait();
-        arrive_e();
+        };
+        // byte offset of (this row, column 32 a + 4 c) in a K-major B / staging atom
+        auto stage_off = [&](int a, int c) {
+            return (uint32_t)a * C::kAtomBytes + (uint32_t)lrow * 128u + (((uint32_t)c ^ (uint32_t)(lrow & 7)) << 4);
+        };
 
-        bool failed = false;
-        uint32_t nd = 0, n4 = 0;   // mma_done / mma4_done phases waited
+        // ---- kernel_2 prologue (walkthrough 2.4: k2 = softmax_row(Q_l K_l^T); 2.5: c)
+        bool failed = !mbar_wait(pro_full, 0);
+        failed = group_any(failed, 3, 256);
+        float coeff = 0.f;
+        if (!failed) {
+            // split Q_l and K_l into tf32 hi + lo in place (fp32 accuracy from three tf32 products)
+            const int chunks = nka * (int)(C::kAtomBytes / 16);   // 16-byte chunks per tile
+            for (int e = et; e < 2 * chunks; e += 256) {
+                const uint32_t base = e < chunks ? C::kOffAhi : C::kOffBhi;
+                const uint32_t off = base + (uint32_t)(e % chunks) * 16u;
+                float4* hi = reinterpret_cast<float4*>(bbuf + off);
+                float4* lo = reinterpret_cast<float4*>(bbuf + off + (C::kOffAlo - C::kOffAhi));
+                const float4 x = *hi;
+                const float4 xh = make_float4(tf32_rna(x.x), tf32_rna(x.y), tf32_rna(x.z), tf32_rna(x.w));
+                *hi = xh;
+                *lo = make_float4(x.x - xh.x, x.y - xh.y, x.z - xh.z, x.w - xh.w);
+            }
+            fence_proxy_async_shared();
+            arrive_e();
+            const bool ok = mbar_wait(mma_done, 0);
+            failed = group_any(!ok, 3, 256);
+        }
+        if (!failed) {
+            tc_fence_after();
+            // row max: this thread's 128 columns, then the other half's through shared memory
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+            for (int jj = 0; jj < 4; ++jj) {
+                uint32_t v[32];
+                tmem_ld32(R1 + lane_base + 32 * (4 * h + jj), v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    mq[i & 3] = max3(mq[i & 3], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            }
+            rx[h * 128 + lrow] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            named_barrier(3, 256);
+            const float mx = fmaxf(rx[lrow], rx[128 + lrow]);
+            // exponentials, kept in place in TMEM; their row sum
+            float ssum = 0.f;
+#pragma unroll 1
+            for (int jj = 0; jj < 4; ++jj) {
+                uint32_t v[32];
+                const uint32_t addr = R1 + lane_base + 32 * (4 * h + jj);
+                tmem_ld32(addr, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float e = __expf(__uint_as_float(v[i]) - mx);
+                    ssum += e;
+                    v[i] = __float_as_uint(e);
+                }
+                tmem_st32(addr, v);
+            }
+            tmem_st_wait();
+            sx[h * 128 + lrow] = ssum;
+            named_barrier(3, 256);
+            const float inv = 1.f / (sx[lrow] + sx[128 + lrow]);
+            // k2 = e / sum: into TMEM as W_0 (R0), into the B buffer as the first P1's right
+            // factor (this CTA's rows are its own B lines), and transposed into global k2^T
+            float rsum = 0.f;
+            float* k2t_col = prm.k2t + (size_t)bh * M * M + row;
+#pragma unroll 1
+            for (int jj = 0; jj < 4; ++jj) {
+                const int a = 4 * h + jj;
+                uint32_t v[32];
+                tmem_ld32(R1 + lane_base + 32 * a, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float pv = __uint_as_float(v[i]) * inv;
+                    rsum += pv;
+                    const float pr = tf32_rna(pv);
+                    v[i] = __float_as_uint(pr);
+                    k2t_col[(size_t)(32 * a + i) * M] = pr;
+                }
+                tmem_st32(R0 + lane_base + 32 * a, v);
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<uint4*>(bbuf + stage_off(a, c)) =
+                        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            }
+            rx[h * 128 + lrow] = rsum;   // rx is free: every thread read its row max before the last barrier
+            fence_proxy_async_shared();   // the staged k2 rows feed the MMA and a TMA store
+            named_barrier(3, 256);
+            // column sums over this CTA's rows (thread et: column et), max row sum of this CTA
+            {
+                const int a = et >> 5, j = et & 31;
+                float cs = 0.f;
+#pragma unroll 8
+                for (int l = 0; l < 128; ++l)
+                    cs += *reinterpret_cast<const float*>(
+                        bbuf + (uint32_t)a * C::kAtomBytes + (uint32_t)l * 128u +
+                        ((((uint32_t)j >> 2) ^ (uint32_t)(l & 7)) << 4) + (uint32_t)(j & 3) * 4u);
+                cs_own[et] = cs;
+                st_remote(mapa(smem_u32(cs_peer + et), rank ^ 1u), cs);
+                const float rs = warp_max(et < 128 ? rx[et] + rx[128 + et] : 0.f);
+                if (lane == 0) wmax[warp] = rs;
+            }
+            named_barrier(3, 256);
+            if (et == 0) {
+                const float rm = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+                rmax[0] = rm;
+                st_remote(mapa(smem_u32(rmax + 1), rank ^ 1u), rm);
+            }
+            __syncwarp();
+            if (lane == 0) arrive_cluster(mapa(smem_u32(cs_ready), rank ^ 1u));
+            // the rows of k2 go to global memory for the later P1s (TMA store of the staging)
+            if (et == 0) {
+                for (int a = 0; a < 8; ++a) tma_store_3d(&maps.k2, bbuf + a * C::kAtomBytes, 32 * a, r0, bh);
+                tma_store_commit();
+            }
+            const bool ok = wait_acq_cluster(cs_ready, 0);
+            failed = group_any(!ok, 3, 256);
+            if (!failed) {
+                const float tot = warp_max(cs_own[et] + cs_peer[et]);
+                if (lane == 0) wmax[warp] = tot;
+                named_barrier(3, 256);
+                float mc = wmax[0];
+#pragma unroll
+                for (int w = 1; w < 8; ++w) mc = fmaxf(mc, wmax[w]);
+                coeff = 1.f / (mc * fmaxf(rmax[0], rmax[1]));
+            }
+            if (et == 0) tma_store_wait_all<0>();
+            if (n_iter == 0 && !failed) {
+                // Z = c k2^T, from the staged rows
+                float* zc = prm.z_out + (size_t)bh * M * M + row;
+#pragma unroll 1
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int a = 4 * h + jj;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 f4 = *reinterpret_cast<const float4*>(bbuf + stage_off(a, c));
+                        zc[(size_t)(32 * a + 4 * c) * M] = coeff * f4.x;
+                        zc[(size_t)(32 * a + 4 * c + 1) * M] = coeff * f4.y;
+                        zc[(size_t)(32 * a + 4 * c + 2) * M] = coeff * f4.z;
+                        zc[(size_t)(32 * a + 4 * c + 3) * M] = coeff * f4.w;
+                    }
+                }
+            } else if (!failed) {
+                tmem_st_wait();
+                arrive_e();     // W_0 in TMEM, k2 lines in the B buffer
+                arrive_wl();    // k2 and k2^T in global memory
+            }
+        }
+
+        // ---- the iteration
+        uint32_t nd = 1, n4 = 0;   // mma_done / mma4_done phases waited
         for (int it = 0; it < n_iter && !failed; ++it) {
             const float sigma = it == 0 ? coeff : (it == 1 ? 0.25f * coeff : 0.25f);
             const float lambda = it == 0 ? 0.25f * coeff : 0.25f;
@@ -410,14 +569,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                     tmem_st32(d_col + lane_base + 32 * a, v);
                 }
                 if (p == 3) {
-                    if (!last_it) {
-                        fence_proxy_async_global();   // W^T is read next by TMA
-                        __syncwarp();
-                        if (lane == 0) {
-                            arrive_cluster(wl_rem);
-                            arrive_cluster(wl_loc);
-                        }
-                    }
+                    if (!last_it) arrive_wl();
                 } else {
                     tmem_st_wait();
                     if (p == 0) fence_proxy_async_cluster();   // X lines (here and in the peer) feed the MMA
@@ -429,7 +581,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
 
     tc_fence_before();
     __syncthreads();
-    cluster_sync_all();   // no arrive or MMA of either CTA is still pending
+    cluster_sync_all();   // no arrive, remote store or MMA of either CTA is still pending
     if (warp == 9) {
         tc_fence_after();
         tmem_dealloc2(tmem, 512);

@@ -260,3 +260,10 @@ def test_invalid_arguments_raise(nys):
     with pytest.raises(nys.NysError) as e:
         nys.forward(q, q, q, m=64)
     assert e.value.status == -2
+
+
+def test_exp2_polynomial_against_cuda_exp2f(nys):
+    """The FMA-pipe 2^x used for part of the softmax exponentials stays within its
+    fitted bound (7.5e-5 relative, degree-3 minimax) of CUDA's exp2f on [-125, 8]."""
+    err = nys.selftest_exp2()
+    assert 0.0 <= err <= 1.0e-4, err
