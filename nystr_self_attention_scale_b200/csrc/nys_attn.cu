@@ -216,7 +216,9 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
     int splits = (n + kps - 1) / kps;
     if (dtype == NYS_BF16) {
         const int chunks = n / 128;
-        p.tc_cps = std::min(chunks, n >= 16384 ? 16 : 8);
+        // 26 chunks (3328 keys) per split from n = 16384 on: fewer, larger items (5 splits at
+        // n = 16384) and fewer partials to merge
+        p.tc_cps = std::min(chunks, n >= 16384 ? 26 : 8);
         p.tc_splits = (chunks + p.tc_cps - 1) / p.tc_cps;
         splits = p.tc_splits;
         kps = p.tc_cps * 128;
