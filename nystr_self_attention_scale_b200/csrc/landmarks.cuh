@@ -36,6 +36,14 @@ landmarks_kernel(const T* __restrict__ q, const T* __restrict__ k, float* __rest
 #pragma unroll
     for (int e = 0; e < V; ++e) acc[e] = 0.f;
     int t = 0;
+    for (; t + 8 <= L; t += 8) {   // eight independent 16-byte loads in flight per thread
+        float x[8][V];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) Elt<T>::load16(src + (long long)(t + u) * d, x[u]);
+#pragma unroll
+        for (int e = 0; e < V; ++e)
+            acc[e] += ((x[0][e] + x[1][e]) + (x[2][e] + x[3][e])) + ((x[4][e] + x[5][e]) + (x[6][e] + x[7][e]));
+    }
     for (; t + 4 <= L; t += 4) {
         float x0[V], x1[V], x2[V], x3[V];
         Elt<T>::load16(src + (long long)(t + 0) * d, x0);

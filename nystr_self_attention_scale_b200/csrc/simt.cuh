@@ -297,11 +297,14 @@ k3v_partial_simt_kernel(const float* __restrict__ ql, const T* __restrict__ k, c
 }
 
 // Merge the key-split partials: k3v[j] = sum_s e^{M_s - M} O_s / sum_s e^{M_s - M} l_s.
-// One thread per (head, landmark row, 4 columns); the split order is fixed, so the
-// result is deterministic. All loads of a thread are independent of each other.
+// One thread per (head, landmark row, 4 columns), one pass: the splits are taken
+// eight at a time with all their loads in flight together, and the running sums
+// are rescaled when a later group raises the maximum. The split order is fixed,
+// so the result is deterministic.
 __global__ void __launch_bounds__(256)
 k3v_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_m,
                    const float* __restrict__ part_l, float* __restrict__ k3v, int BH, int m, int d, int splits) {
+    constexpr int G = 8;
     const int q = d / 4;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (long long)BH * m * q) return;
@@ -310,22 +313,37 @@ k3v_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ p
     const int j = (int)(bj % m);
     const long long bh = bj / m;
     const size_t row0 = (size_t)bh * splits * m + j;   // row of split 0; split s adds s * m
-    float M = -INFINITY;
-#pragma unroll 8
-    for (int s = 0; s < splits; ++s) M = fmaxf(M, __ldg(part_m + row0 + (size_t)s * m));
+    float M = -INFINITY, den = 0.f;
     float4 num = make_float4(0.f, 0.f, 0.f, 0.f);
-    float den = 0.f;
-#pragma unroll 8
-    for (int s = 0; s < splits; ++s) {
-        const size_t row = row0 + (size_t)s * m;
-        const float ms = __ldg(part_m + row);
-        const float f = (ms == -INFINITY) ? 0.f : __expf(ms - M);
-        const float4 o = __ldg(reinterpret_cast<const float4*>(part_o + row * d) + c4);
-        num.x = fmaf(f, o.x, num.x);
-        num.y = fmaf(f, o.y, num.y);
-        num.z = fmaf(f, o.z, num.z);
-        num.w = fmaf(f, o.w, num.w);
-        den = fmaf(f, __ldg(part_l + row), den);
+    for (int s0 = 0; s0 < splits; s0 += G) {
+        float ms[G], ls[G];
+        float4 os[G];
+#pragma unroll
+        for (int e = 0; e < G; ++e) {
+            const size_t row = row0 + (size_t)(s0 + e) * m;
+            const bool ok = s0 + e < splits;
+            ms[e] = ok ? __ldg(part_m + row) : -INFINITY;
+            ls[e] = ok ? __ldg(part_l + row) : 0.f;
+            os[e] = ok ? __ldg(reinterpret_cast<const float4*>(part_o + row * d) + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        float gm = M;
+#pragma unroll
+        for (int e = 0; e < G; ++e) gm = fmaxf(gm, ms[e]);
+        if (gm != -INFINITY && gm != M) {
+            const float sc = M == -INFINITY ? 0.f : __expf(M - gm);
+            num.x *= sc; num.y *= sc; num.z *= sc; num.w *= sc;
+            den *= sc;
+            M = gm;
+        }
+#pragma unroll
+        for (int e = 0; e < G; ++e) {
+            const float f = (ms[e] == -INFINITY) ? 0.f : __expf(ms[e] - M);
+            num.x = fmaf(f, os[e].x, num.x);
+            num.y = fmaf(f, os[e].y, num.y);
+            num.z = fmaf(f, os[e].z, num.z);
+            num.w = fmaf(f, os[e].w, num.w);
+            den = fmaf(f, ls[e], den);
+        }
     }
     const float inv = 1.f / den;
     reinterpret_cast<float4*>(k3v + (size_t)bj * d)[c4] =
