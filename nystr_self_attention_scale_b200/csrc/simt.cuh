@@ -370,9 +370,10 @@ w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __re
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < CW; ++j) acc[i][j] = 0.f;
-    for (int k0 = 0; k0 < m; k0 += 64) {
-        float za[16];   // scalar loads: m need not be a multiple of 4 on the float32 path
-        float4 ka[D / 16];
+    // the next 64-wide slice of Z and k3V is loaded into registers while the current one is used
+    float za[16];   // scalar loads: m need not be a multiple of 4 on the float32 path
+    float4 ka[D / 16];
+    auto load_slice = [&](int k0) {
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int idx = tid + e * 256, r = idx >> 6, c = idx & 63;
@@ -384,7 +385,10 @@ w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __re
             ka[e] = (k0 + r < m) ? __ldg(reinterpret_cast<const float4*>(kb + (size_t)(k0 + r) * D) + c4)
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        __syncthreads();
+    };
+    load_slice(0);
+    for (int k0 = 0; k0 < m; k0 += 64) {
+        __syncthreads();   // the previous slice has been read from shared memory
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int idx = tid + e * 256, r = idx >> 6, c = idx & 63;
@@ -396,17 +400,24 @@ w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __re
             *reinterpret_cast<float4*>(&sK[r][4 * c4]) = ka[e];
         }
         __syncthreads();
+        if (k0 + 64 < m) load_slice(k0 + 64);
 #pragma unroll 8
         for (int kk = 0; kk < 64; ++kk) {
             float a[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) a[i] = sZ[ty * 4 + i][kk];
+            float bv[CW];
+            if constexpr (CW == 4) {
+                const float4 b4 = *reinterpret_cast<const float4*>(&sK[kk][4 * tx]);
+                bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+            } else {
 #pragma unroll
-            for (int j = 0; j < CW; ++j) {
-                const float bv = sK[kk][tx * CW + j];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(a[i], bv, acc[i][j]);
+                for (int j = 0; j < CW; ++j) bv[j] = sK[kk][tx * CW + j];
             }
+#pragma unroll
+            for (int j = 0; j < CW; ++j)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(a[i], bv[j], acc[i][j]);
         }
     }
 #pragma unroll
