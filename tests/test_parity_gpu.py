@@ -217,6 +217,23 @@ def test_edge_shapes(nys, oracle_mod, dtype, B, H, n, d, m):
     _full_check(nys, oracle_mod, x, f"edge {dtype} B{B} H{H} n{n} d{d} m{m}")
 
 
+@pytest.mark.parametrize("d,n_iter,lengths,n", [
+    (32, 6, None, 1024),           # one K atom in the fused kernel_2 product
+    (64, 0, None, 1024),           # n_iter = 0: Z = c k2^T straight from the prologue
+    (64, 1, (700, 1024), 1024),    # one iteration (no W^T scratch round trip), masked keys
+    (32, 3, (300, 2048), 2048),    # d = 32, masked, ragged lengths
+    (64, 6, (1, 1024), 1024),      # masked, some sequences with a single valid key
+])
+def test_pair_inverse_variants(nys, oracle_mod, d, n_iter, lengths, n):
+    """m = 256 on the bf16 path: the CTA-pair inverse with kernel_2 in its prologue, over
+    head dimensions, iteration counts and masks the headline workload does not reach."""
+    import dataclasses
+    w = dataclasses.replace(WORKLOADS["n16384_bf16_corr"], d=d, n_iter=n_iter, lengths=lengths,
+                            zero_pad=lengths is not None)
+    x = make_inputs(w, seed=13, B=2, H=2, n=n)
+    _full_check(nys, oracle_mod, x, f"pair inverse d{d} n_iter{n_iter} lengths{lengths} n{n}")
+
+
 def test_single_valid_key(nys, oracle_mod):
     import dataclasses
     w = dataclasses.replace(WORKLOADS["default_f32_masked"], lengths=(1, 1))
