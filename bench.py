@@ -250,8 +250,33 @@ def cpu_baseline(w, x):
                       f"{sec:.1f} s wall on {min(cores, len(heads))} threads"}
 
 
+def rank_env():
+    """(world size, rank, local rank) from the launcher's environment; (1, 0, 0) when run alone."""
+    return (int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def max_over_ranks(value, world, device):
+    """The largest value of a float over all ranks (the slowest rank's time).
+
+    Identity at world size 1; otherwise one all-reduce(MAX) of a float64 on
+    ``device`` ("cuda" under NCCL, "cpu" under gloo)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, steps, total_ms):
+    """Whole-job tokens/s: the tokens every rank processed over the slowest rank's time."""
+    return tokens_per_rank * world * steps / (total_ms * 1e-3)
+
+
 def run_reference(args, w):
-    rank = int(os.environ.get("RANK", "0"))
+    _, rank, _ = rank_env()
     if rank != 0:
         return 0
     import oracle
@@ -320,9 +345,7 @@ def main():
 
     import torch
     import torch.distributed as dist
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = rank_env()
     torch.cuda.set_device(local)
     if world > 1:
         import datetime
@@ -386,13 +409,9 @@ def main():
     nys.profile_enable(False)
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     status = nys.device_status()
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, "cuda")
     ms_per_step = total_ms / args.steps
-    tokens_all = w.tokens * world * args.steps
-    value = tokens_all / (total_ms * 1e-3)
+    value = job_throughput(w.tokens, world, args.steps, total_ms)
 
     peaks, peak_src = load_peaks()
     launches = sum(n for n, _ in prof.values())
@@ -439,13 +458,10 @@ def main():
             b.record(stream)
             b.synchronize()
             e_ms += a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e_ms], device="cuda", dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e_ms, world, "cuda")
         elt = qh.element_size()
         h2d = 3 * qh.numel() * elt + (0 if mh is None else mh.numel()) + (0 if wh is None else wh.numel() * 4)
-        e2e = {"value": round(w.tokens * world * args.e2e_steps / (e_ms * 1e-3), 1), "unit": UNIT,
+        e2e = {"value": round(job_throughput(w.tokens, world, args.e2e_steps, e_ms), 1), "unit": UNIT,
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(oh.numel() * elt),
                "steps": args.e2e_steps, "ms_per_step": round(e_ms / args.e2e_steps, 3)}
 
