@@ -70,6 +70,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 // loads/stores and named barriers are always reached by every thread.
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 __device__ __forceinline__ bool warp_any(bool v) { return __any_sync(0xffffffffu, v); }
+// true in one lane of a fully converged warp (elect.sync; every lane must execute it).
+// MMA warps run their whole loop converged, waits included, and issue each MMA group and
+// each commit from the elected lane: issuing from a lone lane that also runs the waits
+// leaves the tensor pipe idle around every wait.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t p;
+    asm volatile("{\n\t.reg .pred P;\n\t.reg .b32 r;\n\telect.sync r|P, 0xffffffff;\n\tselp.b32 %0, 1, 0, P;\n\t}"
+                 : "=r"(p));
+    return p != 0;
+}
 // OR of `v` over the `nthreads` threads that use named barrier `bar_id` (a barrier itself).
 __device__ __forceinline__ bool group_any(bool v, int bar_id, int nthreads) {
     uint32_t r;

@@ -113,7 +113,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             mbar_init(&pv_done[b], 1);
         }
         mbar_init(o_free, C::kSoftmaxThreads);
-        mbar_init(mma_done, 1);
+        mbar_init(mma_done, 32);   // one commit per lane of the MMA warp
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -162,64 +162,73 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            bool ok = true;
-            int g = 0, it = 0;
-            auto descQl = [&](int k) { return smem_desc(sbase + C::kOffQl + k * 32, 16, C::kSbo, C::kLayout); };
-            auto descK = [&](int st, int k) {
-                return smem_desc(sbase + C::kOffK + st * C::kTileBytes + k * 32, 16, C::kSbo, C::kLayout);
-            };
-            auto descV = [&](int st, int k) {
-                return smem_desc(sbase + C::kOffV + st * C::kTileBytes + k * 16 * C::kSpan, C::kTileBytes, C::kSbo,
-                                 C::kLayout);
-            };
-            auto issue_S = [&](int j) -> bool {
-                const int b = j & 1, st = j % C::kStages;
-                // S buffer b last held S(j - 2); P(j - 2) V was accumulated once PV(j - 2) completed
-                if (j >= 2 && !mbar_wait(&pv_done[b], ((j - 2) >> 1) & 1)) return false;
-                if (!mbar_wait(&kv_full[st], (j / C::kStages) & 1)) return false;
-                tc_fence_after();
+        // MMA issuer: the whole warp runs the loop and the waits; one elected lane issues each
+        // MMA group and each commit
+        bool ok = true;
+        int g = 0, it = 0;
+        auto descQl = [&](int k) { return smem_desc(sbase + C::kOffQl + k * 32, 16, C::kSbo, C::kLayout); };
+        auto descK = [&](int st, int k) {
+            return smem_desc(sbase + C::kOffK + st * C::kTileBytes + k * 32, 16, C::kSbo, C::kLayout);
+        };
+        auto descV = [&](int st, int k) {
+            return smem_desc(sbase + C::kOffV + st * C::kTileBytes + k * 16 * C::kSpan, C::kTileBytes, C::kSbo,
+                             C::kLayout);
+        };
+        auto wait = [&](uint64_t* bar, uint32_t parity) { return warp_all(mbar_wait(bar, parity)); };
+        auto issue_S = [&](int j) -> bool {
+            const int b = j & 1, st = j % C::kStages;
+            // S buffer b last held S(j - 2); P(j - 2) V was accumulated once PV(j - 2) completed
+            if (j >= 2 && !wait(&pv_done[b], ((j - 2) >> 1) & 1)) return false;
+            if (!wait(&kv_full[st], (j / C::kStages) & 1)) return false;
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
                     mma_bf16_ss(tmem + C::kColS + b * 128, descQl(k), descK(st, k), C::kIdS, k > 0);
-                mma_commit(&s_full[b]);
-                return true;
-            };
-            auto issue_PV = [&](int j, bool first, int item_it) -> bool {
-                const int b = j & 1, st = j % C::kStages;
-                if (!mbar_wait(&p_full[b], (j >> 1) & 1)) return false;
-                // the previous item's O must have been read before it is overwritten
-                if (first && !mbar_wait(o_free, (item_it & 1) ^ 1)) return false;
-                tc_fence_after();
+            }
+            if (elect_one()) mma_commit(&s_full[b]);
+            return true;
+        };
+        auto issue_PV = [&](int j, bool first, int item_it) -> bool {
+            const int b = j & 1, st = j % C::kStages;
+            if (!wait(&p_full[b], (j >> 1) & 1)) return false;
+            // the previous item's O must have been read before it is overwritten
+            if (first && !wait(o_free, (item_it & 1) ^ 1)) return false;
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < C::kChunk / 16; ++k) {
                     // keys 16k .. 16k+15: P of group k / 2, at the start of its 32 S columns
                     const uint32_t pa = tmem + C::kColS + b * 128 + 32 * (k >> 1) + 8 * (k & 1);
                     mma_bf16_ts(tmem + C::kColO, pa, descV(st, k), C::kIdPV, (first && k == 0) ? 0u : 1u);
                 }
+            }
+            if (elect_one()) {
                 mma_commit(&pv_done[b]);
                 mma_commit(&kv_empty[st]);
-                return true;
-            };
-            for (int item = blockIdx.x; item < prm.total_items && ok && !*abort_flag; item += gridDim.x, ++it) {
-                int c0;
-                const int nch = item_chunks(item, &c0);
-                ok = mbar_wait(ql_full, it & 1);
-                if (!ok) break;
-                tc_fence_after();
-                ok = issue_S(g);
-                for (int c = 0; c < nch && ok; ++c) {
-                    const int j = g + c;
-                    if (c + 1 < nch) ok = issue_S(j + 1);
-                    else mma_commit(ql_empty);   // every S MMA of this item is issued
-                    if (ok) ok = issue_PV(j, c == 0, it);
-                }
-                g += nch;
             }
-            if (!ok) *abort_flag = 1;
-            mma_commit(mma_done);
-            mbar_wait(mma_done, 0);
+            return true;
+        };
+        for (int item = blockIdx.x; item < prm.total_items && ok && !warp_any(*abort_flag != 0);
+             item += gridDim.x, ++it) {
+            int c0;
+            const int nch = item_chunks(item, &c0);
+            ok = wait(ql_full, it & 1);
+            if (!ok) break;
+            tc_fence_after();
+            ok = issue_S(g);
+            for (int c = 0; c < nch && ok; ++c) {
+                const int j = g + c;
+                if (c + 1 < nch) ok = issue_S(j + 1);
+                else if (elect_one()) mma_commit(ql_empty);   // every S MMA of this item is issued
+                if (ok) ok = issue_PV(j, c == 0, it);
+            }
+            g += nch;
         }
+        if (!ok) *abort_flag = 1;
+        // one commit per lane (mma_done counts 32 arrivals): the drain covers whichever lane issued
+        mma_commit(mma_done);
+        mbar_wait(mma_done, 0);
     } else if (warp >= 4) {
         const int grp = (warp - 4) >> 2;          // softmax group: keys [32 grp, 32 grp + 32) of a chunk
         const int q4 = warp & 3;

@@ -129,7 +129,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         mbar_init(const_full, 1);
         mbar_init(t_full, 128);
         mbar_init(const_empty, 1);
-        mbar_init(mma_done, 1);
+        mbar_init(mma_done, 32);   // one commit per lane of the MMA warp
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -200,82 +200,92 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (last_use[st] >= 0) mbar_wait(&v_full[st], last_use[st] & 1);
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            uint32_t cf_phase = 0;
-            bool ok = true;
-            auto descQ = [&](int st, int k) {
-                return smem_desc(sbase + C::kOffQ + st * C::kQBytes + k * 32, 16, C::kSbo, C::kLayout);
-            };
-            auto descKl = [&](int k) { return smem_desc(sbase + C::kOffKl + k * 32, 16, C::kSbo, C::kLayout); };
-            auto descWt = [&](int k) {
-                return smem_desc(sbase + C::kOffWt + (k >> 2) * C::kWtBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
-            };
-            auto descT = [&](int k) {
-                return smem_desc(sbase + C::kOffT + (k >> 2) * C::kTBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
-            };
-            auto descV = [&](int st, int k) {
-                return smem_desc(sbase + C::kOffV + st * C::kVBytes + k * 16 * C::kSpan, C::kVBytes, C::kSbo,
-                                 C::kLayout);
-            };
-            auto issue_S = [&](int j) -> bool {
-                const int s = j & 1, st = j % C::kStages;
-                if (!mbar_wait(&slot_free[s], ((j >> 1) & 1) ^ 1)) return false;
-                if (!mbar_wait(&q_full[st], (j / C::kStages) & 1)) return false;
-                tc_fence_after();
-                const uint32_t slot = tmem + s * C::kSlot;
+        // ------------------------------------------------ MMA issuer: the whole warp runs the loop and
+        // the waits; one elected lane issues each MMA group and each commit
+        uint32_t cf_phase = 0;
+        bool ok = true;
+        auto descQ = [&](int st, int k) {
+            return smem_desc(sbase + C::kOffQ + st * C::kQBytes + k * 32, 16, C::kSbo, C::kLayout);
+        };
+        auto descKl = [&](int k) { return smem_desc(sbase + C::kOffKl + k * 32, 16, C::kSbo, C::kLayout); };
+        auto descWt = [&](int k) {
+            return smem_desc(sbase + C::kOffWt + (k >> 2) * C::kWtBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
+        };
+        auto descT = [&](int k) {
+            return smem_desc(sbase + C::kOffT + (k >> 2) * C::kTBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
+        };
+        auto descV = [&](int st, int k) {
+            return smem_desc(sbase + C::kOffV + st * C::kVBytes + k * 16 * C::kSpan, C::kVBytes, C::kSbo,
+                             C::kLayout);
+        };
+        auto wait = [&](uint64_t* bar, uint32_t parity) { return warp_all(mbar_wait(bar, parity)); };
+        auto issue_S = [&](int j) -> bool {
+            const int s = j & 1, st = j % C::kStages;
+            if (!wait(&slot_free[s], ((j >> 1) & 1) ^ 1)) return false;
+            if (!wait(&q_full[st], (j / C::kStages) & 1)) return false;
+            tc_fence_after();
+            const uint32_t slot = tmem + s * C::kSlot;
+            if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) mma_bf16_ss(slot, descQ(st, k), descKl(k), C::kIdS, k > 0);
+            }
+            if (elect_one()) {
                 mma_commit(&s_full[s]);
                 mma_commit(&q_empty[st]);
-                return true;
-            };
-            auto issue_O = [&](int j) -> bool {
-                const int s = j & 1, st = j % C::kStages;
-                if (!mbar_wait(&p_full[s], (j >> 1) & 1)) return false;
-                tc_fence_after();
-                const uint32_t slot = tmem + s * C::kSlot;
+            }
+            return true;
+        };
+        auto issue_O = [&](int j) -> bool {
+            const int s = j & 1, st = j % C::kStages;
+            const uint32_t slot = tmem + s * C::kSlot;
+            // O_conv shares TMEM columns with the second half of S: the conv product waits for P too
+            if (!wait(&p_full[s], (j >> 1) & 1)) return false;
+            tc_fence_after();
+            if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < M / 16; ++k) {
                     // landmarks 16k .. 16k+15: first half from P_A, second half from P_B
                     const uint32_t pa = k < M / 32 ? slot + C::kColPA + k * 8 : slot + C::kColPB + (k - M / 32) * 8;
                     mma_bf16_ts(slot + C::kColOatt, pa, descWt(k), C::kIdPW, k > 0);
                 }
-                if (prm.conv_w != nullptr) {
-                    if (!mbar_wait(&v_full[st], (j / C::kStages) & 1)) return false;
-                    tc_fence_after();
+            }
+            if (prm.conv_w != nullptr) {
+                if (!wait(&v_full[st], (j / C::kStages) & 1)) return false;
+                tc_fence_after();
+                if (elect_one()) {
 #pragma unroll
                     for (int k = 0; k < 12; ++k)
                         mma_bf16_ss(slot + C::kColOconv, descT(k), descV(st, k), C::kIdConv, k > 0);
                 }
-                mma_commit(&o_full[s]);
-                if (prm.conv_w != nullptr) mma_commit(&v_empty[st]);
-                return true;
-            };
-            if (count > 0) {
-                ok = mbar_wait(const_full, cf_phase) && mbar_wait(t_full, cf_phase);
+                if (elect_one()) mma_commit(&v_empty[st]);
+            }
+            if (elect_one()) mma_commit(&o_full[s]);
+            return true;
+        };
+        if (count > 0) {
+            ok = wait(const_full, cf_phase) && wait(t_full, cf_phase);
+            cf_phase ^= 1;
+            tc_fence_after();
+            if (ok) ok = issue_S(0);
+        }
+        for (int i = 0; i < count && ok && !warp_any(*abort_flag != 0); ++i) {
+            const bool has_next = i + 1 < count;
+            const bool next_new_head = has_next && head_start(i + 1);
+            if (has_next && !next_new_head) ok = issue_S(i + 1);
+            if (ok) ok = issue_O(i);
+            if (ok && next_new_head) {
+                if (elect_one()) mma_commit(const_empty);
+                ok = wait(const_full, cf_phase) && wait(t_full, cf_phase);
                 cf_phase ^= 1;
                 tc_fence_after();
-                if (ok) ok = issue_S(0);
+                if (ok) ok = issue_S(i + 1);
             }
-            for (int i = 0; i < count && ok && !*abort_flag; ++i) {
-                const bool has_next = i + 1 < count;
-                const bool next_new_head = has_next && head_start(i + 1);
-                if (has_next && !next_new_head) ok = issue_S(i + 1);
-                if (ok) ok = issue_O(i);
-                if (ok && next_new_head) {
-                    mma_commit(const_empty);
-                    ok = mbar_wait(const_full, cf_phase) && mbar_wait(t_full, cf_phase);
-                    cf_phase ^= 1;
-                    tc_fence_after();
-                    if (ok) ok = issue_S(i + 1);
-                }
-            }
-            if (!ok) *abort_flag = 1;
-            // every MMA issued has completed before TMEM can be released
-            mma_commit(mma_done);
-            mbar_wait(mma_done, 0);
         }
+        if (!ok) *abort_flag = 1;
+        // every MMA issued has completed before TMEM can be released: one commit per lane
+        // (mma_done counts 32 arrivals), so the drain covers whichever lane issued
+        mma_commit(mma_done);
+        mbar_wait(mma_done, 0);
     } else if (warp >= 2 && warp < 10) {
         // ------------------------------------------------ softmax: two warpgroups, one tile,
         // group g reads landmark columns [g M/2, g M/2 + M/2) of its row

@@ -359,15 +359,20 @@ __global__ void __launch_bounds__(128, 1) pinv_tc_kernel(const PinvTcParams prm)
                         ++consumed;
                         tc_fence_after();
                         const uint32_t sa = sbase + st * C::kStage, sb = sa + C::kAChunk;
+                        // one operand form per group of four MMAs: a run-time choice between
+                        // forms inside the group serialises the MMAs
+                        if (a_src) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t bdesc = smem_desc(sb + kk * 32, 16, 1024, kLayoutSw128);
-                            const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
-                            if (a_src)
-                                mma_tf32_ss(d_col, smem_desc(sa + kk * 32, 16, 1024, kLayoutSw128), bdesc,
-                                            C::kIdesc, acc);
-                            else
-                                mma_tf32_ts(d_col, (uint32_t)a_tmem + c * 32 + kk * 8, bdesc, C::kIdesc, acc);
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_tf32_ss(d_col, smem_desc(sa + kk * 32, 16, 1024, kLayoutSw128),
+                                            smem_desc(sb + kk * 32, 16, 1024, kLayoutSw128), C::kIdesc,
+                                            (c > 0 || kk > 0) ? 1u : 0u);
+                        } else {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_tf32_ts(d_col, (uint32_t)a_tmem + c * 32 + kk * 8,
+                                            smem_desc(sb + kk * 32, 16, 1024, kLayoutSw128), C::kIdesc,
+                                            (c > 0 || kk > 0) ? 1u : 0u);
                         }
                         mma_commit(&empty[st]);
                         // refill the stage of the previous chunk with chunk c - 1 + kStages

@@ -210,7 +210,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         mbar_init(mma4_done, 1);
         mbar_init(e_ready, 16);    // one arrival per epilogue warp of either CTA
         mbar_init(wl_ready, 16);
-        mbar_init(drain, 1);
+        mbar_init(drain, 32);     // one commit per lane of the MMA warp
         mbar_init(pro_full, 1);
         mbar_init(cs_ready, 8);    // one arrival per epilogue warp of the peer
         fence_mbar_init();
@@ -267,29 +267,32 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         }
         __syncwarp();
     } else if (warp == 9) {
-        // ------------------------------------------------ MMA issuer (first CTA of the pair)
-        if (leader && lane == 0) {
+        // ------------------------------------------------ MMA issuer (first CTA of the pair): the
+        // whole warp runs the loop and the waits; one elected lane issues each MMA group and commit
+        if (leader) {
             const uint32_t bs = smem_u32(bbuf);
             bool ok = true;
             uint32_t ne = 0, nf = 0;   // e_ready phases waited, streamed products issued
             // kernel_2: S2 = Q_l K_l^T from split tf32 operands, hi.hi + hi.lo + lo.hi
-            ok = wait_acq_cluster(e_ready, ne & 1u);
+            ok = warp_all(wait_acq_cluster(e_ready, ne & 1u));
             ++ne;
             if (ok) {
                 tc_fence_after();
-                const uint32_t aoff[3] = {C::kOffAhi, C::kOffAhi, C::kOffAlo};
-                const uint32_t boff[3] = {C::kOffBhi, C::kOffBlo, C::kOffBhi};
-                uint32_t acc = 0;
-                for (int t = 0; t < 3; ++t)
-                    for (int a = 0; a < nka; ++a)
+                if (elect_one()) {
+                    const uint32_t aoff[3] = {C::kOffAhi, C::kOffAhi, C::kOffAlo};
+                    const uint32_t boff[3] = {C::kOffBhi, C::kOffBlo, C::kOffBhi};
+                    uint32_t acc = 0;
+                    for (int t = 0; t < 3; ++t)
+                        for (int a = 0; a < nka; ++a)
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t ka = a * C::kAtomBytes + kk * 32;
-                            mma2_ss(R1, smem_desc(bs + aoff[t] + ka, 16, 1024, kLayoutSw128),
-                                    smem_desc(bs + boff[t] + ka, 16, 1024, kLayoutSw128), C::kIdesc, acc);
-                            acc = 1;
-                        }
-                commit2(mma_done, 3);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                const uint32_t ka = a * C::kAtomBytes + kk * 32;
+                                mma2_ss(R1, smem_desc(bs + aoff[t] + ka, 16, 1024, kLayoutSw128),
+                                        smem_desc(bs + boff[t] + ka, 16, 1024, kLayoutSw128), C::kIdesc, acc);
+                                acc = 1;
+                            }
+                }
+                if (elect_one()) commit2(mma_done, 3);
             }
             for (int it = 0; it < n_iter && ok; ++it) {
                 for (int p = 0; p < 4 && ok; ++p) {
@@ -297,29 +300,32 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                     const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
                     const bool streamed = p == 3 || (p == 0 && it > 0);
                     if (p != 0 || it == 0) {
-                        ok = wait_acq_cluster(e_ready, ne & 1u);   // left factor (and X, or k2) in place
+                        ok = warp_all(wait_acq_cluster(e_ready, ne & 1u));   // left factor (and X, or k2) in place
                         ++ne;
                         if (!ok) break;
                     }
                     tc_fence_after();
                     for (int kc = 0; kc < 8; ++kc) {
                         if (streamed) {
-                            ok = mbar_wait(&bfull[kc], nf & 1u);
+                            ok = warp_all(mbar_wait(&bfull[kc], nf & 1u));
                             if (!ok) break;
                             tc_fence_after();
                         }
+                        if (elect_one()) {
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            mma2_ts(d_col, a_col + kc * 32 + kk * 8,
-                                    smem_desc(bs + kc * C::kAtomBytes + kk * 32, 16, 1024, kLayoutSw128), C::kIdesc,
-                                    (kc | kk) != 0 ? 1u : 0u);
-                        if (p >= 2) commit2(&bfree[kc], 3);   // the producer refills this atom next
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma2_ts(d_col, a_col + kc * 32 + kk * 8,
+                                        smem_desc(bs + kc * C::kAtomBytes + kk * 32, 16, 1024, kLayoutSw128),
+                                        C::kIdesc, (kc | kk) != 0 ? 1u : 0u);
+                            if (p >= 2) commit2(&bfree[kc], 3);   // the producer refills this atom next
+                        }
                     }
                     if (streamed) ++nf;
-                    if (ok) commit2(p == 3 ? mma4_done : mma_done, 3);
+                    if (ok && elect_one()) commit2(p == 3 ? mma4_done : mma_done, 3);
                 }
             }
-            // every MMA issued here has completed before the pair tears down
+            // every MMA issued here has completed before the pair tears down: one commit per
+            // lane (drain counts 32 arrivals), so the drain covers whichever lane issued
             commit2(drain, 1);
             mbar_wait(drain, 0);
         }
