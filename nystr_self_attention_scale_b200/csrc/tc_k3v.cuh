@@ -16,16 +16,24 @@
 // max exceeds it by more than 2^8 (log2 units); then O and the running sum are
 // rescaled once. Every exponential of a row uses the same reference, so the
 // result is the exact softmax; P stays below 256, well inside bf16 range.
-// Each item writes the unnormalised partial (O, reference max, running sum) of
-// its split; a deterministic combine over splits follows.
+// An item's chunks run as two independent streams: chunk c goes to stream
+// c % 2, which has its own S buffer, P buffer, O accumulator, reference max
+// and running sum in TMEM / registers. P has its own TMEM columns, so a
+// stream's next S MMA only waits until the softmax has loaded the current
+// scores, and runs while the exponentials are computed. Each stream writes the
+// unnormalised partial (O, reference max, running sum) of its half of the
+// split as a partial of its own (split 2 s + stream); a deterministic combine
+// over the partials follows. The stream of a chunk depends only on its place
+// in its split, so a head's result does not depend on the rest of the batch.
 //
-// Warp roles (640 threads): warp 0 TMA producer and TMEM allocator, warp 1 MMA
-// issuer, warps 4-19 four softmax warpgroups that split every chunk's 128 keys
-// (32 each), exchanging the chunk max through shared memory; four warps per
-// SM sub-partition hide the TMEM and MUFU latencies. Each group writes its P
-// into the first half of its own 32 S columns (the P.V MMA takes its A
-// operand from the four ranges). S is double buffered in TMEM; K/V chunks use
-// a 3-stage shared-memory ring.
+// Warp roles (608 threads): warp 0 TMA producer and TMEM allocator, warps 1
+// and 18 the MMA issuers of streams 0 and 1 (so that neither stream's MMAs wait
+// behind the other's), warps 2-17 the softmax: stream t owns warps 2 + 8 t .. 9 + 8 t, two
+// warpgroups that split each of its chunks' 128 keys (64 each), exchanging the
+// chunk max through shared memory. Each SM sub-partition runs four softmax
+// warps, two per stream. Each group writes its P (bf16 pairs) into its half
+// of the stream's P buffer.
+// K/V chunks use a 4-stage shared-memory ring.
 #pragma once
 
 #include "sm100.cuh"
@@ -38,38 +46,39 @@ struct K3vTc {
     static constexpr int kSpan = D * 2;
     static constexpr uint32_t kLayout = D == 64 ? sm100::kLayoutSw128 : sm100::kLayoutSw64;
     static constexpr uint32_t kSbo = 8 * kSpan;
-    static constexpr int kStages = 3;
+    static constexpr int kStages = 4;
     static constexpr uint32_t kTileBytes = 128 * kSpan;
     static constexpr uint32_t kOffQl = 0;
     static constexpr uint32_t kOffK = kOffQl + kTileBytes;
     static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
     static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
-    static constexpr int kNumBars = 2 + 2 * kStages + 7 + 1;
-    static constexpr int kGroups = 4;                                     // softmax warpgroups
-    static constexpr int kSoftmaxThreads = kGroups * 128;
-    static constexpr int kThreads = 128 + kSoftmaxThreads;               // warps 0-3 + the groups
-    static constexpr uint32_t kOffXch = kOffBar + kNumBars * 8;          // [2][4][128] chunk maxima
-    static constexpr uint32_t kOffLx = kOffXch + 2 * kGroups * 128 * 4;  // [4][128] partial sums
-    static constexpr uint32_t kOffMisc = kOffLx + kGroups * 128 * 4;
+    static constexpr int kNumBars = 2 + 2 * kStages + 10 + 1;
+    static constexpr int kStreams = 2;                                    // softmax streams
+    static constexpr int kTeamThreads = 256;                              // two warpgroups per stream
+    static constexpr int kThreads = 96 + kStreams * kTeamThreads;        // warps 0, 1, 18 + the streams
+    static constexpr uint32_t kOffXch = kOffBar + kNumBars * 8;          // [2 streams][2 groups][128] maxima
+    static constexpr uint32_t kOffLx = kOffXch + 2 * 2 * 128 * 4;        // [2 streams][2 groups][128] sums
+    static constexpr uint32_t kOffMisc = kOffLx + 2 * 2 * 128 * 4;
     // at least 116 KB so that only one CTA (and one 512-column TMEM allocation) fits per SM
     static constexpr uint32_t kSmemNeed = kOffMisc + 16 + 1024;
     static constexpr uint32_t kSmemBytes = kSmemNeed > 118784 ? kSmemNeed : 118784;
     static constexpr int kTmemCols = 512;
-    static constexpr int kColS = 0, kColO = 256;   // S[b] at 128 b; P halves at 128 b + {0, 64}
+    // TMEM columns of stream t: S at 128 t, P (bf16 pairs) at 256 + 64 t, O at 384 + D t
+    static constexpr int kColS = 0, kColP = 256, kColO = 384;
     static constexpr uint32_t kIdS = sm100::make_idesc(128, kChunk, sm100::kFmtBf16, sm100::kFmtBf16, 0, 0);
     static constexpr uint32_t kIdPV = sm100::make_idesc(128, D, sm100::kFmtBf16, sm100::kFmtBf16, 0, 1);
 };
 
 struct K3vTcParams {
     const uint32_t* mask_bits;  // [B, n / 32] key-validity bits, or null for no mask
-    float* part_o;         // [BH, splits, m, d]
-    float* part_m;         // [BH, splits, m]  running max (natural-log units)
-    float* part_l;         // [BH, splits, m]  running sum
+    float* part_o;         // [BH, 2 splits, m, d]  (partial 2 s + t: stream t of split s)
+    float* part_m;         // [BH, 2 splits, m]  running max (natural-log units)
+    float* part_l;         // [BH, 2 splits, m]  running sum
     int H, n, m, halves, splits, chunks_per_split, total_items;
 };
 
 template <int D>
-__global__ void __launch_bounds__(640, 1)
+__global__ void __launch_bounds__(K3vTc<D>::kThreads, 1)
 k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant__ CUtensorMap map_k,
               const __grid_constant__ CUtensorMap map_v, const K3vTcParams prm) {
     using C = K3vTc<D>;
@@ -82,11 +91,12 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
     uint64_t* ql_empty = bars + 1;
     uint64_t* kv_full = bars + 2;                  // [kStages]
     uint64_t* kv_empty = bars + 2 + C::kStages;    // [kStages]
-    uint64_t* s_full = bars + 2 + 2 * C::kStages;  // [2] S(j) in TMEM
-    uint64_t* p_full = s_full + 2;                 // [2] P(j) in TMEM (128 arrivals)
-    uint64_t* pv_done = s_full + 4;                // [2] P(j) V(j) accumulated into O
-    uint64_t* o_free = s_full + 6;                 // the item's O has been read (128 arrivals)
-    uint64_t* mma_done = s_full + 7;
+    uint64_t* s_full = bars + 2 + 2 * C::kStages;  // [stream] S of its current chunk in TMEM
+    uint64_t* p_full = s_full + 2;                 // [stream] P in TMEM (256 arrivals)
+    uint64_t* pv_done = s_full + 4;                // [stream] P V accumulated into its O
+    uint64_t* o_free = s_full + 6;                 // [stream] the item's O has been read (256 arrivals)
+    uint64_t* s_free = s_full + 8;                 // [stream] its S has been loaded (256 arrivals)
+    uint64_t* mma_done = s_full + 10;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
 
@@ -102,18 +112,19 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
 
     if (threadIdx.x == 0) {
         mbar_init(ql_full, 1);
-        mbar_init(ql_empty, 1);
+        mbar_init(ql_empty, 2);   // one commit per MMA issuer
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&kv_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], C::kSoftmaxThreads);
+            mbar_init(&p_full[b], C::kTeamThreads);
             mbar_init(&pv_done[b], 1);
+            mbar_init(&o_free[b], C::kTeamThreads);
+            mbar_init(&s_free[b], C::kTeamThreads);
         }
-        mbar_init(o_free, C::kSoftmaxThreads);
-        mbar_init(mma_done, 32);   // one commit per lane of the MMA warp
+        mbar_init(mma_done, 64);   // one commit per lane of the two MMA warps
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -161,11 +172,12 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 if (ql_issued >= 0) mbar_wait(ql_full, ql_issued & 1);
             }
         }
-    } else if (warp == 1) {
-        // MMA issuer: the whole warp runs the loop and the waits; one elected lane issues each
-        // MMA group and each commit
+    } else if (warp == 1 || warp == 18) {
+        // MMA issuer of stream t (chunks c of an item with c % 2 == t): the whole warp runs the
+        // loop and the waits; one elected lane issues each MMA group and each commit
+        const int t = warp == 1 ? 0 : 1;
         bool ok = true;
-        int g = 0, it = 0;
+        int g = 0, it = 0, u = 0;   // chunks before this item, items, chunks of this stream
         auto descQl = [&](int k) { return smem_desc(sbase + C::kOffQl + k * 32, 16, C::kSbo, C::kLayout); };
         auto descK = [&](int st, int k) {
             return smem_desc(sbase + C::kOffK + st * C::kTileBytes + k * 32, 16, C::kSbo, C::kLayout);
@@ -175,40 +187,6 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                              C::kLayout);
         };
         auto wait = [&](uint64_t* bar, uint32_t parity) { return warp_all(mbar_wait(bar, parity)); };
-        auto issue_S = [&](int j) -> bool {
-            const int b = j & 1, st = j % C::kStages;
-            // S buffer b last held S(j - 2); P(j - 2) V was accumulated once PV(j - 2) completed
-            if (j >= 2 && !wait(&pv_done[b], ((j - 2) >> 1) & 1)) return false;
-            if (!wait(&kv_full[st], (j / C::kStages) & 1)) return false;
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k)
-                    mma_bf16_ss(tmem + C::kColS + b * 128, descQl(k), descK(st, k), C::kIdS, k > 0);
-            }
-            if (elect_one()) mma_commit(&s_full[b]);
-            return true;
-        };
-        auto issue_PV = [&](int j, bool first, int item_it) -> bool {
-            const int b = j & 1, st = j % C::kStages;
-            if (!wait(&p_full[b], (j >> 1) & 1)) return false;
-            // the previous item's O must have been read before it is overwritten
-            if (first && !wait(o_free, (item_it & 1) ^ 1)) return false;
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int k = 0; k < C::kChunk / 16; ++k) {
-                    // keys 16k .. 16k+15: P of group k / 2, at the start of its 32 S columns
-                    const uint32_t pa = tmem + C::kColS + b * 128 + 32 * (k >> 1) + 8 * (k & 1);
-                    mma_bf16_ts(tmem + C::kColO, pa, descV(st, k), C::kIdPV, (first && k == 0) ? 0u : 1u);
-                }
-            }
-            if (elect_one()) {
-                mma_commit(&pv_done[b]);
-                mma_commit(&kv_empty[st]);
-            }
-            return true;
-        };
         for (int item = blockIdx.x; item < prm.total_items && ok && !warp_any(*abort_flag != 0);
              item += gridDim.x, ++it) {
             int c0;
@@ -216,32 +194,78 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             ok = wait(ql_full, it & 1);
             if (!ok) break;
             tc_fence_after();
-            ok = issue_S(g);
-            for (int c = 0; c < nch && ok; ++c) {
-                const int j = g + c;
-                if (c + 1 < nch) ok = issue_S(j + 1);
-                else if (elect_one()) mma_commit(ql_empty);   // every S MMA of this item is issued
-                if (ok) ok = issue_PV(j, c == 0, it);
+            // S of chunk c (the stream's u-th): its S buffer is free once the softmax has loaded
+            // the previous scores
+            auto issue_S = [&](int c, int uu) -> bool {
+                const int gc = g + c, st = gc % C::kStages;
+                if (uu > 0 && !wait(&s_free[t], (uu - 1) & 1)) return false;
+                if (!wait(&kv_full[st], (gc / C::kStages) & 1)) return false;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_bf16_ss(tmem + C::kColS + t * 128, descQl(k), descK(st, k), C::kIdS, k > 0);
+                }
+                if (elect_one()) mma_commit(&s_full[t]);
+                return true;
+            };
+            if (t < nch) ok = issue_S(t, u);
+            for (int c = t; c < nch && ok; c += 2, ++u) {
+                const int gc = g + c, st = gc % C::kStages;
+                // the next S of the stream goes first, so that it runs during this chunk's softmax
+                if (c + 2 < nch) {
+                    if (!(ok = issue_S(c + 2, u + 1))) break;
+                } else if (elect_one()) {
+                    mma_commit(ql_empty);   // this stream's last S of the item is issued
+                }
+                // P V into the stream's O, once its softmax has written P; the first of the item
+                // also waits until the stream's previous O has been read
+                const bool first = c < 2;
+                if (!(ok = wait(&p_full[t], u & 1))) break;
+                if (first && !(ok = wait(&o_free[t], (it & 1) ^ 1))) break;
+                tc_fence_after();
+                if (elect_one()) {
+#pragma unroll
+                    for (int k = 0; k < C::kChunk / 16; ++k) {
+                        // keys 16k .. 16k+15: P of group k / 4, in its 32 columns of the P buffer
+                        const uint32_t pa = tmem + C::kColP + t * 64 + 32 * (k >> 2) + 8 * (k & 3);
+                        mma_bf16_ts(tmem + C::kColO + t * D, pa, descV(st, k), C::kIdPV,
+                                    (first && k == 0) ? 0u : 1u);
+                    }
+                }
+                if (elect_one()) {
+                    mma_commit(&pv_done[t]);
+                    mma_commit(&kv_empty[st]);
+                }
             }
+            // a stream with no chunk in this item still releases Q_l once
+            if (ok && t >= nch && elect_one()) mma_commit(ql_empty);
             g += nch;
         }
         if (!ok) *abort_flag = 1;
-        // one commit per lane (mma_done counts 32 arrivals): the drain covers whichever lane issued
+        // one commit per lane (mma_done counts both warps' 64 arrivals): the drain covers
+        // whichever lane issued
         mma_commit(mma_done);
         mbar_wait(mma_done, 0);
-    } else if (warp >= 4) {
-        const int grp = (warp - 4) >> 2;          // softmax group: keys [32 grp, 32 grp + 32) of a chunk
+    } else if (warp >= 2 && warp < 18) {
+        const int sw = warp - 2;
+        const int t = sw >> 3;                      // stream: chunks c with c % 2 == t
+        const int grp = (sw >> 2) & 1;              // keys [64 grp, 64 grp + 64) of each chunk
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const float sc = split_scale(D) * kLog2e;   // exponent scale of the raw S = Q_l . K^T
         constexpr float kSlack = 8.f;               // log2 units: P stays below 2^8
-        constexpr int kT = C::kSoftmaxThreads;
-        float* xch = reinterpret_cast<float*>(sm + C::kOffXch);   // [2 buffers][4 groups][128]
-        float* lx = reinterpret_cast<float*>(sm + C::kOffLx);     // [4 groups][128]
-        int g = 0, it = 0;
+        constexpr int kT = C::kTeamThreads;
+        const int bar_id = 1 + t;                   // this stream's named barrier
+        float* xch = reinterpret_cast<float*>(sm + C::kOffXch) + t * 256;   // [2 groups][128]
+        float* lx = reinterpret_cast<float*>(sm + C::kOffLx) + t * 256;     // [2 groups][128]
+        const uint32_t sbuf = tmem + lane_base + C::kColS + t * 128 + 64 * grp;
+        const uint32_t pbuf = tmem + lane_base + C::kColP + t * 64 + 32 * grp;
+        const uint32_t obuf = tmem + lane_base + C::kColO + t * D + 32 * grp;
+        int u = 0, it = 0;   // chunks this stream has taken, items
         for (int item = blockIdx.x; item < prm.total_items; item += gridDim.x, ++it) {
-            if (group_any(*abort_flag != 0, 1, kT)) break;
+            if (group_any(*abort_flag != 0, bar_id, kT)) break;
             const int bh = item / per_bh, half = (item / prm.splits) % prm.halves;
             const int split = item % prm.splits;
             const int b_idx = bh / prm.H;
@@ -249,58 +273,62 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             const int nch = item_chunks(item, &c0);
             float m_ref = -INFINITY, l_run = 0.f;   // reference max (log2 units) and this group's sum
             bool ok = true;
-            for (int c = 0; c < nch; ++c) {
-                const int j = g + c, b = j & 1;
-                const int key0 = (c0 + c) * C::kChunk;
-                // key-validity bits of this group's 32 keys (bit k = key key0 + 32 grp + k)
-                const uint32_t mb = prm.mask_bits != nullptr
-                                        ? __ldg(prm.mask_bits + (size_t)b_idx * (prm.n / 32) + key0 / 32 + grp)
-                                        : ~0u;
-                const bool full = mb == ~0u;
+            int mine = 0;                           // chunks of this item taken by the stream
+            for (int c = t; c < nch; c += 2, ++u, ++mine) {
+                const int key0 = (c0 + c) * C::kChunk + 64 * grp;
+                // key-validity bits of this group's 64 keys (bit k of word h = key key0 + 32 h + k)
+                uint32_t mb[2] = {~0u, ~0u};
+                if (prm.mask_bits != nullptr) {
+                    const uint32_t* w = prm.mask_bits + (size_t)b_idx * (prm.n / 32) + key0 / 32;
+                    mb[0] = __ldg(w);
+                    mb[1] = __ldg(w + 1);
+                }
+                const bool full = (mb[0] & mb[1]) == ~0u;
                 // a wait that runs out leaves S unread: the group still passes the chunk's one
-                // barrier below (which also ORs the failure across the groups) and then stops
-                ok = warp_all(mbar_wait(&s_full[b], (j >> 1) & 1));
+                // barrier below (which also ORs the failure across the two groups) and then stops
+                ok = warp_all(mbar_wait(&s_full[t], u & 1));
                 tc_fence_after();
-                const uint32_t sbuf = tmem + lane_base + C::kColS + b * 128;
-                uint32_t v[32];
-                if (ok) {
-                    tmem_ld32(sbuf + 32 * grp, v);
-                    tmem_ld_wait();
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) v[e] = 0u;
-                }
-                if (!full) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (!((mb >> e) & 1u)) v[e] = __float_as_uint(-INFINITY);
-                }
+                // pass 1: the max of this group's 64 scores (the scores are loaded again for the
+                // exponentials, which keeps the register footprint small)
                 float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four short max chains
+                if (ok) {
+                    uint32_t v[2][32];   // keys 32 h + e of this group's 64
+                    tmem_ld32(sbuf, v[0]);
+                    tmem_ld32(sbuf + 32, v[1]);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    mq[e & 3] = max3(mq[e & 3], __uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-                xch[(b * 4 + grp) * 128 + r] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-                if (group_any(!ok, 1, kT)) { ok = false; break; }   // also publishes xch
-                const float* xr = xch + b * 4 * 128 + r;
-                const float cmax = fmaxf(fmaxf(xr[0], xr[128]), fmaxf(xr[256], xr[384]));
-                const float cm = cmax * sc;
+                    for (int h = 0; h < 2; ++h) {
+                        if (!full) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if (!((mb[h] >> e) & 1u)) v[h][e] = __float_as_uint(-INFINITY);
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            mq[(2 * h + e) & 3] = max3(mq[(2 * h + e) & 3], __uint_as_float(v[h][2 * e]),
+                                                       __uint_as_float(v[h][2 * e + 1]));
+                    }
+                }
+                xch[grp * 128 + r] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+                if (group_any(!ok, bar_id, kT)) { ok = false; break; }   // also publishes xch
+                const float cm = fmaxf(xch[r], xch[128 + r]) * sc;
                 // move the reference only when this chunk's max exceeds it by more than the slack
-                // (every group takes the same decision: same maxima, same history)
+                // (both groups take the same decision: same maxima, same history)
                 const bool move = cm > m_ref + kSlack;
                 const float m_new = move ? cm : m_ref;
                 const float alpha = move ? ex2(m_ref - m_new) : 1.f;   // m_ref = -inf gives 0
-                if (grp < D / 32 && c > 0 && warp_any(move && m_ref != -INFINITY)) {
-                    // rescale this warp's rows of O (group g: columns 32 g .. 32 g + 31) once
-                    // P(j - 1) V has been accumulated
-                    ok = warp_all(mbar_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1));
+                if (grp < D / 32 && mine > 0 && warp_any(move && m_ref != -INFINITY)) {
+                    // rescale this warp's rows of O (group g: columns 32 g .. 32 g + 31) once the
+                    // stream's previous P V has been accumulated
+                    ok = warp_all(mbar_wait(&pv_done[t], (u - 1) & 1));
                     if (ok) {
                         tc_fence_after();
                         uint32_t o[32];
-                        tmem_ld32(tmem + lane_base + C::kColO + grp * 32, o);
+                        tmem_ld32(obuf, o);
                         tmem_ld_wait();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tmem + lane_base + C::kColO + grp * 32, o);
+                        tmem_st32(obuf, o);
                     }
                 }
                 const float mo = m_new == -INFINITY ? 0.f : m_new;   // rows with every key padded so far: P = 0
@@ -310,38 +338,62 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 // bf16 (nearest even); the running sum adds the fp32 values.
                 const uint64_t sc2 = f2(sc, sc), nmo2 = f2(-mo, -mo);
                 uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-                uint32_t pk[16];
-                if (full) {
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h) {
+                    // pass 2, 32 keys per TMEM load; after the last load the S buffer is released
+                    // to the stream's next S MMA
+                    uint32_t v[32];
+                    tmem_ld32(sbuf + 32 * h, v);
+                    tmem_ld_wait();
+                    if (h == 1) {
+                        tc_fence_before();
+                        mbar_arrive(&s_free[t]);
+                    }
+                    if (!full) {
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint64_t x2 =
-                            f2_fma(f2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, nmo2);
-                        float e0, e1;
-                        if ((e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7) {
-                            exp2_poly_pair(x2, e0, e1);
-                        } else {
+                        for (int e = 0; e < 32; ++e)
+                            if (!((mb[h] >> e) & 1u)) v[e] = __float_as_uint(-INFINITY);
+                    }
+                    uint32_t pk[16];
+                    if (full) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const uint64_t x2 = f2_fma(
+                                f2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2,
+                                nmo2);
+                            float e0, e1;
+                            if ((e & 7) == 2 || (e & 7) == 5 || (e & 7) == 7) {
+                                exp2_poly_pair(x2, e0, e1);
+                            } else {
+                                float x0, x1;
+                                f2_split(x2, x0, x1);
+                                e0 = ex2(x0);
+                                e1 = ex2(x1);
+                            }
+                            pk[e] = pack_bf16_rn(e0, e1);
+                            acc[e & 1] = f2_add(acc[e & 1], f2(e0, e1));
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const uint64_t x2 = f2_fma(
+                                f2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2,
+                                nmo2);
                             float x0, x1;
                             f2_split(x2, x0, x1);
-                            e0 = ex2(x0);
-                            e1 = ex2(x1);
+                            const float e0 = ex2(x0), e1 = ex2(x1);
+                            pk[e] = pack_bf16_rn(e0, e1);
+                            acc[e & 1] = f2_add(acc[e & 1], f2(e0, e1));
                         }
-                        pk[e] = pack_bf16_rn(e0, e1);
-                        acc[e & 1] = f2_add(acc[e & 1], f2(e0, e1));
                     }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const uint64_t x2 =
-                            f2_fma(f2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1])), sc2, nmo2);
-                        float x0, x1;
-                        f2_split(x2, x0, x1);
-                        const float e0 = ex2(x0), e1 = ex2(x1);
-                        pk[e] = pack_bf16_rn(e0, e1);
-                        acc[e & 1] = f2_add(acc[e & 1], f2(e0, e1));
+                    // this group's P (keys 32 h ..) into its 32 columns of the P buffer, which the
+                    // stream's previous P V must have finished reading
+                    if (h == 0 && u > 0) {
+                        if (!warp_all(mbar_wait(&pv_done[t], (u - 1) & 1))) ok = false;
+                        tc_fence_after();
                     }
+                    tmem_st16(pbuf + 16 * h, pk);
                 }
-                // this group's P: 16 columns at the start of its own (already read) 32 S columns
-                tmem_st16(sbuf + 32 * grp, pk);
                 float sum;
                 {
                     float a0, a1, b0, b1;
@@ -351,41 +403,48 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 }
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&p_full[b]);
+                mbar_arrive(&p_full[t]);
                 l_run = fmaf(l_run, alpha, sum);
                 m_ref = m_new;
             }
-            // the item's O is complete once its last P V has been accumulated; groups 0 .. D/32 - 1
-            // each stream out 32 columns, group 0 adds the four partial sums
+            // the stream's partial of this split: its O is complete once its last P V has been
+            // accumulated; group g streams out columns 32 g .. 32 g + 31, group 0 adds the sums.
+            // A stream that took no chunk of the item writes an empty partial (O = 0, max -inf).
             const int row = half * C::kRows + r;
-            const size_t prow = ((size_t)bh * prm.splits + split) * prm.m + row;
-            if (ok && nch > 0 && grp < D / 32) {
-                const int jl = g + nch - 1;
-                ok = warp_all(mbar_wait(&pv_done[jl & 1], (jl >> 1) & 1));
-                if (ok) {
-                    tc_fence_after();
-                    uint32_t t[32];
-                    tmem_ld32(tmem + lane_base + C::kColO + grp * 32, t);
-                    tmem_ld_wait();
-                    if (row < prm.m) {
-                        float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D + grp * 32);
+            const size_t prow = ((size_t)bh * 2 * prm.splits + 2 * split + t) * prm.m + row;
+            if (ok && grp < D / 32) {
+                if (mine > 0) {
+                    ok = warp_all(mbar_wait(&pv_done[t], (u - 1) & 1));
+                    if (ok) tc_fence_after();
+                }
+                float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D + grp * 32);
+#pragma unroll 1
+                for (int h = 0; h < 2 && ok; ++h) {   // 16 columns per TMEM load
+                    uint32_t o[16];
+                    if (mine > 0) {
+                        tmem_ld16(obuf + 16 * h, o);
+                        tmem_ld_wait();
+                    } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            dst[e] = make_float4(__uint_as_float(t[4 * e]), __uint_as_float(t[4 * e + 1]),
-                                                 __uint_as_float(t[4 * e + 2]), __uint_as_float(t[4 * e + 3]));
+                        for (int e = 0; e < 16; ++e) o[e] = 0u;
+                    }
+                    if (row < prm.m) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            dst[4 * h + e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                                                         __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
                     }
                 }
             }
             tc_fence_before();
-            mbar_arrive(o_free);
+            mbar_arrive(&o_free[t]);
             lx[grp * 128 + r] = l_run;
-            if (group_any(!ok, 1, kT)) { *abort_flag = 1; break; }   // also publishes lx
-            g += nch;
+            if (group_any(!ok, bar_id, kT)) { *abort_flag = 1; break; }   // also publishes lx
             if (grp == 0 && row < prm.m) {
                 prm.part_m[prow] = m_ref == -INFINITY ? -INFINITY : m_ref * kLn2;
-                prm.part_l[prow] = (lx[r] + lx[128 + r]) + (lx[256 + r] + lx[384 + r]);
+                prm.part_l[prow] = lx[r] + lx[128 + r];
             }
-            named_barrier(1, kT);   // lx is read before the next item overwrites it
+            named_barrier(bar_id, kT);   // lx is read before the next item overwrites it
         }
     }
 

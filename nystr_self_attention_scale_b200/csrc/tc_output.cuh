@@ -19,11 +19,11 @@
 // warps 10-13 epilogue (and the Toeplitz build), warp 14 TMA producer of the
 // V halos. A warp w reaches TMEM lanes 32 (w % 4) .. +31, so each group of four
 // warps covers all 128 rows. Two TMEM slots alternate between consecutive
-// tiles. Both softmax warpgroups work on the same tile, each on half of the
-// landmark columns (row maxima are exchanged through shared memory), which
-// halves the time a slot is held by the softmax. Each group writes its P
-// into its own half of the S columns, and the P.W MMA takes its A operand
-// from those two column ranges. Every wait is bounded.
+// tiles, and softmax group g owns slot g: it takes every other tile, whole
+// rows (all landmark columns), so neither group waits for the other and the
+// two, at different points of their tiles, hide each other's TMEM latency on
+// each SM sub-partition. P is written, packed, over the first M/2 columns of
+// the slot, where the P.W MMA reads its A operand. Every wait is bounded.
 #pragma once
 
 #include "sm100.cuh"
@@ -47,13 +47,13 @@ struct OutTc {
     static constexpr uint32_t kTBlock = 128 * 128;    // [128][64] bf16 K-block of T
     static constexpr uint32_t kTBytes = 3 * kTBlock;
     static constexpr uint32_t kOutBytes = kRows * kSpan;
-    // TMEM slot (256 columns): S in [0, M); P of the two column halves at [0, M/4) and
-    // [M/2, M/2 + M/4); O_att and O_conv in columns the softmax no longer needs
+    // TMEM slot (256 columns): S in [0, M); P (bf16 pairs) over [0, M/2); O_att and O_conv
+    // after P, in S columns the softmax has finished reading before the O MMAs are issued
     static constexpr int kSlot = 256;
     static constexpr int kTmemCols = 2 * kSlot;
-    static constexpr int kColPA = 0, kColPB = M / 2;
-    static constexpr int kColOatt = M == 256 ? M / 4 : M;
-    static constexpr int kColOconv = M == 256 ? 3 * M / 4 : M + D;
+    static constexpr int kColP = 0;
+    static constexpr int kColOatt = M == 256 ? M / 2 : M;
+    static constexpr int kColOconv = kColOatt + D;
     static_assert(kColOconv + D <= kSlot, "TMEM slot layout");
     static constexpr uint32_t kOffQ = 0;
     static constexpr uint32_t kOffV = kOffQ + kStages * kQBytes;
@@ -61,9 +61,8 @@ struct OutTc {
     static constexpr uint32_t kOffWt = kOffKl + kKlBytes;
     static constexpr uint32_t kOffT = kOffWt + kWtBytes;
     static constexpr uint32_t kOffOut = kOffT + kTBytes;
-    static constexpr uint32_t kOffPmax = kOffOut + kOutBytes;   // [2 slots][2 groups][128] float
-    static constexpr uint32_t kOffPsum = kOffPmax + 2 * 2 * 128 * 4;
-    static constexpr uint32_t kOffBar = kOffPsum + 2 * 2 * 128 * 4;
+    static constexpr uint32_t kOffPsum = kOffOut + kOutBytes;   // [2 slots][128] float row sums
+    static constexpr uint32_t kOffBar = kOffPsum + 2 * 128 * 4;
     static constexpr int kNumBars = 20;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -104,7 +103,6 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint64_t* v_empty = bars + 18;   // [2] V stage reusable (its conv MMA completed)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
-    float* pmax = reinterpret_cast<float*>(sm + C::kOffPmax);
     float* psum = reinterpret_cast<float*>(sm + C::kOffPsum);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -120,7 +118,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mbar_init(&q_full[b], 1);
             mbar_init(&q_empty[b], 1);
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 256);
+            mbar_init(&p_full[b], 128);
             mbar_init(&o_full[b], 1);
             mbar_init(&slot_free[b], 128);
             mbar_init(&v_full[b], 1);
@@ -243,11 +241,8 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             tc_fence_after();
             if (elect_one()) {
 #pragma unroll
-                for (int k = 0; k < M / 16; ++k) {
-                    // landmarks 16k .. 16k+15: first half from P_A, second half from P_B
-                    const uint32_t pa = k < M / 32 ? slot + C::kColPA + k * 8 : slot + C::kColPB + (k - M / 32) * 8;
-                    mma_bf16_ts(slot + C::kColOatt, pa, descWt(k), C::kIdPW, k > 0);
-                }
+                for (int k = 0; k < M / 16; ++k)   // landmarks 16k .. 16k+15: 8 packed P columns
+                    mma_bf16_ts(slot + C::kColOatt, slot + C::kColP + k * 8, descWt(k), C::kIdPW, k > 0);
             }
             if (prm.conv_w != nullptr) {
                 if (!wait(&v_full[st], (j / C::kStages) & 1)) return false;
@@ -287,29 +282,26 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         mma_commit(mma_done);
         mbar_wait(mma_done, 0);
     } else if (warp >= 2 && warp < 10) {
-        // ------------------------------------------------ softmax: two warpgroups, one tile,
-        // group g reads landmark columns [g M/2, g M/2 + M/2) of its row
-        constexpr int kHalf = M / 2;
+        // ------------------------------------------------ softmax: group g takes the tiles i with
+        // i % 2 == g (TMEM slot g), one whole row of S per thread
         const int g = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const float sc = split_scale(D) * kLog2e;  // S holds Q . K_l^T with K_l already scaled
-        for (int i = 0; i < count && !warp_any(*abort_flag != 0); ++i) {
-            const int s = i & 1;
-            const bool ok = warp_all(mbar_wait(&s_full[s], (i >> 1) & 1));
+        constexpr int kB = M < 64 ? M : 64;        // S columns per TMEM wait
+        for (int i = g; i < count && !warp_any(*abort_flag != 0); i += 2) {
+            const int s = g;
+            if (!warp_all(mbar_wait(&s_full[s], (i >> 1) & 1))) { *abort_flag = 1; break; }
             tc_fence_after();
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
-            const uint32_t scol = slot + g * kHalf;
-            // pass 1: the max of this half-row, 64 columns per wait (skipped after a failed wait;
-            // the exchange barrier below ORs the failure over both groups)
-            constexpr int kB = kHalf < 64 ? kHalf : 64;
+            // pass 1: the row max, kB columns per wait
             float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four short max chains
 #pragma unroll 1
-            for (int c0 = 0; c0 < (ok ? kHalf : 0); c0 += kB) {
+            for (int c0 = 0; c0 < M; c0 += kB) {
                 uint32_t v[kB / 32][32];
 #pragma unroll
-                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(scol + c0 + bq * 32, v[bq]);
+                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(slot + c0 + bq * 32, v[bq]);
                 tmem_ld_wait();
 #pragma unroll
                 for (int bq = 0; bq < kB / 32; ++bq)
@@ -317,24 +309,19 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     for (int j = 0; j < 16; ++j)
                         mq[j & 3] = max3(mq[j & 3], __uint_as_float(v[bq][2 * j]), __uint_as_float(v[bq][2 * j + 1]));
             }
-            float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-            pmax[(s * 2 + g) * 128 + r] = mx;
-            if (group_any(!ok, 3, 256)) { *abort_flag = 1; break; }   // also publishes pmax
-            mx = fmaxf(mx, pmax[(s * 2 + (g ^ 1)) * 128 + r]);
-            const float mo = mx * sc;
-            // pass 2: P into this group's own half of the S columns, in increasing column order,
-            // so it only overwrites scores this thread has already read
-            const uint32_t pcol = slot + (g == 0 ? C::kColPA : C::kColPB);
+            const float mo = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sc;
+            // pass 2: P over the first M/2 columns, in increasing column order, so it only
+            // overwrites scores this thread has already read.
             // exponentials on packed fp32 pairs: the MUFU unit takes 10 of every 16 pairs, the FMA
             // pipe the other 6 (polynomial 2^x), so neither pipe alone bounds the loop. P is rounded
             // to bf16 (nearest even); the row sum adds the fp32 values.
             const uint64_t sc2 = f2(sc, sc), nmo2 = f2(-mo, -mo);
             uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
 #pragma unroll 1
-            for (int c0 = 0; c0 < kHalf; c0 += kB) {
+            for (int c0 = 0; c0 < M; c0 += kB) {
                 uint32_t v[kB / 32][32];
 #pragma unroll
-                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(scol + c0 + bq * 32, v[bq]);
+                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(slot + c0 + bq * 32, v[bq]);
                 tmem_ld_wait();
 #pragma unroll
                 for (int bq = 0; bq < kB / 32; ++bq) {
@@ -355,7 +342,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         pk[j] = pack_bf16_rn(e0, e1);
                         acc[j & 1] = f2_add(acc[j & 1], f2(e0, e1));
                     }
-                    tmem_st16(pcol + (c0 + bq * 32) / 2, pk);
+                    tmem_st16(slot + C::kColP + (c0 + bq * 32) / 2, pk);
                 }
             }
             tmem_st_wait();
@@ -363,7 +350,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 float a0, a1, b0, b1;
                 f2_split(acc[0], a0, a1);
                 f2_split(acc[1], b0, b1);
-                psum[(s * 2 + g) * 128 + r] = (a0 + a1) + (b0 + b1);
+                psum[s * 128 + r] = (a0 + a1) + (b0 + b1);
             }
             tc_fence_before();
             mbar_arrive(&p_full[s]);
@@ -416,7 +403,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 break;
             }
             tc_fence_after();
-            const float li = 1.f / (psum[(s * 2) * 128 + r] + psum[(s * 2 + 1) * 128 + r]);
+            const float li = 1.f / psum[s * 128 + r];
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
             uint32_t outp[D / 2];
 #pragma unroll
