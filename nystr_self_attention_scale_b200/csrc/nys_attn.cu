@@ -220,7 +220,7 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
         // n = 16384) and fewer partials to merge
         p.tc_cps = std::min(chunks, n >= 16384 ? 26 : 8);
         p.tc_splits = (chunks + p.tc_cps - 1) / p.tc_cps;
-        splits = 2 * p.tc_splits;   // two partials (streams) per key split
+        splits = p.tc_splits;
         kps = p.tc_cps * 128;
     }
     p.splits = splits;

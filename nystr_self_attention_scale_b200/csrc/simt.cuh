@@ -352,14 +352,16 @@ k3v_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ p
 
 // W = Z (k3 V) (walkthrough 2.4, reassociated as k1 (Z (k3 V))): one CTA per
 // 64-row tile of one head; the inner dimension is staged 64 at a time through
-// shared memory with all of a thread's loads issued before its stores. Also
-// writes W^T in bf16 ([d, m] per head) when wt16 is given.
+// shared memory with all of a thread's loads issued before its stores. The Z
+// slice is stored transposed, so that a thread's four rows at one k are one
+// 16-byte shared load, as are its columns of k3V: two loads per 4 x CW block of
+// FMAs. Also writes W^T in bf16 ([d, m] per head) when wt16 is given.
 template <int D>
 __global__ void __launch_bounds__(256)
 w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __restrict__ w,
          __nv_bfloat16* __restrict__ wt16, int m) {
     constexpr int CW = D / 16;                       // columns per thread
-    __shared__ __align__(16) float sZ[64][64 + 4];   // [row][k]
+    __shared__ __align__(16) float sZ[64][64 + 4];   // [k][row]
     __shared__ __align__(16) float sK[64][D + 4];    // [k][col]
     const int bh = blockIdx.x, r0 = blockIdx.y * 64;
     const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
@@ -392,7 +394,7 @@ w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __re
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
             const int idx = tid + e * 256, r = idx >> 6, c = idx & 63;
-            sZ[r][c] = za[e];
+            sZ[c][r] = za[e];
         }
 #pragma unroll
         for (int e = 0; e < D / 16; ++e) {
@@ -403,9 +405,8 @@ w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __re
         if (k0 + 64 < m) load_slice(k0 + 64);
 #pragma unroll 8
         for (int kk = 0; kk < 64; ++kk) {
-            float a[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a[i] = sZ[ty * 4 + i][kk];
+            const float4 a4 = *reinterpret_cast<const float4*>(&sZ[kk][ty * 4]);
+            const float a[4] = {a4.x, a4.y, a4.z, a4.w};
             float bv[CW];
             if constexpr (CW == 4) {
                 const float4 b4 = *reinterpret_cast<const float4*>(&sK[kk][4 * tx]);

@@ -20,11 +20,12 @@
 // c % 2, which has its own S buffer, P buffer, O accumulator, reference max
 // and running sum in TMEM / registers. P has its own TMEM columns, so a
 // stream's next S MMA only waits until the softmax has loaded the current
-// scores, and runs while the exponentials are computed. Each stream writes the
-// unnormalised partial (O, reference max, running sum) of its half of the
-// split as a partial of its own (split 2 s + stream); a deterministic combine
-// over the partials follows. The stream of a chunk depends only on its place
-// in its split, so a head's result does not depend on the rest of the batch.
+// scores, and runs while the exponentials are computed. At the end of an item
+// the threads of stream 0 merge the two streams' (O, reference max, running
+// sum) row by row and write the unnormalised partial of the split; a
+// deterministic combine over splits follows. The stream of a chunk depends
+// only on its place in its split, so a head's result does not depend on the
+// rest of the batch.
 //
 // Warp roles (608 threads): warp 0 TMA producer and TMEM allocator, warps 1
 // and 18 the MMA issuers of streams 0 and 1 (so that neither stream's MMAs wait
@@ -58,7 +59,8 @@ struct K3vTc {
     static constexpr int kThreads = 96 + kStreams * kTeamThreads;        // warps 0, 1, 18 + the streams
     static constexpr uint32_t kOffXch = kOffBar + kNumBars * 8;          // [2 streams][2 groups][128] maxima
     static constexpr uint32_t kOffLx = kOffXch + 2 * 2 * 128 * 4;        // [2 streams][2 groups][128] sums
-    static constexpr uint32_t kOffMisc = kOffLx + 2 * 2 * 128 * 4;
+    static constexpr uint32_t kOffMx = kOffLx + 2 * 2 * 128 * 4;         // [2 streams][128] reference maxima
+    static constexpr uint32_t kOffMisc = kOffMx + 2 * 128 * 4;
     // at least 116 KB so that only one CTA (and one 512-column TMEM allocation) fits per SM
     static constexpr uint32_t kSmemNeed = kOffMisc + 16 + 1024;
     static constexpr uint32_t kSmemBytes = kSmemNeed > 118784 ? kSmemNeed : 118784;
@@ -71,9 +73,9 @@ struct K3vTc {
 
 struct K3vTcParams {
     const uint32_t* mask_bits;  // [B, n / 32] key-validity bits, or null for no mask
-    float* part_o;         // [BH, 2 splits, m, d]  (partial 2 s + t: stream t of split s)
-    float* part_m;         // [BH, 2 splits, m]  running max (natural-log units)
-    float* part_l;         // [BH, 2 splits, m]  running sum
+    float* part_o;         // [BH, splits, m, d]
+    float* part_m;         // [BH, splits, m]  running max (natural-log units)
+    float* part_l;         // [BH, splits, m]  running sum
     int H, n, m, halves, splits, chunks_per_split, total_items;
 };
 
@@ -259,13 +261,17 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         constexpr int kT = C::kTeamThreads;
         const int bar_id = 1 + t;                   // this stream's named barrier
         float* xch = reinterpret_cast<float*>(sm + C::kOffXch) + t * 256;   // [2 groups][128]
-        float* lx = reinterpret_cast<float*>(sm + C::kOffLx) + t * 256;     // [2 groups][128]
+        float* lx_all = reinterpret_cast<float*>(sm + C::kOffLx);   // [2 streams][2 groups][128]
+        float* mx_all = reinterpret_cast<float*>(sm + C::kOffMx);   // [2 streams][128]
+        constexpr int kCta = 2 * C::kTeamThreads;   // both streams: named barrier 3
         const uint32_t sbuf = tmem + lane_base + C::kColS + t * 128 + 64 * grp;
         const uint32_t pbuf = tmem + lane_base + C::kColP + t * 64 + 32 * grp;
         const uint32_t obuf = tmem + lane_base + C::kColO + t * D + 32 * grp;
         int u = 0, it = 0;   // chunks this stream has taken, items
         for (int item = blockIdx.x; item < prm.total_items; item += gridDim.x, ++it) {
-            if (group_any(*abort_flag != 0, bar_id, kT)) break;
+            // both streams take every item-level decision together (barrier 3), so that neither
+            // waits at that barrier for a stream that has left
+            if (group_any(*abort_flag != 0, 3, kCta)) break;
             const int bh = item / per_bh, half = (item / prm.splits) % prm.halves;
             const int split = item % prm.splits;
             const int b_idx = bh / prm.H;
@@ -407,44 +413,60 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 l_run = fmaf(l_run, alpha, sum);
                 m_ref = m_new;
             }
-            // the stream's partial of this split: its O is complete once its last P V has been
-            // accumulated; group g streams out columns 32 g .. 32 g + 31, group 0 adds the sums.
-            // A stream that took no chunk of the item writes an empty partial (O = 0, max -inf).
-            const int row = half * C::kRows + r;
-            const size_t prow = ((size_t)bh * 2 * prm.splits + 2 * split + t) * prm.m + row;
-            if (ok && grp < D / 32) {
-                if (mine > 0) {
-                    ok = warp_all(mbar_wait(&pv_done[t], (u - 1) & 1));
-                    if (ok) tc_fence_after();
-                }
-                float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D + grp * 32);
+            // the split's partial: each stream publishes its row statistics and waits for its last
+            // P V; then the threads of stream 0 merge the two streams' O (group g: columns
+            // 32 g .. 32 g + 31) and group 0 of stream 0 writes the merged maximum and sum. A
+            // stream that took no chunk of the item contributes nothing (its TMEM is not read).
+            lx_all[(t * 2 + grp) * 128 + r] = l_run;
+            if (grp == 0) mx_all[t * 128 + r] = m_ref;
+            if (ok && mine > 0) ok = warp_all(mbar_wait(&pv_done[t], (u - 1) & 1));
+            if (group_any(!ok, 3, kCta)) { *abort_flag = 1; break; }   // also publishes lx, mx
+            tc_fence_after();
+            if (t == 0) {
+                const int row = half * C::kRows + r;
+                const size_t prow = ((size_t)bh * prm.splits + split) * prm.m + row;
+                const bool has1 = nch > 1;                       // stream 1 took chunk 1, 3, ...
+                const float m0 = mx_all[r], m1 = has1 ? mx_all[128 + r] : -INFINITY;
+                const float mm = fmaxf(m0, m1);
+                const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - mm);
+                const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - mm);
+                if (grp < D / 32) {
+                    float4* dst = reinterpret_cast<float4*>(prm.part_o + prow * D + grp * 32);
 #pragma unroll 1
-                for (int h = 0; h < 2 && ok; ++h) {   // 16 columns per TMEM load
-                    uint32_t o[16];
-                    if (mine > 0) {
-                        tmem_ld16(obuf + 16 * h, o);
+                    for (int h = 0; h < 2; ++h) {   // 16 columns per TMEM load
+                        uint32_t o0[16], o1[16];
+                        tmem_ld16(obuf + 16 * h, o0);   // stream 0 always has chunk 0
+                        if (has1) {
+                            tmem_ld16(obuf + D + 16 * h, o1);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) o1[e] = 0u;   // a1 = 0 as well
+                        }
                         tmem_ld_wait();
-                    } else {
+                        if (row < prm.m) {
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) o[e] = 0u;
-                    }
-                    if (row < prm.m) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            dst[4 * h + e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                                                         __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+                            for (int e = 0; e < 4; ++e)
+                                dst[4 * h + e] = make_float4(
+                                    a0 * __uint_as_float(o0[4 * e]) + a1 * __uint_as_float(o1[4 * e]),
+                                    a0 * __uint_as_float(o0[4 * e + 1]) + a1 * __uint_as_float(o1[4 * e + 1]),
+                                    a0 * __uint_as_float(o0[4 * e + 2]) + a1 * __uint_as_float(o1[4 * e + 2]),
+                                    a0 * __uint_as_float(o0[4 * e + 3]) + a1 * __uint_as_float(o1[4 * e + 3]));
+                        }
                     }
                 }
+                if (grp == 0 && row < prm.m) {
+                    const float l0 = lx_all[r] + lx_all[128 + r];
+                    const float l1 = has1 ? lx_all[256 + r] + lx_all[384 + r] : 0.f;
+                    prm.part_m[prow] = mm == -INFINITY ? -INFINITY : mm * kLn2;
+                    prm.part_l[prow] = a0 * l0 + a1 * l1;
+                }
+                // both O accumulators have been read: the next item's first P V of either stream
+                // may overwrite them
+                tc_fence_before();
+                mbar_arrive(&o_free[0]);
+                mbar_arrive(&o_free[1]);
             }
-            tc_fence_before();
-            mbar_arrive(&o_free[t]);
-            lx[grp * 128 + r] = l_run;
-            if (group_any(!ok, bar_id, kT)) { *abort_flag = 1; break; }   // also publishes lx
-            if (grp == 0 && row < prm.m) {
-                prm.part_m[prow] = m_ref == -INFINITY ? -INFINITY : m_ref * kLn2;
-                prm.part_l[prow] = lx[r] + lx[128 + r];
-            }
-            named_barrier(bar_id, kT);   // lx is read before the next item overwrites it
+            named_barrier(3, kCta);   // the statistics are read before the next item overwrites them
         }
     }
 
