@@ -157,8 +157,9 @@ struct PinvPair {
     // [2][128] row max / sum halves, [256] own column sums, [256] the peer's, [8] warp maxima,
     // [2] own and peer max row sum
     static constexpr uint32_t kOffBar = kOffRed + (2 * 128 + 2 * 128 + 256 + 256 + 8 + 8) * 4;
-    // barriers: bfull[8], bfree[8], mma_done, mma4_done, e_ready, wl_ready, drain, pro_full, cs_ready
-    static constexpr uint32_t kOffMisc = kOffBar + 24 * 8;
+    // barriers: bfull[8], bfree[8], mma_done, mma4_done, e_ready, wl_ready, drain, pro_full, cs_ready,
+    // e_step[2]
+    static constexpr uint32_t kOffMisc = kOffBar + 26 * 8;
     static constexpr uint32_t kSmemNeed = kOffMisc + 64 + 1024;
     // more than half of the SM's shared memory: no other CTA (and no other TMEM user) shares the SM
     static constexpr uint32_t kSmemBytes = kSmemNeed < 200 * 1024 ? 200 * 1024 : kSmemNeed;
@@ -191,6 +192,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     uint64_t* drain = wl_ready + 1;
     uint64_t* pro_full = drain + 1;      // Q_l / K_l tiles landed (each CTA)
     uint64_t* cs_ready = pro_full + 1;   // the peer's column sums are in cs_peer (each CTA)
+    uint64_t* e_step = cs_ready + 1;     // [2] CTA 0: epilogue steps 2 h, 2 h + 1 of P2 / P3 done in both CTAs
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -213,6 +215,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         mbar_init(drain, 32);     // one commit per lane of the MMA warp
         mbar_init(pro_full, 1);
         mbar_init(cs_ready, 8);    // one arrival per epilogue warp of the peer
+        for (int j = 0; j < 2; ++j) mbar_init(&e_step[j], 16);   // one arrival per epilogue warp
         fence_mbar_init();
     }
     if (warp == 9) {
@@ -294,18 +297,29 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 }
                 if (elect_one()) commit2(mma_done, 3);
             }
+            uint32_t ns = 0;   // e_step phases waited
             for (int it = 0; it < n_iter && ok; ++it) {
                 for (int p = 0; p < 4 && ok; ++p) {
                     const uint32_t a_col = (p == 0 || p == 2) ? R0 : R1;
                     const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
                     const bool streamed = p == 3 || (p == 0 && it > 0);
-                    if (p != 0 || it == 0) {
+                    // P3 and P4 start on the first half of their left factor while the epilogue of
+                    // the previous product still writes the rest (its steps 0, 1 write atoms 0, 1,
+                    // 4, 5 in both CTAs, steps 2, 3 the others); the other products wait for all
+                    const bool stepped = p >= 2;
+                    if (!stepped && (p != 0 || it == 0)) {
                         ok = warp_all(wait_acq_cluster(e_ready, ne & 1u));   // left factor (and X, or k2) in place
                         ++ne;
                         if (!ok) break;
                     }
                     tc_fence_after();
-                    for (int kc = 0; kc < 8; ++kc) {
+                    for (int i = 0; i < 8; ++i) {
+                        const int kc = (i & 1) ? 4 + (i >> 1) : (i >> 1);   // atoms 0, 4, 1, 5, ...
+                        if (stepped && (i & 3) == 0) {
+                            ok = warp_all(wait_acq_cluster(&e_step[i >> 2], ns & 1u));
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
                         if (streamed) {
                             ok = warp_all(mbar_wait(&bfull[kc], nf & 1u));
                             if (!ok) break;
@@ -316,10 +330,11 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                             for (int kk = 0; kk < 4; ++kk)
                                 mma2_ts(d_col, a_col + kc * 32 + kk * 8,
                                         smem_desc(bs + kc * C::kAtomBytes + kk * 32, 16, 1024, kLayoutSw128),
-                                        C::kIdesc, (kc | kk) != 0 ? 1u : 0u);
+                                        C::kIdesc, (i | kk) != 0 ? 1u : 0u);
                             if (p >= 2) commit2(&bfree[kc], 3);   // the producer refills this atom next
                         }
                     }
+                    if (stepped) ++ns;
                     if (streamed) ++nf;
                     if (ok && elect_one()) commit2(p == 3 ? mma4_done : mma_done, 3);
                 }
@@ -350,6 +365,13 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             tc_fence_before();
             __syncwarp();
             if (lane == 0) arrive_cluster(e_ready0);
+        };
+        const uint32_t e_step0 = mapa(smem_u32(e_step), 0);
+        auto arrive_step = [&](int half) {   // steps 2 half, 2 half + 1 of T written (this warp's part)
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) arrive_cluster(e_step0 + 8u * (uint32_t)half);
         };
         auto arrive_wl = [&]() {
             fence_proxy_async_global();   // read next by TMA
@@ -573,12 +595,13 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(tf32_rna(e[i]));
                     tmem_st32(d_col + lane_base + 32 * a, v);
+                    if ((p == 1 || p == 2) && (jj & 1)) arrive_step(jj >> 1);   // P3 / P4 may start on these atoms
                 }
                 if (p == 3) {
                     if (!last_it) arrive_wl();
-                } else {
+                } else if (p == 0) {
                     tmem_st_wait();
-                    if (p == 0) fence_proxy_async_cluster();   // X lines (here and in the peer) feed the MMA
+                    fence_proxy_async_cluster();   // X lines (here and in the peer) feed the MMA
                     arrive_e();
                 }
             }
