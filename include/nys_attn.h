@@ -186,6 +186,15 @@ int nys_attn_selftest_exp2(float* max_rel_err);
  */
 int nys_attn_profile_enable(int on);
 int nys_attn_profile_read(int kernel_id, int* launches, double* total_ms);
+/*
+ * nys_attn_profile_mask -- restricts the timing to the kernels whose bit
+ * (1 << kernel_id) is set in `mask` (all of them by default). Each timed
+ * launch adds two event records to its stream, which delay the next launch,
+ * so a benchmark that times the whole forward brackets only the kernel it
+ * reports. Takes effect for launches after the call; the counters are not
+ * cleared. Returns NYS_OK.
+ */
+int nys_attn_profile_mask(unsigned int mask);
 int nys_attn_kernel_count(void);
 const char* nys_attn_kernel_name(int kernel_id);
 

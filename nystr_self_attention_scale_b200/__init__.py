@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
     lib.nys_attn_profile_enable.argtypes = [i]
     lib.nys_attn_profile_enable.restype = i
     lib.nys_attn_profile_read.argtypes = [i, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_double)]
+    lib.nys_attn_profile_mask.argtypes = [ctypes.c_uint]
+    lib.nys_attn_profile_mask.restype = i
     lib.nys_attn_profile_read.restype = i
     lib.nys_attn_kernel_count.restype = i
     lib.nys_attn_kernel_name.argtypes = [i]
@@ -201,6 +203,19 @@ def version() -> int:
 def profile_enable(on: bool = True) -> None:
     """Start (or stop) per-kernel CUDA-event timing; clears the counters."""
     lib.nys_attn_profile_enable(1 if on else 0)
+
+
+def profile_mask(kernels=None) -> None:
+    """Time only the named kernels (an iterable of names from profile_read()), or all of
+    them when `kernels` is None."""
+    if kernels is None:
+        mask = 0xFFFFFFFF
+    else:
+        names = [lib.nys_attn_kernel_name(k).decode() for k in range(lib.nys_attn_kernel_count())]
+        mask = 0
+        for name in kernels:
+            mask |= 1 << names.index(name)
+    _check(lib.nys_attn_profile_mask(mask), "profile_mask")
 
 
 def profile_read() -> dict:

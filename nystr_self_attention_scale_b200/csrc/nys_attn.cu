@@ -145,6 +145,7 @@ const char* const kKernelNames[K_COUNT] = {"landmarks", "pinv", "k3v_partial", "
 struct ProfRecord { int kid; cudaEvent_t a, b; };
 std::mutex g_prof_mu;
 bool g_prof_on = false;
+unsigned int g_prof_mask = ~0u;   // kernels whose launches are timed
 std::vector<ProfRecord> g_prof;
 int g_prof_launches[K_COUNT];
 double g_prof_ms[K_COUNT];
@@ -154,7 +155,7 @@ struct ProfScope {
     cudaStream_t s;
     cudaEvent_t a = nullptr, b = nullptr;
     ProfScope(int kid_, cudaStream_t s_) : kid(kid_), s(s_) {
-        if (!g_prof_on) return;
+        if (!g_prof_on || !((g_prof_mask >> kid) & 1u)) return;
         cudaEventCreate(&a);
         cudaEventCreate(&b);
         cudaEventRecord(a, s);
@@ -484,32 +485,37 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
         ProfScope ps(K_LANDMARKS, s);
         landmarks_kernel<bf><<<grid, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, D, m);
     }
+    // kernel_3 V (+ mask bits, + combine) runs on the auxiliary stream, concurrently with the
+    // inverse on the caller's stream: the inverse is the longer branch at the supported sizes,
+    // and a kernel that follows its predecessor on the same stream starts sooner than one
+    // released by a cross-stream event
     if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
     if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
-    switch (m) {
-        case 64: rc = launch_pinv_tc<64>(p, st, ql, kl, z, ws, st.aux); break;
-        case 128: rc = launch_pinv_tc<128>(p, st, ql, kl, z, ws, st.aux); break;
-        case 256: rc = launch_pinv_pair(p, st, ql, kl, z, ws, st.aux); break;
-        default: return NYS_ERR_UNSUPPORTED;
-    }
-    if (rc != NYS_OK) return rc;
-    if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
     if (mask) {
         const int words = p.B * (n / 32);
-        ProfScope ps(K_MASKBITS, s);
-        mask_bits_kernel<<<(words + 255) / 256, 256, 0, s>>>(mask, mbits, p.B, n);
+        ProfScope ps(K_MASKBITS, st.aux);
+        mask_bits_kernel<<<(words + 255) / 256, 256, 0, st.aux>>>(mask, mbits, p.B, n);
     }
     // the inverse runs concurrently on its own SMs (one CTA per SM, one per 128 landmark
     // rows of each head); the persistent kernel_3 V grid takes the rest
     const int pinv_ctas = BH * ((m + 127) / 128);
     const int k3v_sms = std::max(st.sm_count / 4, st.sm_count - pinv_ctas);
-    rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, k3v_sms, s);
+    rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, k3v_sms, st.aux);
     if (rc != NYS_OK) return rc;
     {
         const long long threads = (long long)BH * m * (D / 4);
-        ProfScope ps(K_COMBINE, s);
-        k3v_combine_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, s>>>(po, pm, pl, k3v, BH, m, D, p.splits);
+        ProfScope ps(K_COMBINE, st.aux);
+        k3v_combine_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st.aux>>>(po, pm, pl, k3v, BH, m, D,
+                                                                                   p.splits);
     }
+    if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
+    switch (m) {
+        case 64: rc = launch_pinv_tc<64>(p, st, ql, kl, z, ws, s); break;
+        case 128: rc = launch_pinv_tc<128>(p, st, ql, kl, z, ws, s); break;
+        case 256: rc = launch_pinv_pair(p, st, ql, kl, z, ws, s); break;
+        default: return NYS_ERR_UNSUPPORTED;
+    }
+    if (rc != NYS_OK) return rc;
     if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;
     {
         ProfScope ps(K_W, s);
@@ -744,6 +750,12 @@ int nys_attn_profile_enable(int on) {
         nys::g_prof_ms[i] = 0.0;
         nys::g_prof_launches[i] = 0;
     }
+    return NYS_OK;
+}
+
+int nys_attn_profile_mask(unsigned int mask) {
+    std::lock_guard<std::mutex> lock(nys::g_prof_mu);
+    nys::g_prof_mask = mask;
     return NYS_OK;
 }
 

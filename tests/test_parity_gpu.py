@@ -284,3 +284,29 @@ def test_exp2_polynomial_against_cuda_exp2f(nys):
     fitted bound (7.5e-5 relative, degree-3 minimax) of CUDA's exp2f on [-125, 8]."""
     err = nys.selftest_exp2()
     assert 0.0 <= err <= 1.0e-4, err
+
+
+# ------------------------------------------------------------------ kernel timing selection
+
+def test_profile_mask_times_only_selected_kernels(nys):
+    """nys_attn_profile_mask: with one kernel selected, only its launches are timed; with the
+    mask cleared again every kernel of the forward is."""
+    x = make_inputs(WORKLOADS["sweep_n1024_conv"], B=1, H=2)
+    try:
+        nys.profile_mask(["pinv"])
+        nys.profile_enable(True)
+        gpu_forward(x, nys, torch)
+        gpu_forward(x, nys, torch)
+        got = nys.profile_read()
+        nys.profile_enable(False)
+        assert got["pinv"][0] == 2 and got["pinv"][1] > 0.0
+        assert all(n == 0 for name, (n, _) in got.items() if name != "pinv"), got
+        nys.profile_mask(None)
+        nys.profile_enable(True)
+        gpu_forward(x, nys, torch)
+        got = nys.profile_read()
+        for name in ("landmarks", "pinv", "k3v_partial", "k3v_combine", "w_product", "output"):
+            assert got[name][0] == 1, (name, got)
+    finally:
+        nys.profile_enable(False)
+        nys.profile_mask(None)
