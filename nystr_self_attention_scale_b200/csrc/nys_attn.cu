@@ -31,8 +31,9 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
     bool ready = false;
     int sm_count = 0;
-    cudaStream_t aux = nullptr;       // forked stream for the iterative inverse
+    cudaStream_t aux = nullptr;       // forked stream for kernel_3 V (bf16) or the inverse (float32)
     cudaEvent_t fork = nullptr, join = nullptr;
+    cudaEvent_t started = nullptr;    // every CTA of the CTA-pair inverse has begun
     std::mutex launch_mu;             // serialises the fork/join event use of one device
 };
 
@@ -50,6 +51,7 @@ int device_state(DeviceState** out) {
         if (cudaStreamCreateWithFlags(&st.aux, cudaStreamNonBlocking) != cudaSuccess) return NYS_ERR_CUDA;
         if (cudaEventCreateWithFlags(&st.fork, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
         if (cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&st.started, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
         // Keep freed async allocations in the pool so per-call workspace is cheap.
         cudaMemPool_t pool;
         if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
@@ -448,13 +450,18 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
     cfg.blockDim = dim3(C::kThreads);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // `started` fires once every CTA pair has begun: kernel_3 V is held back until then, so
+    // that its persistent grid takes the SMs the pairs leave instead of splitting SM pairs
+    attr[1].id = cudaLaunchAttributeLaunchCompletionEvent;
+    attr[1].val.launchCompletionEvent.event = st.started;
+    attr[1].val.launchCompletionEvent.flags = 0;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     ProfScope ps(K_PINV, s);
     if (cudaLaunchKernelEx(&cfg, pinv_pair_kernel, maps, prm) != cudaSuccess) return NYS_ERR_CUDA;
     return NYS_OK;
@@ -488,9 +495,20 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     // kernel_3 V (+ mask bits, + combine) runs on the auxiliary stream, concurrently with the
     // inverse on the caller's stream: the inverse is the longer branch at the supported sizes,
     // and a kernel that follows its predecessor on the same stream starts sooner than one
-    // released by a cross-stream event
-    if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
-    if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
+    // released by a cross-stream event. At m = 256 the auxiliary stream waits until every
+    // CTA pair of the inverse has started (see launch_pinv_pair); otherwise until the
+    // landmarks are done.
+    if (m == 256) {
+        rc = launch_pinv_pair(p, st, ql, kl, z, ws, s);
+        if (rc != NYS_OK) return rc;
+        if (cudaStreamWaitEvent(st.aux, st.started, 0) != cudaSuccess) return NYS_ERR_CUDA;
+    } else {
+        if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
+        rc = m == 64 ? launch_pinv_tc<64>(p, st, ql, kl, z, ws, s)
+           : m == 128 ? launch_pinv_tc<128>(p, st, ql, kl, z, ws, s) : NYS_ERR_UNSUPPORTED;
+        if (rc != NYS_OK) return rc;
+    }
     if (mask) {
         const int words = p.B * (n / 32);
         ProfScope ps(K_MASKBITS, st.aux);
@@ -509,13 +527,6 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
                                                                                    p.splits);
     }
     if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
-    switch (m) {
-        case 64: rc = launch_pinv_tc<64>(p, st, ql, kl, z, ws, s); break;
-        case 128: rc = launch_pinv_tc<128>(p, st, ql, kl, z, ws, s); break;
-        case 256: rc = launch_pinv_pair(p, st, ql, kl, z, ws, s); break;
-        default: return NYS_ERR_UNSUPPORTED;
-    }
-    if (rc != NYS_OK) return rc;
     if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;
     {
         ProfScope ps(K_W, s);
