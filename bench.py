@@ -63,10 +63,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def source_digest():
+# the sources a kernel's launches depend on (its own header, the shared helpers, the launch code)
+KERNEL_SOURCES = {
+    "landmarks": ["landmarks.cuh"],
+    "pinv": ["tc_pinv_pair.cuh", "tc_pinv.cuh", "sm100.cuh"],
+    "k3v_partial": ["tc_k3v.cuh", "sm100.cuh"],
+    "k3v_combine": ["simt.cuh"],
+    "w_product": ["simt.cuh"],
+    "output": ["tc_output.cuh", "sm100.cuh"],
+}
+
+
+def source_digest(kernel=None):
+    """Digest of the CUDA sources of `kernel` (every source file when None): a traffic figure
+    captured with ncu is only reported while the sources it was captured from are unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nystr_self_attention_scale_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = sorted(os.listdir(csrc)) if kernel not in KERNEL_SOURCES else \
+        sorted(KERNEL_SOURCES[kernel] + ["common.cuh", "nys_attn.cu"])
+    for name in names:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -448,7 +463,7 @@ def main():
         with open(tf) as f:
             tr = json.load(f)
         ent = tr.get(dom)
-        if ent and ent.get("source_digest") == source_digest() and ent.get("workload") == w.name:
+        if ent and ent.get("source_digest") == source_digest(dom) and ent.get("workload") == w.name:
             traffic = ent.get("bytes_per_launch")
     simt = set(SIMT_KERNELS)
     if w.dtype == "f32":  # the float32 path runs every stage on CUDA cores
