@@ -91,9 +91,14 @@ int nys_attn_forward(const void* q, const void* k, const void* v, const uint8_t*
  * nys_attn_forward_host -- the same operation on HOST buffers (same shapes,
  * layouts and checks). Copies the inputs to the device, runs the forward on
  * `stream`, copies the result back into `out` and synchronises `stream`
- * before returning. Host buffers should be pinned (cudaHostAlloc) for full
- * copy bandwidth; pageable memory works but is slower. Device buffers are
- * taken with cudaMallocAsync and released before return.
+ * before returning. The batch is processed in up to 8 chunks of (batch, head)
+ * slices, contiguous in every tensor, so that the copy of one chunk's inputs
+ * and of another's output overlap the forward of a third (two library-owned
+ * copy streams); the result is bitwise the same as one forward over the whole
+ * batch. One call per device at a time (calls from several host threads are
+ * serialised). Host buffers should be pinned (cudaHostAlloc) for full copy
+ * bandwidth and overlap; pageable memory works but is slower. Device buffers
+ * are taken with cudaMallocAsync and released before return.
  */
 int nys_attn_forward_host(const void* q, const void* k, const void* v, const uint8_t* key_mask,
                           const float* conv_w, int B, int H, int n, int d, int m, int n_iter,

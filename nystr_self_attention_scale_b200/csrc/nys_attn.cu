@@ -27,6 +27,7 @@ namespace nys {
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kHostChunks = 8;   // pipeline depth of the host entry (copies overlap compute)
 
 struct DeviceState {
     bool ready = false;
@@ -35,6 +36,10 @@ struct DeviceState {
     cudaEvent_t fork = nullptr, join = nullptr;
     cudaEvent_t started = nullptr;    // every CTA of the CTA-pair inverse has begun
     std::mutex launch_mu;             // serialises the fork/join event use of one device
+    // host entry: copy streams and the events of its chunk pipeline
+    cudaStream_t copy_in = nullptr, copy_out = nullptr;
+    cudaEvent_t alloc_ev = nullptr, in_ev[kHostChunks] = {}, done_ev[kHostChunks] = {}, out_ev = nullptr;
+    std::mutex host_mu;               // one host-entry call per device at a time
 };
 
 std::mutex g_mu;
@@ -52,6 +57,14 @@ int device_state(DeviceState** out) {
         if (cudaEventCreateWithFlags(&st.fork, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
         if (cudaEventCreateWithFlags(&st.join, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
         if (cudaEventCreateWithFlags(&st.started, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaStreamCreateWithFlags(&st.copy_in, cudaStreamNonBlocking) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaStreamCreateWithFlags(&st.copy_out, cudaStreamNonBlocking) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&st.alloc_ev, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&st.out_ev, cudaEventDisableTiming) != cudaSuccess) return NYS_ERR_CUDA;
+        for (int c = 0; c < kHostChunks; ++c)
+            if (cudaEventCreateWithFlags(&st.in_ev[c], cudaEventDisableTiming) != cudaSuccess ||
+                cudaEventCreateWithFlags(&st.done_ev[c], cudaEventDisableTiming) != cudaSuccess)
+                return NYS_ERR_CUDA;
         // Keep freed async allocations in the pool so per-call workspace is cheap.
         cudaMemPool_t pool;
         if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
@@ -638,9 +651,14 @@ int nys_attn_forward_host(const void* q, const void* k, const void* v, const uin
                           int dtype, void* out, void* stream) {
     int rc = nys::validate(q, k, v, out, B, H, n, d, m, n_iter, dtype);
     if (rc != NYS_OK) return rc;
+    nys::DeviceState* st = nullptr;
+    rc = nys::device_state(&st);
+    if (rc != NYS_OK) return rc;
+    std::lock_guard<std::mutex> host_lock(st->host_mu);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t elt = dtype == NYS_F32 ? 4 : 2;
-    const size_t tensor = (size_t)B * H * n * d * elt;
+    const size_t head = (size_t)n * d * elt;            // bytes of one (batch, head) slice
+    const size_t tensor = (size_t)B * H * head;
     const size_t mask_bytes = key_mask ? (size_t)B * n : 0;
     const size_t w_bytes = conv_w ? (size_t)H * NYS_CONV_TAPS * sizeof(float) : 0;
     const size_t o_q = 0, o_k = nys::align_up(tensor), o_v = 2 * o_k, o_o = 3 * o_k;
@@ -652,18 +670,65 @@ int nys_attn_forward_host(const void* q, const void* k, const void* v, const uin
         return NYS_ERR_NOMEM;
     }
     char* b = static_cast<char*>(buf);
-    bool ok = cudaMemcpyAsync(b + o_q, q, tensor, cudaMemcpyHostToDevice, s) == cudaSuccess &&
-              cudaMemcpyAsync(b + o_k, k, tensor, cudaMemcpyHostToDevice, s) == cudaSuccess &&
-              cudaMemcpyAsync(b + o_v, v, tensor, cudaMemcpyHostToDevice, s) == cudaSuccess;
-    if (ok && key_mask) ok = cudaMemcpyAsync(b + o_mask, key_mask, mask_bytes, cudaMemcpyHostToDevice, s) == cudaSuccess;
-    if (ok && conv_w) ok = cudaMemcpyAsync(b + o_w, conv_w, w_bytes, cudaMemcpyHostToDevice, s) == cudaSuccess;
-    rc = ok ? NYS_OK : NYS_ERR_CUDA;
-    if (rc == NYS_OK)
-        rc = nys_attn_forward(b + o_q, b + o_k, b + o_v, key_mask ? (const uint8_t*)(b + o_mask) : nullptr,
-                              conv_w ? (const float*)(b + o_w) : nullptr, B, H, n, d, m, n_iter, dtype,
-                              b + o_o, stream);
-    if (rc == NYS_OK && cudaMemcpyAsync(out, b + o_o, tensor, cudaMemcpyDeviceToHost, s) != cudaSuccess)
-        rc = NYS_ERR_CUDA;
+    const char* hq = static_cast<const char*>(q);
+    const char* hk = static_cast<const char*>(k);
+    const char* hv = static_cast<const char*>(v);
+    char* ho = static_cast<char*>(out);
+    // Chunks of (batch, head) slices, contiguous in every tensor: whole batch elements when
+    // B >= kHostChunks, otherwise head ranges of one batch element. A head's result does not
+    // depend on the rest of the batch, so chunk c's forward runs while chunk c + 1's inputs
+    // are copied in and chunk c - 1's output is copied out (three streams, two copy engines).
+    struct Chunk { int b0, nb, h0, nh; };
+    Chunk ch[nys::kHostChunks];
+    int nch = 0;
+    if (B >= nys::kHostChunks) {
+        for (int c = 0; c < nys::kHostChunks; ++c) {
+            const int b0 = (int)((long long)B * c / nys::kHostChunks);
+            const int b1 = (int)((long long)B * (c + 1) / nys::kHostChunks);
+            ch[nch++] = {b0, b1 - b0, 0, H};
+        }
+    } else {
+        // head groups per batch element: B * g <= kHostChunks, so every head is covered
+        const int g = std::max(1, std::min(H, nys::kHostChunks / B));
+        for (int bb = 0; bb < B; ++bb)
+            for (int c = 0; c < g; ++c) {
+                const int h0 = H * c / g, h1 = H * (c + 1) / g;
+                ch[nch++] = {bb, 1, h0, h1 - h0};
+            }
+    }
+    bool ok = cudaEventRecord(st->alloc_ev, s) == cudaSuccess &&
+              cudaStreamWaitEvent(st->copy_in, st->alloc_ev, 0) == cudaSuccess;
+    if (ok && conv_w) ok = cudaMemcpyAsync(b + o_w, conv_w, w_bytes, cudaMemcpyHostToDevice, st->copy_in) == cudaSuccess;
+    int issued = 0;
+    for (int c = 0; c < nch && ok && rc == NYS_OK; ++c) {
+        const Chunk& k_ = ch[c];
+        const size_t off = ((size_t)k_.b0 * H + k_.h0) * head;
+        const size_t bytes = (size_t)k_.nb * k_.nh * head;
+        ok = cudaMemcpyAsync(b + o_q + off, hq + off, bytes, cudaMemcpyHostToDevice, st->copy_in) == cudaSuccess &&
+             cudaMemcpyAsync(b + o_k + off, hk + off, bytes, cudaMemcpyHostToDevice, st->copy_in) == cudaSuccess &&
+             cudaMemcpyAsync(b + o_v + off, hv + off, bytes, cudaMemcpyHostToDevice, st->copy_in) == cudaSuccess;
+        if (ok && key_mask && k_.h0 == 0)   // a batch element's mask rows, with its first chunk
+            ok = cudaMemcpyAsync(b + o_mask + (size_t)k_.b0 * n, key_mask + (size_t)k_.b0 * n, (size_t)k_.nb * n,
+                                 cudaMemcpyHostToDevice, st->copy_in) == cudaSuccess;
+        ok = ok && cudaEventRecord(st->in_ev[c], st->copy_in) == cudaSuccess &&
+             cudaStreamWaitEvent(s, st->in_ev[c], 0) == cudaSuccess;
+        if (!ok) break;
+        rc = nys_attn_forward(b + o_q + off, b + o_k + off, b + o_v + off,
+                              key_mask ? (const uint8_t*)(b + o_mask) + (size_t)k_.b0 * n : nullptr,
+                              conv_w ? (const float*)(b + o_w) + (size_t)k_.h0 * NYS_CONV_TAPS : nullptr, k_.nb,
+                              k_.nh, n, d, m, n_iter, dtype, b + o_o + off, s);
+        if (rc != NYS_OK) break;
+        ok = cudaEventRecord(st->done_ev[c], s) == cudaSuccess &&
+             cudaStreamWaitEvent(st->copy_out, st->done_ev[c], 0) == cudaSuccess &&
+             cudaMemcpyAsync(ho + off, b + o_o + off, bytes, cudaMemcpyDeviceToHost, st->copy_out) == cudaSuccess;
+        ++issued;
+    }
+    if (rc == NYS_OK && (!ok || issued != nch)) rc = NYS_ERR_CUDA;
+    // the buffer is released on `stream` after every copy that uses it
+    cudaEventRecord(st->out_ev, st->copy_out);
+    cudaStreamWaitEvent(s, st->out_ev, 0);
+    cudaEventRecord(st->alloc_ev, st->copy_in);
+    cudaStreamWaitEvent(s, st->alloc_ev, 0);
     cudaFreeAsync(buf, s);
     if (cudaStreamSynchronize(s) != cudaSuccess && rc == NYS_OK) rc = NYS_ERR_CUDA;
     return rc;
