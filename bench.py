@@ -33,6 +33,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -63,15 +64,25 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-# the sources a kernel's launches depend on (its own header, the shared helpers, the launch code)
+# the sources a kernel's launches depend on: its own headers and the host functions that plan
+# and configure its launch (text taken from nys_attn.cu)
 KERNEL_SOURCES = {
-    "landmarks": ["landmarks.cuh"],
-    "pinv": ["tc_pinv_pair.cuh", "tc_pinv.cuh", "sm100.cuh"],
-    "k3v_partial": ["tc_k3v.cuh", "sm100.cuh"],
-    "k3v_combine": ["simt.cuh"],
-    "w_product": ["simt.cuh"],
-    "output": ["tc_output.cuh", "sm100.cuh"],
+    "landmarks": (["landmarks.cuh"], ["launch_bf16", "launch_simt"]),
+    "pinv": (["tc_pinv_pair.cuh", "tc_pinv.cuh", "sm100.cuh"], ["launch_pinv_pair", "launch_pinv_tc", "launch_bf16"]),
+    "k3v_partial": (["tc_k3v.cuh", "sm100.cuh"], ["launch_k3v_tc", "launch_bf16"]),
+    "k3v_combine": (["simt.cuh"], ["launch_bf16", "launch_simt"]),
+    "w_product": (["simt.cuh"], ["launch_bf16", "launch_simt"]),
+    "output": (["tc_output.cuh", "sm100.cuh"], ["launch_output_tc", "launch_bf16"]),
 }
+
+
+def _function_text(src, name):
+    """The text of the top-level function `name` (from its signature to its closing brace)."""
+    mt = re.search(r"\n[A-Za-z_][\w:<>]*\s+" + name + r"\(", src)
+    if mt is None:
+        raise KeyError(name)
+    j = src.find("\n}\n", mt.start())
+    return src[mt.start():j + 3]
 
 
 def source_digest(kernel=None):
@@ -79,11 +90,19 @@ def source_digest(kernel=None):
     captured with ncu is only reported while the sources it was captured from are unchanged."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "nystr_self_attention_scale_b200", "csrc")
-    names = sorted(os.listdir(csrc)) if kernel not in KERNEL_SOURCES else \
-        sorted(KERNEL_SOURCES[kernel] + ["common.cuh", "nys_attn.cu"])
-    for name in names:
+    if kernel not in KERNEL_SOURCES:
+        for name in sorted(os.listdir(csrc)):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+        return h.hexdigest()[:16]
+    headers, funcs = KERNEL_SOURCES[kernel]
+    for name in sorted(headers + ["common.cuh"]):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
+    with open(os.path.join(csrc, "nys_attn.cu")) as f:
+        src = f.read()
+    for fn in funcs + ["make_plan"]:
+        h.update(fn.encode() + _function_text(src, fn).encode())
     return h.hexdigest()[:16]
 
 

@@ -85,3 +85,15 @@ def test_reference_arm_under_torchrun_world2():
     assert line["config"]["workload"] == "tiny_f32"
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_kernel_source_digests_resolve():
+    """Every kernel's traffic-validity digest finds its headers and launch functions, and
+    differs from the digest of another kernel's sources."""
+    digests = {k: bench.source_digest(k) for k in bench.KERNEL_SOURCES}
+    assert all(len(d) == 16 for d in digests.values())
+    assert digests["pinv"] != digests["output"] != digests["k3v_partial"]
+    with open(os.path.join(ROOT, "nystr_self_attention_scale_b200", "csrc", "nys_attn.cu")) as f:
+        src = f.read()
+    text = bench._function_text(src, "launch_pinv_pair")
+    assert text.lstrip().startswith("int launch_pinv_pair(") and text.rstrip().endswith("}")
