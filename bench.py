@@ -65,14 +65,15 @@ def load_peaks():
 
 
 # the sources a kernel's launches depend on: its own headers and the host functions that plan
-# and configure its launch (text taken from nys_attn.cu)
+# and configure its launch (text taken from nys_attn.cu); a kernel launched inline in the
+# forward's orchestration depends on that whole function
 KERNEL_SOURCES = {
     "landmarks": (["landmarks.cuh"], ["launch_bf16", "launch_simt"]),
-    "pinv": (["tc_pinv_pair.cuh", "tc_pinv.cuh", "sm100.cuh"], ["launch_pinv_pair", "launch_pinv_tc", "launch_bf16"]),
-    "k3v_partial": (["tc_k3v.cuh", "sm100.cuh"], ["launch_k3v_tc", "launch_bf16"]),
+    "pinv": (["tc_pinv_pair.cuh", "tc_pinv.cuh", "sm100.cuh"], ["launch_pinv_pair", "launch_pinv_tc"]),
+    "k3v_partial": (["tc_k3v.cuh", "sm100.cuh"], ["launch_k3v_tc"]),
     "k3v_combine": (["simt.cuh"], ["launch_bf16", "launch_simt"]),
     "w_product": (["simt.cuh"], ["launch_bf16", "launch_simt"]),
-    "output": (["tc_output.cuh", "sm100.cuh"], ["launch_output_tc", "launch_bf16"]),
+    "output": (["tc_output.cuh", "sm100.cuh"], ["launch_output_tc"]),
 }
 
 
