@@ -1,0 +1,67 @@
+"""The benchmark's work model and roofline arithmetic, against closed forms.
+
+The step's ideal bytes (Q, K, V read and out written once) and its FLOP, split into
+the dense contractions (Q K_l^T, P W, Q_l K^T, P V, Q_l K_l^T, Z k3V), the inverse
+(8 m^3 per iteration) and the 65-tap conv, are checked against the figures derived
+directly from the method's operation counts for the n = 16384 and n = 4096 bf16
+workloads; the per-kernel roofline picks the bound whose ideal time is longer.
+"""
+import pytest
+
+import bench
+from workloads import WORKLOADS
+
+PEAKS = {"hbm_gbs": 6557.8, "bf16_tflops": 1664.0, "sm_max_mhz": 1965.0}
+
+
+def _split(w):
+    BH, n, d, m = w.BH, w.n, w.d, w.m
+    gemm = BH * (4 * 2 * n * m * d + 2 * 2 * m * m * d)
+    pinv = BH * w.n_iter * 8 * m ** 3
+    conv = BH * 2 * 65 * n * d if w.conv else 0
+    return gemm, pinv, conv
+
+
+def _printed(x):
+    """Half a unit of the last printed digit of a figure given to three significant digits."""
+    s = f"{x}"
+    decimals = len(s.split(".")[1]) if "." in s else 0
+    return 0.5 * 10 ** -decimals + 1e-9
+
+
+@pytest.mark.parametrize("name,mbytes,gemm_g,pinv_g,conv_g", [
+    ("n16384_bf16_corr", 268.4, 69.3, 25.8, 4.36),      # B4 H8 n16384 d64 m256, conv on
+    ("longcls_bf16_masked", 67.1, 8.72, 6.44, 1.09),    # B32 H2 n4096 d32 m128, conv on
+])
+def test_step_work_matches_operation_counts(name, mbytes, gemm_g, pinv_g, conv_g):
+    w = WORKLOADS[name]
+    t_roof, nbytes, flops = bench.roofline_bound_time(w, PEAKS)
+    gemm, pinv, conv = _split(w)
+    assert nbytes == 4 * w.BH * w.n * w.d * 2
+    assert nbytes / 1e6 == pytest.approx(mbytes, abs=_printed(mbytes))
+    assert gemm / 1e9 == pytest.approx(gemm_g, abs=_printed(gemm_g))
+    assert pinv / 1e9 == pytest.approx(pinv_g, abs=_printed(pinv_g))
+    assert conv / 1e9 == pytest.approx(conv_g, abs=_printed(conv_g))
+    assert flops == gemm + pinv + conv
+    assert t_roof == max(nbytes / (PEAKS["hbm_gbs"] * 1e9), flops / (PEAKS["bf16_tflops"] * 1e12))
+
+
+def test_headline_step_is_compute_bound_at_about_60_us():
+    t_roof, _, _ = bench.roofline_bound_time(WORKLOADS["n16384_bf16_corr"], PEAKS)
+    assert t_roof * 1e6 == pytest.approx(59.73, abs=0.05)
+
+
+def test_kernel_rooflines_pick_the_longer_bound():
+    w = WORKLOADS["n16384_bf16_corr"]
+    # the inverse: tf32 on the tensor core, FLOP-bound (25.8 GFLOP against 12.6 MB)
+    r = bench.roofline_for(w, "pinv", 0.130, PEAKS, bench.SIMT_KERNELS, None)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["algorithmic_flops"] == w.BH * w.n_iter * 8 * w.m ** 3
+    assert r["peak"] == pytest.approx(1664.0 * 1.1 / 2.25, abs=0.1)
+    assert r["achieved"] == pytest.approx(r["algorithmic_flops"] / 0.130e-3 / 1e12, rel=1e-3)
+    assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], rel=1e-3)
+    # the landmark means: pure traffic, HBM-bound
+    r = bench.roofline_for(w, "landmarks", 0.030, PEAKS, bench.SIMT_KERNELS, 139063040)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 139063040
+    assert r["algorithmic_bytes"] == 2 * w.BH * w.n * w.d * 2 + 2 * w.BH * w.m * w.d * 4
+    assert r["achieved"] == pytest.approx(r["algorithmic_bytes"] / 0.030e-3 / 1e9, rel=1e-3)
