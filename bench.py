@@ -185,6 +185,21 @@ def roofline_bound_time(w, peaks):
     return max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peak * 1e12)), nbytes, flops
 
 
+def roofline_bound_time_pipes(w, peaks):
+    """The same bound with every FLOP charged at the rate of the pipe that executes it: on the
+    bf16 path the inverse's iteration runs in tf32 on the tensor core (kernel_2's three-term
+    split product included), the contractions and the Toeplitz conv in bf16; fp32 runs all of
+    it on the CUDA cores (then equal to roofline_bound_time)."""
+    if w.dtype != "bf16":
+        return roofline_bound_time(w, peaks)[0]
+    m, n, d = w.m, w.n, w.d
+    nbytes = 4 * w.BH * n * d * 2
+    bf16 = w.BH * (4 * 2 * n * m * d + 2 * m * m * d + (2 * 65 * n * d if w.conv else 0))
+    tf32 = w.BH * (w.n_iter * 8 * m ** 3 + 3 * 2 * m * m * d)
+    t_flops = bf16 / (peaks["bf16_tflops"] * 1e12) + tf32 / (compute_peak_tflops("tensor_tf32", peaks, False) * 1e12)
+    return max(nbytes / (peaks["hbm_gbs"] * 1e9), t_flops)
+
+
 # ---------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -491,6 +506,7 @@ def main():
     roof = roofline_for(w, dom, prof[dom][1] / max(1, prof[dom][0]), peaks, simt, traffic)
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
     t_roof, ideal_bytes, total_flops = roofline_bound_time(w, peaks)
+    t_pipes = roofline_bound_time_pipes(w, peaks)
 
     e2e = None
     if not args.no_e2e:
@@ -538,6 +554,9 @@ def main():
             "roofline": roof,
             "step_roofline": {"t_roof_us": round(t_roof * 1e6, 2), "frac": round(t_roof / (ms_per_step * 1e-3), 4),
                               "ideal_bytes": ideal_bytes, "flops": total_flops},
+            "step_roofline_pipes": {"t_roof_us": round(t_pipes * 1e6, 2),
+                                    "frac": round(t_pipes / (ms_per_step * 1e-3), 4),
+                                    "note": "inverse (and kernel_2) at the tf32 tensor rate, the rest at bf16"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "kernels": kernels,
             "kernels_source": f"separate untimed pass of {breakdown_steps} steps, every launch bracketed by "

@@ -65,3 +65,17 @@ def test_kernel_rooflines_pick_the_longer_bound():
     assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 139063040
     assert r["algorithmic_bytes"] == 2 * w.BH * w.n * w.d * 2 + 2 * w.BH * w.m * w.d * 4
     assert r["achieved"] == pytest.approx(r["algorithmic_bytes"] / 0.030e-3 / 1e9, rel=1e-3)
+
+
+def test_pipe_aware_bound_charges_the_inverse_at_tf32():
+    w = WORKLOADS["n16384_bf16_corr"]
+    t = bench.roofline_bound_time_pipes(w, PEAKS)
+    tf32 = PEAKS["bf16_tflops"] * 1.1 / 2.25
+    m, n, d = w.m, w.n, w.d
+    expect = (w.BH * (8 * n * m * d + 2 * m * m * d + 2 * 65 * n * d) / (PEAKS["bf16_tflops"] * 1e12)
+              + w.BH * (6 * 8 * m ** 3 + 6 * m * m * d) / (tf32 * 1e12))
+    assert t == pytest.approx(expect, rel=1e-12)
+    assert 75e-6 < t < 77e-6                                   # about 76 us: compute-bound
+    assert t > bench.roofline_bound_time(w, PEAKS)[0]          # never below the plain bound here
+    wf = WORKLOADS["default_f32_masked"]                       # fp32: both bounds are the same
+    assert bench.roofline_bound_time_pipes(wf, PEAKS) == bench.roofline_bound_time(wf, PEAKS)[0]
