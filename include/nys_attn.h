@@ -105,6 +105,16 @@ int nys_attn_forward_host(const void* q, const void* k, const void* v, const uin
                           int dtype, void* out, void* stream);
 
 /*
+ * nys_attn_host_plan -- the chunks nys_attn_forward_host runs the batch in (host
+ * only, no GPU work): up to 8 chunks of (batch, head) slices, each contiguous in
+ * every [B, H, n, d] tensor -- whole batch elements when B >= 8, otherwise head
+ * ranges of one batch element -- covering every slice exactly once. Writes
+ * (b0, nb, h0, nh) per chunk into `chunks` (room for max_chunks >= 8 chunks,
+ * 4 ints each) and returns the count, or NYS_ERR_INVALID_ARG.
+ */
+int nys_attn_host_plan(int B, int H, int* chunks, int max_chunks);
+
+/*
  * nys_attn_forward_debug -- nys_attn_forward plus copies of the intermediate
  * stages, for tests. Each stage pointer is a device float32 buffer or NULL:
  *   q_l, k_l [B, H, m, d]   landmarks of the scaled Q and K (walkthrough 2.3)

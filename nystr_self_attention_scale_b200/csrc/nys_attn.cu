@@ -646,6 +646,30 @@ int nys_attn_forward_debug(const void* q, const void* k, const void* v, const ui
                     w, static_cast<cudaStream_t>(stream));
 }
 
+int nys_attn_host_plan(int B, int H, int* chunks, int max_chunks) {
+    // Chunks of (batch, head) slices, contiguous in every [B, H, n, d] tensor: whole batch
+    // elements when B >= kHostChunks, otherwise head ranges of one batch element, B * g <= 8.
+    if (B <= 0 || H <= 0 || !chunks || max_chunks < nys::kHostChunks) return NYS_ERR_INVALID_ARG;
+    int nch = 0;
+    if (B >= nys::kHostChunks) {
+        for (int c = 0; c < nys::kHostChunks; ++c) {
+            const int b0 = (int)((long long)B * c / nys::kHostChunks);
+            const int b1 = (int)((long long)B * (c + 1) / nys::kHostChunks);
+            chunks[4 * nch] = b0; chunks[4 * nch + 1] = b1 - b0; chunks[4 * nch + 2] = 0; chunks[4 * nch + 3] = H;
+            ++nch;
+        }
+    } else {
+        const int g = std::max(1, std::min(H, nys::kHostChunks / B));   // head groups per batch element
+        for (int bb = 0; bb < B; ++bb)
+            for (int c = 0; c < g; ++c) {
+                const int h0 = H * c / g, h1 = H * (c + 1) / g;
+                chunks[4 * nch] = bb; chunks[4 * nch + 1] = 1; chunks[4 * nch + 2] = h0; chunks[4 * nch + 3] = h1 - h0;
+                ++nch;
+            }
+    }
+    return nch;
+}
+
 int nys_attn_forward_host(const void* q, const void* k, const void* v, const uint8_t* key_mask,
                           const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
                           int dtype, void* out, void* stream) {
@@ -678,24 +702,16 @@ int nys_attn_forward_host(const void* q, const void* k, const void* v, const uin
     // B >= kHostChunks, otherwise head ranges of one batch element. A head's result does not
     // depend on the rest of the batch, so chunk c's forward runs while chunk c + 1's inputs
     // are copied in and chunk c - 1's output is copied out (three streams, two copy engines).
+    int plan[4 * nys::kHostChunks];
+    const int nch = nys_attn_host_plan(B, H, plan, nys::kHostChunks);
+    if (nch <= 0) {
+        cudaFreeAsync(buf, s);
+        cudaStreamSynchronize(s);
+        return NYS_ERR_INVALID_ARG;
+    }
     struct Chunk { int b0, nb, h0, nh; };
     Chunk ch[nys::kHostChunks];
-    int nch = 0;
-    if (B >= nys::kHostChunks) {
-        for (int c = 0; c < nys::kHostChunks; ++c) {
-            const int b0 = (int)((long long)B * c / nys::kHostChunks);
-            const int b1 = (int)((long long)B * (c + 1) / nys::kHostChunks);
-            ch[nch++] = {b0, b1 - b0, 0, H};
-        }
-    } else {
-        // head groups per batch element: B * g <= kHostChunks, so every head is covered
-        const int g = std::max(1, std::min(H, nys::kHostChunks / B));
-        for (int bb = 0; bb < B; ++bb)
-            for (int c = 0; c < g; ++c) {
-                const int h0 = H * c / g, h1 = H * (c + 1) / g;
-                ch[nch++] = {bb, 1, h0, h1 - h0};
-            }
-    }
+    for (int c = 0; c < nch; ++c) ch[c] = {plan[4 * c], plan[4 * c + 1], plan[4 * c + 2], plan[4 * c + 3]};
     bool ok = cudaEventRecord(st->alloc_ev, s) == cudaSuccess &&
               cudaStreamWaitEvent(st->copy_in, st->alloc_ev, 0) == cudaSuccess;
     if (ok && conv_w) ok = cudaMemcpyAsync(b + o_w, conv_w, w_bytes, cudaMemcpyHostToDevice, st->copy_in) == cudaSuccess;

@@ -113,3 +113,25 @@ def test_defaults_match_the_pages():
     hdr = open(os.path.join(ROOT, "include", "nys_attn.h")).read()
     assert f"#define NYS_CONV_TAPS {rows['conv_kernel_size']}" in hdr
     assert f"#define NYS_DEFAULT_N_ITER {rows['iterative_inv_n_iter']}" in hdr
+
+
+def test_host_plan_covers_every_slice_once(lib):
+    """The host entry's chunk plan: at most 8 chunks, each contiguous in a [B, H, n, d]
+    tensor (whole batch elements, or a head range of one), covering every slice once."""
+    import ctypes
+    lib.nys_attn_host_plan.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_int]
+    lib.nys_attn_host_plan.restype = ctypes.c_int
+    buf = (ctypes.c_int * 32)()
+    for B in range(1, 40):
+        for H in range(1, 20):
+            n = lib.nys_attn_host_plan(B, H, buf, 8)
+            assert 1 <= n <= 8, (B, H, n)
+            seen = []
+            for c in range(n):
+                b0, nb, h0, nh = buf[4 * c:4 * c + 4]
+                assert nb >= 1 and nh >= 1 and (nb == 1 or (h0 == 0 and nh == H)), (B, H, c)
+                seen += [(b, h) for b in range(b0, b0 + nb) for h in range(h0, h0 + nh)]
+            assert sorted(seen) == [(b, h) for b in range(B) for h in range(H)], (B, H)
+    assert lib.nys_attn_host_plan(0, 1, buf, 8) == -1
+    assert lib.nys_attn_host_plan(1, 1, buf, 7) == -1
+    assert lib.nys_attn_host_plan(1, 1, None, 8) == -1
