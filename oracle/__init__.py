@@ -48,11 +48,14 @@ def _load():
         lib.nys_oracle_landmarks.argtypes = [fp, i, i, i, dp]
         lib.nys_oracle_softmax_rows.argtypes = [dp, i, i, u8p]
         lib.nys_oracle_iterative_inv.argtypes = [dp, i, i, dp]
+        lib.nys_oracle_iterative_inv_opt.argtypes = [dp, i, i, i, dp]
         lib.nys_oracle_init_coeff.argtypes = [dp, i]
         lib.nys_oracle_init_coeff.restype = ctypes.c_double
+        lib.nys_oracle_init_coeff_exact.argtypes = [dp, i]
+        lib.nys_oracle_init_coeff_exact.restype = ctypes.c_double
         lib.nys_oracle_dwconv_add.argtypes = [fp, fp, i, i, dp]
-        lib.nys_oracle_forward.argtypes = [fp, fp, fp, u8p, fp, i, i, i, i, i, i, ip, i, i,
-                                           dp, dp, dp, dp, dp, dp]
+        lib.nys_oracle_forward.argtypes = [fp, fp, fp, u8p, fp, i, i, i, i, i, i, i, i, ip, i, i,
+                                           dp, dp, dp, dp, dp, dp, dp]
         lib.nys_oracle_forward.restype = ctypes.c_int
         lib.nys_oracle_max_threads.restype = ctypes.c_int
         _lib = lib
@@ -91,17 +94,21 @@ def softmax_rows(s: np.ndarray, keep: Optional[np.ndarray] = None) -> np.ndarray
     return s
 
 
-def iterative_inv(a: np.ndarray, n_iter: int = 6) -> np.ndarray:
+def iterative_inv(a: np.ndarray, n_iter: int = 6, init_option: int = 0) -> np.ndarray:
+    """Iterative inverse of walkthrough 2.5; init_option 0 = default Z_0 scalar,
+    1 = the exact coefficient 1 / ||a||_1 (inv_coeff_init_option = True)."""
     a = np.ascontiguousarray(a, dtype=np.float64)
     m = a.shape[0]
     z = np.empty((m, m), np.float64)
-    _load().nys_oracle_iterative_inv(_ptr(a, ctypes.c_double), m, n_iter, _ptr(z, ctypes.c_double))
+    _load().nys_oracle_iterative_inv_opt(_ptr(a, ctypes.c_double), m, n_iter, int(init_option),
+                                         _ptr(z, ctypes.c_double))
     return z
 
 
-def init_coeff(a: np.ndarray) -> float:
+def init_coeff(a: np.ndarray, init_option: int = 0) -> float:
     a = np.ascontiguousarray(a, dtype=np.float64)
-    return float(_load().nys_oracle_init_coeff(_ptr(a, ctypes.c_double), a.shape[0]))
+    fn = _load().nys_oracle_init_coeff_exact if init_option else _load().nys_oracle_init_coeff
+    return float(fn(_ptr(a, ctypes.c_double), a.shape[0]))
 
 
 def dwconv(v: np.ndarray, w: np.ndarray) -> np.ndarray:
@@ -116,12 +123,16 @@ def dwconv(v: np.ndarray, w: np.ndarray) -> np.ndarray:
 
 
 def forward(q, k, v, mask=None, conv_w=None, m: int = 64, n_iter: int = 6,
-            rows: Optional[Sequence[int]] = None, threads: int = 0, stages: bool = False):
+            rows: Optional[Sequence[int]] = None, threads: int = 0, stages: bool = False,
+            init_option: int = 0, exact: bool = False, probs: bool = False):
     """Oracle forward over [B, H, n, d] float32 inputs; returns float64 output.
 
     ``rows`` selects query rows (same for every head): output [B, H, len(rows), d].
     With ``stages=True`` also returns a dict of per-head Q_l, K_l, kernel_2, Z and
-    kernel_3 V.
+    kernel_3 V (Nystrom path only); with ``probs=True`` the dict also holds "probs",
+    the attention weights of walkthrough 2.7 ([B, H, rows, m] = kernel_1 Z, or
+    [B, H, rows, n] on the exact path). ``init_option`` selects the Z_0 scalar
+    (0 default, 1 exact coefficient); ``exact=True`` takes path A (2.1).
     """
     q, k, v = _f32(q), _f32(k), _f32(v)
     B, H, n, d = q.shape
@@ -129,20 +140,24 @@ def forward(q, k, v, mask=None, conv_w=None, m: int = 64, n_iter: int = 6,
     nr = n if rows_arr is None else len(rows_arr)
     out = np.empty((B, H, nr, d), np.float64)
     st = None
-    if stages:
-        st = dict(ql=np.empty((B, H, m, d)), kl=np.empty((B, H, m, d)),
+    if stages or probs:
+        st = {}
+    if stages and not exact:
+        st.update(ql=np.empty((B, H, m, d)), kl=np.empty((B, H, m, d)),
                   k2=np.empty((B, H, m, m)), z=np.empty((B, H, m, m)),
                   k3v=np.empty((B, H, m, d)))
+    if probs:
+        st["probs"] = np.empty((B, H, nr, n if exact else m))
     mask_arr = None if mask is None else np.ascontiguousarray(mask, dtype=np.uint8)
     w_arr = None if conv_w is None else _f32(conv_w)
     dp = ctypes.c_double
+    g = (lambda key: _ptr(st[key], dp) if st is not None and key in st else None)
     rc = _load().nys_oracle_forward(
         _ptr(q, ctypes.c_float), _ptr(k, ctypes.c_float), _ptr(v, ctypes.c_float),
         _ptr(mask_arr, ctypes.c_uint8), _ptr(w_arr, ctypes.c_float), B, H, n, d, m, n_iter,
+        int(init_option), 1 if exact else 0,
         _ptr(rows_arr, ctypes.c_int), nr, int(threads), _ptr(out, dp),
-        _ptr(st["ql"], dp) if st else None, _ptr(st["kl"], dp) if st else None,
-        _ptr(st["k2"], dp) if st else None, _ptr(st["z"], dp) if st else None,
-        _ptr(st["k3v"], dp) if st else None)
+        g("ql"), g("kl"), g("k2"), g("z"), g("k3v"), g("probs"))
     if rc != 0:
         raise ValueError("oracle rejected the shape")
-    return (out, st) if stages else out
+    return (out, st) if (stages or probs) else out

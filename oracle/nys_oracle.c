@@ -19,13 +19,19 @@
  *        Z <- 1/4 Z (13I - X(15I - X(7I - X))), X = kernel_2 Z
  *   2.6  context += depthwise Conv2d over the sequence axis of V,
  *        kernel (65,1), padding (32,0), groups = heads, no bias
+ *   2.7  output_attentions returns attention_probs = kernel_1 Z [n x m]
+ *   2.1  path A (num_landmarks == segment length): exact softmax attention,
+ *        softmax(Q K^T + mask) V, with the same d^-1/4 scaling and conv
  *
  * Readings where the pages are silent or ambiguous (all listed in the
  * design notes):
  *   - the segment length is the runtime n / m (n divisible by m);
- *   - the Nystrom path is taken for every m, including m == n;
+ *   - the Nystrom path is taken for every m, including m == n, unless the
+ *     caller asks for path A explicitly;
  *   - Z_0 = c * kernel_2^T with c = 1 / (max column sum * max row sum),
- *     both taken per (batch, head);
+ *     both taken per (batch, head); with the exact-coefficient option
+ *     c = 1 / max column sum (the row sums of a softmax are 1);
+ *   - path A adds the conv of 2.6 like the Nystrom path;
  *   - a masked key gets score -inf in kernel_3 only (probability exactly 0);
  *   - Conv2d is cross-correlation: tap t multiplies V[i + t - 32], zero
  *     outside [0, n).
@@ -43,6 +49,8 @@
 #endif
 
 #define NYS_ORACLE_TAPS 65
+
+static void scaled_copy(const float* x, int n, int d, double s, double* y);
 
 /* Walkthrough 2.2: the 1/sqrt(d) softmax scale split evenly over Q and K. */
 static double split_scale(int d) { return 1.0 / sqrt(sqrt((double)d)); }
@@ -107,7 +115,7 @@ static void sub_from_scaled_identity(double* M, int m, double diag_value) {
         }
 }
 
-/* Scalar of the "original" Z_0 initialisation: 1 / (max column sum * max row sum). */
+/* Scalar of the default Z_0 initialisation: 1 / (max column sum * max row sum). */
 double nys_oracle_init_coeff(const double* A, int m) {
     double max_col = -INFINITY, max_row = -INFINITY;
     for (int c = 0; c < m; ++c) {
@@ -124,16 +132,35 @@ double nys_oracle_init_coeff(const double* A, int m) {
 }
 
 /*
+ * Scalar of the "exact coefficient" Z_0 initialisation (walkthrough 2.5, second
+ * bullet; the inv_coeff_init_option row of the 3.1 table): c = 1 / ||A||_1, the
+ * largest column sum. Reading: the rows of kernel_2 are normalised by its softmax,
+ * so ||A||_inf = 1 and the exact coefficient 1 / (||A||_1 ||A||_inf) is 1 / ||A||_1;
+ * the row factor is taken as 1, not computed.
+ */
+double nys_oracle_init_coeff_exact(const double* A, int m) {
+    double max_col = -INFINITY;
+    for (int c = 0; c < m; ++c) {
+        double s = 0.0;
+        for (int r = 0; r < m; ++r) s += A[(size_t)r * m + c];
+        max_col = s > max_col ? s : max_col;
+    }
+    return 1.0 / max_col;
+}
+
+/*
  * Walkthrough 2.5: iterative Moore-Penrose inverse of the m x m matrix A.
  *   Z = c A^T;  repeat n_iter times:
  *     X = A Z;  T = 7I - X;  T = X T;  T = 15I - T;  T = X T;  T = 13I - T;  Z = 1/4 Z T
+ * init_option 0: c from nys_oracle_init_coeff (the default); 1: from
+ * nys_oracle_init_coeff_exact (inv_coeff_init_option = True).
  */
-void nys_oracle_iterative_inv(const double* A, int m, int n_iter, double* Z) {
+void nys_oracle_iterative_inv_opt(const double* A, int m, int n_iter, int init_option, double* Z) {
     const size_t mm = (size_t)m * m;
     double* X = (double*)malloc(mm * sizeof(double));
     double* T = (double*)malloc(mm * sizeof(double));
     double* U = (double*)malloc(mm * sizeof(double));
-    const double c = nys_oracle_init_coeff(A, m);
+    const double c = init_option ? nys_oracle_init_coeff_exact(A, m) : nys_oracle_init_coeff(A, m);
     for (int r = 0; r < m; ++r)
         for (int k = 0; k < m; ++k) Z[(size_t)r * m + k] = c * A[(size_t)k * m + r];
     for (int it = 0; it < n_iter; ++it) {
@@ -152,6 +179,10 @@ void nys_oracle_iterative_inv(const double* A, int m, int n_iter, double* Z) {
     free(U);
 }
 
+void nys_oracle_iterative_inv(const double* A, int m, int n_iter, double* Z) {
+    nys_oracle_iterative_inv_opt(A, m, n_iter, 0, Z);
+}
+
 /* Walkthrough 2.6: out[i][c] += sum_t w[t] * v[i + t - 32][c], zero outside [0, n). */
 void nys_oracle_dwconv_add(const float* v, const float* w, int n, int d, double* out) {
     const int half = NYS_ORACLE_TAPS / 2;
@@ -167,6 +198,60 @@ void nys_oracle_dwconv_add(const float* v, const float* w, int n, int d, double*
         }
 }
 
+/* 2.6 for selected rows: out[r][c] += sum_t w[t] * v[rows[r] + t - 32][c] (rows == NULL: all n). */
+static void conv_rows_add(const float* v, const float* w, int n, int d, const int* rows, int nr,
+                          double* out) {
+    if (!rows) {
+        nys_oracle_dwconv_add(v, w, n, d, out);
+        return;
+    }
+    const int half = NYS_ORACLE_TAPS / 2;
+    for (int r = 0; r < nr; ++r)
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int t = 0; t < NYS_ORACLE_TAPS; ++t) {
+                int src = rows[r] + t - half;
+                if (src < 0 || src >= n) continue;
+                acc += (double)w[t] * (double)v[(size_t)src * d + c];
+            }
+            out[(size_t)r * d + c] += acc;
+        }
+}
+
+/*
+ * Walkthrough 2.1, path A: when num_landmarks equals the segment length the layer
+ * computes full softmax attention instead of the approximation. One (batch, head):
+ * with Qs = d^-1/4 Q and Ks = d^-1/4 K (2.2, applied before either path),
+ *   probs = softmax_row(Qs Ks^T + mask)   [n x n], padded keys -> 0
+ *   out   = probs V, then the conv of 2.6 is added.
+ * rows / n_rows select the query rows as in nys_oracle_head; probs_out (or NULL)
+ * receives the selected rows of probs, [n_rows, n].
+ */
+int nys_oracle_exact_head(const float* q, const float* k, const float* v, const uint8_t* keep,
+                          const float* w, int n, int d, const int* rows, int n_rows, double* out,
+                          double* probs_out) {
+    if (n <= 0 || d <= 0) return -1;
+    const double s = split_scale(d);
+    const int nr = rows ? n_rows : n;
+    double* ks = (double*)malloc((size_t)n * d * sizeof(double));
+    double* vd = (double*)malloc((size_t)n * d * sizeof(double));
+    double* qs = (double*)malloc((size_t)nr * d * sizeof(double));
+    double* p = (double*)malloc((size_t)nr * n * sizeof(double));
+    scaled_copy(k, n, d, s, ks);
+    scaled_copy(v, n, d, 1.0, vd);
+    for (int r = 0; r < nr; ++r) {
+        int i = rows ? rows[r] : r;
+        for (int c = 0; c < d; ++c) qs[(size_t)r * d + c] = s * (double)q[(size_t)i * d + c];
+    }
+    matmul_bt(qs, ks, nr, d, n, p);
+    nys_oracle_softmax_rows(p, nr, n, keep);
+    matmul(p, vd, nr, n, d, out);
+    if (w) conv_rows_add(v, w, n, d, rows, nr, out);
+    if (probs_out) memcpy(probs_out, p, (size_t)nr * n * sizeof(double));
+    free(ks); free(vd); free(qs); free(p);
+    return 0;
+}
+
 /* Scaled copy of a [n, d] float32 block into double. */
 static void scaled_copy(const float* x, int n, int d, double s, double* y) {
     for (size_t e = 0; e < (size_t)n * d; ++e) y[e] = s * (double)x[e];
@@ -179,10 +264,10 @@ static void scaled_copy(const float* x, int n, int d, double s, double* y) {
  * NULL): ql, kl [m, d]; k2, z [m, m]; k3v [m, d].
  */
 int nys_oracle_head(const float* q, const float* k, const float* v, const uint8_t* keep,
-                    const float* w, int n, int d, int m, int n_iter,
+                    const float* w, int n, int d, int m, int n_iter, int init_option,
                     const int* rows, int n_rows, double* out,
                     double* ql_out, double* kl_out, double* k2_out, double* z_out,
-                    double* k3v_out) {
+                    double* k3v_out, double* probs_out) {
     if (n <= 0 || d <= 0 || m <= 0 || n % m != 0 || m > n || n_iter < 0) return -1;
     const double s = split_scale(d);
     const int nr = rows ? n_rows : n;
@@ -207,7 +292,7 @@ int nys_oracle_head(const float* q, const float* k, const float* v, const uint8_
     nys_oracle_softmax_rows(k2, m, m, NULL);
 
     /* 2.5 Z = iterative_inv(kernel_2) */
-    nys_oracle_iterative_inv(k2, m, n_iter, z);
+    nys_oracle_iterative_inv_opt(k2, m, n_iter, init_option, z);
 
     /* 2.4 kernel_3 = softmax(Q_l Ks^T + mask); new_value = kernel_3 V */
     scaled_copy(k, n, d, s, ks);
@@ -229,23 +314,9 @@ int nys_oracle_head(const float* q, const float* k, const float* v, const uint8_
     matmul(probs, k3v, nr, m, d, out);
 
     /* 2.6 context += depthwise conv of V */
-    if (w) {
-        if (!rows) {
-            nys_oracle_dwconv_add(v, w, n, d, out);
-        } else {
-            const int half = NYS_ORACLE_TAPS / 2;
-            for (int r = 0; r < nr; ++r)
-                for (int c = 0; c < d; ++c) {
-                    double acc = 0.0;
-                    for (int t = 0; t < NYS_ORACLE_TAPS; ++t) {
-                        int src = rows[r] + t - half;
-                        if (src < 0 || src >= n) continue;
-                        acc += (double)w[t] * (double)v[(size_t)src * d + c];
-                    }
-                    out[(size_t)r * d + c] += acc;
-                }
-        }
-    }
+    if (w) conv_rows_add(v, w, n, d, rows, nr, out);
+    /* 2.7 the attention weights returned for output_attentions: attention_probs = kernel_1 Z */
+    if (probs_out) memcpy(probs_out, probs, (size_t)nr * m * sizeof(double));
 
     if (ql_out) memcpy(ql_out, ql, (size_t)m * d * sizeof(double));
     if (kl_out) memcpy(kl_out, kl, (size_t)m * d * sizeof(double));
@@ -261,15 +332,19 @@ int nys_oracle_head(const float* q, const float* k, const float* v, const uint8_
  * Whole batch: q, k, v [B, H, n, d]; mask [B, n] or NULL; conv_w [H, 65] or NULL.
  * rows/n_rows as in nys_oracle_head (the same rows for every head); out is
  * [B, H, n_rows, d] (n_rows = n when rows == NULL). Optional per-head stage
- * outputs: ql, kl, k3v [B, H, m, d]; k2, z [B, H, m, m]. threads <= 0 uses
- * the OpenMP default. Returns 0, or -1 on an invalid shape.
+ * outputs: ql, kl, k3v [B, H, m, d]; k2, z [B, H, m, m]; probs [B, H, n_rows, m]
+ * (kernel_1 Z), or [B, H, n_rows, n] on the exact path. init_option selects the
+ * Z_0 coefficient (0 default, 1 exact); exact != 0 takes path A (m, n_iter and
+ * init_option unused; the stage outputs other than probs are not written).
+ * threads <= 0 uses the OpenMP default. Returns 0, or -1 on an invalid shape.
  */
 int nys_oracle_forward(const float* q, const float* k, const float* v, const uint8_t* mask,
                        const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
-                       const int* rows, int n_rows, int threads, double* out,
-                       double* ql, double* kl, double* k2, double* z, double* k3v) {
-    if (B <= 0 || H <= 0 || n <= 0 || d <= 0 || m <= 0 || n % m != 0 || m > n || n_iter < 0)
-        return -1;
+                       int init_option, int exact, const int* rows, int n_rows, int threads,
+                       double* out, double* ql, double* kl, double* k2, double* z, double* k3v,
+                       double* probs) {
+    if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return -1;
+    if (!exact && (m <= 0 || n % m != 0 || m > n || n_iter < 0)) return -1;
     const int nr = rows ? n_rows : n;
     int bad = 0;
 #ifdef _OPENMP
@@ -282,11 +357,19 @@ int nys_oracle_forward(const float* q, const float* k, const float* v, const uin
         const int b = bh / H, h = bh % H;
         const size_t off = (size_t)bh * n * d;
         const size_t md = (size_t)bh * m * d, mm = (size_t)bh * m * m;
-        bad |= nys_oracle_head(q + off, k + off, v + off, mask ? mask + (size_t)b * n : NULL,
-                               conv_w ? conv_w + (size_t)h * NYS_ORACLE_TAPS : NULL, n, d, m,
-                               n_iter, rows, nr, out + (size_t)bh * nr * d,
-                               ql ? ql + md : NULL, kl ? kl + md : NULL, k2 ? k2 + mm : NULL,
-                               z ? z + mm : NULL, k3v ? k3v + md : NULL) != 0;
+        const uint8_t* keep = mask ? mask + (size_t)b * n : NULL;
+        const float* wh = conv_w ? conv_w + (size_t)h * NYS_ORACLE_TAPS : NULL;
+        if (exact) {
+            bad |= nys_oracle_exact_head(q + off, k + off, v + off, keep, wh, n, d, rows, nr,
+                                         out + (size_t)bh * nr * d,
+                                         probs ? probs + (size_t)bh * nr * n : NULL) != 0;
+        } else {
+            bad |= nys_oracle_head(q + off, k + off, v + off, keep, wh, n, d, m, n_iter, init_option,
+                                   rows, nr, out + (size_t)bh * nr * d,
+                                   ql ? ql + md : NULL, kl ? kl + md : NULL, k2 ? k2 + mm : NULL,
+                                   z ? z + mm : NULL, k3v ? k3v + md : NULL,
+                                   probs ? probs + (size_t)bh * nr * m : NULL) != 0;
+        }
     }
     return bad ? -1 : 0;
 }

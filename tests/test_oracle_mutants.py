@@ -34,6 +34,16 @@ MUTANTS = {
     "init_row_sum_twice": ("return 1.0 / (max_col * max_row);", "return 1.0 / (max_row * max_row);"),
     "extra_iteration": ("for (int it = 0; it < n_iter; ++it) {", "for (int it = 0; it <= n_iter; ++it) {"),
     "z_transposed_in_product": ("matmul(k1, z, nr, m, m, probs);", "matmul_bt(k1, z, nr, m, m, probs);"),
+    "init_exact_row_sums": ("        for (int r = 0; r < m; ++r) s += A[(size_t)r * m + c];\n        max_col = s > max_col ? s : max_col;\n    }\n    return 1.0 / max_col;",
+                            "        for (int r = 0; r < m; ++r) s += A[(size_t)c * m + r];\n        max_col = s > max_col ? s : max_col;\n    }\n    return 1.0 / max_col;"),
+    "init_option_ignored": ("const double c = init_option ? nys_oracle_init_coeff_exact(A, m) : nys_oracle_init_coeff(A, m);",
+                            "const double c = nys_oracle_init_coeff(A, m);"),
+    "exact_mask_ignored": ("nys_oracle_softmax_rows(p, nr, n, keep);", "nys_oracle_softmax_rows(p, nr, n, NULL);"),
+    "exact_no_conv": ("    if (w) conv_rows_add(v, w, n, d, rows, nr, out);\n    if (probs_out) memcpy(probs_out, p,",
+                      "    if (probs_out) memcpy(probs_out, p,"),
+    "exact_unscaled_k": ("    scaled_copy(k, n, d, s, ks);\n    scaled_copy(v, n, d, 1.0, vd);\n    for (int r = 0; r < nr; ++r) {",
+                         "    scaled_copy(k, n, d, 1.0, ks);\n    scaled_copy(v, n, d, 1.0, vd);\n    for (int r = 0; r < nr; ++r) {"),
+    "probs_are_kernel1": ("if (probs_out) memcpy(probs_out, probs, ", "if (probs_out) memcpy(probs_out, k1, "),
 }
 
 

@@ -7,6 +7,8 @@ index or axis, or a transposed operand anywhere in the oracle fails at least
 one of them. Citations name "Nystromformer source walkthrough"
 (blog.gitcode.com) and its sections.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import scipy.special
@@ -109,6 +111,35 @@ def test_init_coeff_is_inverse_of_one_times_inf_norm(oracle_mod):
     a = _rng(8).random((40, 40))
     assert oracle_mod.init_coeff(a) == pytest.approx(
         1.0 / (np.linalg.norm(a, 1) * np.linalg.norm(a, np.inf)), rel=1e-14)
+
+
+def test_init_coeff_exact_is_inverse_of_one_norm(oracle_mod):
+    """The exact-coefficient option (walkthrough 2.5, second bullet): c = 1 / ||A||_1."""
+    a = _rng(18).random((40, 40))
+    assert oracle_mod.init_coeff(a, init_option=1) == pytest.approx(1.0 / np.linalg.norm(a, 1), rel=1e-14)
+
+
+@pytest.mark.parametrize("n_iter", [0, 1, 6])
+def test_iterative_inv_exact_coefficient_closed_form(oracle_mod, n_iter):
+    """With Z_0 = A^T / ||A||_1 every iterate is the SVD closed form at c = 1 / ||A||_1. The
+    coefficient presumes rows summing to at most 1 (a softmax kernel); this matrix is a
+    softmax kernel with rows scaled to sums in [0.5, 0.9], so its column sums, its row sums
+    and the two coefficients all differ while the iteration still converges."""
+    a = _kernel2_like(24, 19, scale=1.5) * np.linspace(0.5, 0.9, 24)[:, None]
+    assert np.linalg.norm(a, 1) > 1.2 * np.linalg.norm(a, np.inf)
+    assert abs(oracle_mod.init_coeff(a, 1) / oracle_mod.init_coeff(a, 0) - 1.0) > 0.05
+    z = oracle_mod.iterative_inv(a, n_iter, init_option=1)
+    ref = _phi_closed_form(a, 1.0 / np.linalg.norm(a, 1), n_iter)
+    assert np.linalg.norm(z - ref) <= 1e-10 * np.linalg.norm(ref)
+
+
+def test_exact_coefficient_on_a_softmax_kernel_is_the_default(oracle_mod):
+    """For kernel_2 (rows normalised by the softmax) the row factor of the default
+    coefficient is 1, so both options give the same Z up to rounding."""
+    a = _kernel2_like(64, 20, scale=2.0)
+    z0 = oracle_mod.iterative_inv(a, 6)
+    z1 = oracle_mod.iterative_inv(a, 6, init_option=1)
+    assert np.linalg.norm(z1 - z0) <= 1e-12 * np.linalg.norm(z0)
 
 
 def test_iterative_inv_converges_to_library_pinv(oracle_mod):
@@ -255,3 +286,59 @@ def test_rejects_bad_shapes(oracle_mod):
     q = np.zeros((1, 1, 100, 8), np.float32)
     with pytest.raises(ValueError):
         oracle_mod.forward(q, q, q, m=64)  # 100 % 64 != 0
+
+
+# ---------------------------------------------------------------- exact branch (2.1) and the
+# returned attention weights (2.7)
+
+def _sdpa(q, k, v, mask=None):
+    """torch's scaled_dot_product_attention in float64 (scale 1/sqrt(d)): the library routine
+    whose definition path A of walkthrough 2.1 names."""
+    t = lambda a: torch.from_numpy(np.asarray(a, dtype=np.float64))
+    am = None if mask is None else torch.from_numpy(mask[None, :] > 0)
+    return torch.nn.functional.scaled_dot_product_attention(t(q)[None], t(k)[None], t(v)[None],
+                                                            attn_mask=am)[0].numpy()
+
+
+@pytest.mark.parametrize("masked", [False, True])
+def test_exact_path_is_library_attention_plus_conv(oracle_mod, masked):
+    w = dataclasses.replace(WORKLOADS["default_f32_masked"], lengths=(40, 150))
+    x = make_inputs(w, seed=21, B=2, H=2, n=192)
+    mask = x["mask"] if masked else None
+    assert mask is None or (mask == 0).any(axis=1).all()
+    out, st = oracle_mod.forward(x["q"], x["k"], x["v"], mask, x["conv_w"], exact=True, probs=True)
+    conv = torch.nn.functional.conv2d(torch.from_numpy(x["v"].astype(np.float64)),
+                                      torch.from_numpy(x["conv_w"].astype(np.float64)).view(2, 1, 65, 1),
+                                      padding=(32, 0), groups=2).numpy()
+    for b in range(2):
+        for h in range(2):
+            mk = None if mask is None else mask[b]
+            ref = _sdpa(x["q"][b, h], x["k"][b, h], x["v"][b, h], mk)
+            np.testing.assert_allclose(out[b, h], ref + conv[b, h], rtol=1e-10, atol=1e-12)
+            if mk is not None:
+                assert np.all(st["probs"][b, h][:, mk == 0] == 0.0)
+            np.testing.assert_allclose(st["probs"][b, h].sum(1), 1.0, atol=1e-12)
+
+
+def test_exact_path_equals_nystrom_at_m_equals_n(oracle_mod):
+    """m = n with a converged inverse reproduces path A (A A^+ A = A, walkthrough 2.1)."""
+    r = _rng(22)
+    n, d = 48, 16
+    q, k, v = (r.standard_normal((1, 1, n, d)).astype(np.float32) for _ in range(3))
+    a = oracle_mod.forward(q, k, v, None, None, exact=True)
+    b = oracle_mod.forward(q, k, v, None, None, m=n, n_iter=30)
+    assert np.linalg.norm(a - b) / np.linalg.norm(a) < 1e-9
+
+
+def test_probs_are_kernel1_times_z(oracle_mod):
+    """The returned weights (2.7) times kernel_3 V give the attention term (2.4), and at m = n
+    with a converged inverse they are A A^+ = I for the nonsingular A of these inputs."""
+    w = WORKLOADS["default_f32_masked"]
+    x = make_inputs(w, seed=23, B=1, H=2, n=128)
+    out, st = oracle_mod.forward(x["q"], x["k"], x["v"], x["mask"], None, m=16, stages=True, probs=True)
+    for h in range(2):
+        np.testing.assert_allclose(st["probs"][0, h] @ st["k3v"][0, h], out[0, h], rtol=1e-10, atol=1e-12)
+    r = _rng(24)
+    q, k, v = (r.standard_normal((1, 1, 32, 16)).astype(np.float32) for _ in range(3))
+    _, st = oracle_mod.forward(q, k, v, None, None, m=32, n_iter=30, probs=True)
+    np.testing.assert_allclose(st["probs"][0, 0], np.eye(32), atol=1e-9)
