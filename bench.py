@@ -109,16 +109,26 @@ def source_digest(kernel=None):
 
 # ---------------------------------------------------------------- algorithmic work per launch
 
-def kernel_work(w, kernel):
+def kernel_work(w, kernel, path="nystrom"):
     """(algorithmic bytes, algorithmic flops, compute unit) of one launch of `kernel`.
 
     Bytes count each input element read once and each output written once;
     flops count 2 per multiply-add of the dense contractions (softmax
-    exponentials are not counted)."""
+    exponentials are not counted). On the exact branch (path A) kernel_3 V's
+    machinery runs with all n query rows: 4 n^2 d flops per head, Q, K, V read;
+    its epilogue (merge, conv, output) is the "output" kernel."""
     elt = 4 if w.dtype == "f32" else 2
     BH, n, d, m = w.BH, w.n, w.d, w.m
     tensor = BH * n * d * elt
     unit = "alu" if w.dtype == "f32" else "tensor"
+    if path == "exact":
+        if kernel == "k3v_partial":
+            return 3 * tensor, BH * 4 * n * n * d, unit
+        if kernel == "output":
+            return 2 * tensor + BH * n * d * 4 * 3, BH * 2 * 65 * n * d if w.conv else 0, "alu"
+        if kernel == "mask_bits":
+            return w.B * n + w.B * n // 8, 0, "alu"
+        raise KeyError(kernel)
     if kernel == "landmarks":
         return 2 * tensor + 2 * BH * m * d * 4, 0, "alu"
     if kernel == "pinv":
@@ -151,8 +161,8 @@ def compute_peak_tflops(unit, peaks, kernel_impl_simt):
 SIMT_KERNELS = {"landmarks", "k3v_combine", "w_product", "kernel2", "mask_bits"}
 
 
-def roofline_for(w, kernel, avg_ms, peaks, simt_set, traffic):
-    nbytes, flops, unit = kernel_work(w, kernel)
+def roofline_for(w, kernel, avg_ms, peaks, simt_set, traffic, path="nystrom"):
+    nbytes, flops, unit = kernel_work(w, kernel, path)
     simt = kernel in simt_set
     t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
     cpk = compute_peak_tflops(unit, peaks, simt)
@@ -198,6 +208,38 @@ def roofline_bound_time_pipes(w, peaks):
     tf32 = w.BH * (w.n_iter * 8 * m ** 3 + 3 * 2 * m * m * d)
     t_flops = bf16 / (peaks["bf16_tflops"] * 1e12) + tf32 / (compute_peak_tflops("tensor_tf32", peaks, False) * 1e12)
     return max(nbytes / (peaks["hbm_gbs"] * 1e9), t_flops)
+
+
+def roofline_bound_time_exact(w, peaks):
+    """The exact branch (path A): t_roof = max(ideal bytes / HBM, flops / peak) with 4 n^2 d
+    flops per head (Q K^T and P V) plus the conv; same ideal bytes as the Nystrom step."""
+    elt = 4 if w.dtype == "f32" else 2
+    nbytes = 4 * w.BH * w.n * w.d * elt
+    flops = w.BH * (4 * w.n * w.n * w.d + (2 * 65 * w.n * w.d if w.conv else 0))
+    peak = peaks["bf16_tflops"] if w.dtype == "bf16" else compute_peak_tflops("alu", peaks, True)
+    return max(nbytes / (peaks["hbm_gbs"] * 1e9), flops / (peak * 1e12)), nbytes, flops
+
+
+MUFU_EX2_PER_CLK_SM = 16   # nominal special-function-unit rate of ex2.approx.f32 per SM
+
+
+def step_exponentials(w, path="nystrom"):
+    """Exponentials of one step: kernel_1 (n x m) and kernel_3 (m x n) per head; kernel_2's
+    m x m is negligible and not counted. The exact branch: n x n per head."""
+    if path == "exact":
+        return w.BH * w.n * w.n
+    return 2 * w.BH * w.n * w.m
+
+
+def roofline_bound_time_exp(w, peaks, path="nystrom"):
+    """The pipe-aware bound with the softmax exponentials added: every exponential charged to
+    the MUFU unit at its nominal ex2.f32 rate (16 per clock per SM at the maximum SM clock),
+    and the step bounded by the slowest of HBM traffic, tensor-pipe FLOP and MUFU time (the
+    three pipes run concurrently). The kernels also evaluate part of the exponentials as
+    FMA-pipe polynomials, so a kernel can beat the MUFU term; it is a reference, not a floor."""
+    t_exp = step_exponentials(w, path) / (N_SMS * MUFU_EX2_PER_CLK_SM * peaks.get("sm_max_mhz", 1965.0) * 1e6)
+    base = roofline_bound_time_exact(w, peaks)[0] if path == "exact" else roofline_bound_time_pipes(w, peaks)
+    return max(base, t_exp), t_exp
 
 
 # ---------------------------------------------------------------- clocks
@@ -389,6 +431,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-flush", action="store_true")
+    ap.add_argument("--path", default="nystrom", choices=["nystrom", "exact"],
+                    help="exact: the layer's path A (exact softmax attention), through nys_attn_forward_ex")
+    ap.add_argument("--inv-init", default="default", choices=["default", "exact"],
+                    help="exact: the exact-coefficient Z_0 (inv_coeff_init_option), through nys_attn_forward_ex")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         ap.error("--warmup must be >= 3")
@@ -425,8 +471,14 @@ def main():
         flush.zero_()
         torch.sum(flush_clean, dim=0, keepdim=True, out=flush_sink)
 
+    use_ex = args.path != "nystrom" or args.inv_init != "default"
+
     def step():
-        nys.forward(q, k, v, mask=mask, conv_w=conv_w, m=w.m, n_iter=w.n_iter, out=out)
+        if use_ex:
+            nys.forward_ex(q, k, v, mask=mask, conv_w=conv_w, m=w.m, n_iter=w.n_iter, out=out,
+                           inv_coeff_init_option=args.inv_init == "exact", exact=args.path == "exact")
+        else:
+            nys.forward(q, k, v, mask=mask, conv_w=conv_w, m=w.m, n_iter=w.n_iter, out=out)
 
     for _ in range(args.warmup):
         if not args.no_flush:
@@ -503,13 +555,20 @@ def main():
     simt = set(SIMT_KERNELS)
     if w.dtype == "f32":  # the float32 path runs every stage on CUDA cores
         simt |= {"pinv", "k3v_partial", "output"}
-    roof = roofline_for(w, dom, prof[dom][1] / max(1, prof[dom][0]), peaks, simt, traffic)
+    if args.path == "exact":
+        traffic = None   # the ncu traffic figures are for the Nystrom path's kernels
+    roof = roofline_for(w, dom, prof[dom][1] / max(1, prof[dom][0]), peaks, simt, traffic, args.path)
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
-    t_roof, ideal_bytes, total_flops = roofline_bound_time(w, peaks)
-    t_pipes = roofline_bound_time_pipes(w, peaks)
+    if args.path == "exact":
+        t_roof, ideal_bytes, total_flops = roofline_bound_time_exact(w, peaks)
+        t_pipes = t_roof
+    else:
+        t_roof, ideal_bytes, total_flops = roofline_bound_time(w, peaks)
+        t_pipes = roofline_bound_time_pipes(w, peaks)
+    t_exp_roof, t_exp = roofline_bound_time_exp(w, peaks, args.path)
 
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not use_ex:
         qh = torch.from_numpy(x["q"]).to(dt).pin_memory()
         kh = torch.from_numpy(x["k"]).to(dt).pin_memory()
         vh = torch.from_numpy(x["v"]).to(dt).pin_memory()
@@ -537,7 +596,7 @@ def main():
                "steps": args.e2e_steps, "ms_per_step": round(e_ms / args.e2e_steps, 3)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not use_ex:
         cpu = cpu_baseline(w, x)
 
     if rank == 0:
@@ -549,6 +608,7 @@ def main():
             "config": {"workload": w.name, "B": w.B, "H": w.H, "n": w.n, "d": w.d, "m": w.m,
                        "n_iter": w.n_iter, "conv": w.conv, "mask": w.lengths is not None,
                        "inputs": w.dist, "parallelism": "replicas" if world > 1 else "single",
+                       "path": args.path, "inv_init": args.inv_init,
                        "l2": "not flushed" if args.no_flush else
                        "flushed before every step (256 MiB write, then a 256 MiB read of another buffer; untimed)"},
             "roofline": roof,
@@ -557,6 +617,12 @@ def main():
             "step_roofline_pipes": {"t_roof_us": round(t_pipes * 1e6, 2),
                                     "frac": round(t_pipes / (ms_per_step * 1e-3), 4),
                                     "note": "inverse (and kernel_2) at the tf32 tensor rate, the rest at bf16"},
+            "step_roofline_exp": {"t_roof_us": round(t_exp_roof * 1e6, 2),
+                                  "frac": round(t_exp_roof / (ms_per_step * 1e-3), 4),
+                                  "t_exp_us": round(t_exp * 1e6, 2),
+                                  "exponentials": step_exponentials(w, args.path),
+                                  "note": "pipe-aware bound with every softmax exponential on the MUFU "
+                                          f"unit at {MUFU_EX2_PER_CLK_SM}/clk/SM"},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "kernels": kernels,
             "kernels_source": f"separate untimed pass of {breakdown_steps} steps, every launch bracketed by "

@@ -48,6 +48,12 @@ extern "C" {
 #define NYS_CONV_TAPS 65
 /* Default iteration count of the iterative inverse (walkthrough 2.5). */
 #define NYS_DEFAULT_N_ITER 6
+/* Z_0 scaling of the iterative inverse (walkthrough 2.5, the two bullets; the
+ * inv_coeff_init_option row of the 3.1 table): DEFAULT takes
+ * c = 1 / (max column sum * max row sum) of kernel_2, EXACT (the option set
+ * to True) takes c = 1 / max column sum = 1 / ||kernel_2||_1. */
+#define NYS_INV_INIT_DEFAULT 0
+#define NYS_INV_INIT_EXACT 1
 
 typedef enum {
     NYS_F32 = 0,   /* float32 in, float32 out, float32 arithmetic               */
@@ -86,6 +92,33 @@ typedef enum {
 int nys_attn_forward(const void* q, const void* k, const void* v, const uint8_t* key_mask,
                      const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
                      int dtype, void* out, void* stream);
+
+/*
+ * nys_attn_forward_ex -- nys_attn_forward with the layer's other options.
+ *
+ *   inv_init    NYS_INV_INIT_DEFAULT, or NYS_INV_INIT_EXACT for the
+ *               "exact coefficient" Z_0 = k2^T / ||k2||_1 (walkthrough 2.5,
+ *               second bullet; inv_coeff_init_option = True in the 3.1 table)
+ *   exact       0: the Nystrom path. Nonzero: path A of walkthrough 2.1, the
+ *               branch the layer takes when num_landmarks equals the segment
+ *               length: out = softmax_row(Qs Ks^T + mask) V + dwconv65(V), with
+ *               Qs, Ks scaled by d^-1/4 as in 2.2 and the same mask and conv
+ *               conventions. m, n_iter and inv_init are then ignored (not
+ *               checked); bf16 needs n % 128 == 0.
+ *   attn_probs  NULL, or a device float32 buffer for the attention weights the
+ *               layer returns with output_attentions (walkthrough 2.7):
+ *               [B, H, n, m] = kernel_1 Z on the Nystrom path, [B, H, n, n]
+ *               = softmax_row(Qs Ks^T + mask) on the exact path. Computed in
+ *               float32 on CUDA cores from the inputs and the call's float32
+ *               stages; it does not feed the main output.
+ * Everything else (layouts, checks, asynchrony, scratch) is as for
+ * nys_attn_forward; an inv_init other than the two values returns
+ * NYS_ERR_INVALID_ARG.
+ */
+int nys_attn_forward_ex(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                        const float* conv_w, int B, int H, int n, int d, int m, int n_iter,
+                        int dtype, int inv_init, int exact, void* out, float* attn_probs,
+                        void* stream);
 
 /*
  * nys_attn_forward_host -- the same operation on HOST buffers (same shapes,
@@ -147,16 +180,21 @@ int nys_attn_forward_debug(const void* q, const void* k, const void* v, const ui
  *             Z_0 = k2^T / (max column sum * max row sum)
  *   stream    a cudaStream_t (NULL = legacy default stream)
  * Supported: d in {32, 64}, 1 <= m <= 256, any BH >= 1 (heads run in
- * batches that fit the array; one head needs 5 m^2 floats). A head that
- * would need more than the array returns NYS_ERR_SCRATCH_LIMIT; bad
- * arguments return NYS_ERR_INVALID_ARG / NYS_ERR_UNSUPPORTED before any
- * launch. The call allocates nothing (no cudaMalloc, cudaFree or
- * allocating library routine).
+ * batches that fit the array; one head needs 5 m^2 floats, at most
+ * 1.25 MiB at m = 256, so a batch holds at least 6 heads). m > 256 returns
+ * NYS_ERR_UNSUPPORTED; NYS_ERR_SCRATCH_LIMIT is reserved for a head larger
+ * than the array, which no supported m reaches. Bad arguments return
+ * NYS_ERR_INVALID_ARG / NYS_ERR_UNSUPPORTED before any launch; a failed
+ * launch returns NYS_ERR_CUDA at once, without launching the remaining
+ * batches. The call allocates nothing (no cudaMalloc, cudaFree or
+ * allocating library routine). The buffers are not checked beyond null:
+ * q_l, k_l must hold BH*m*d floats and z BH*m*m floats.
  *
  * Set-up: the first call on a device (with that device current) looks up
  * the array's device address once; make that first call before any stream
- * capture begins. The array is held by every GPU that loads the library
- * until the process exits.
+ * capture begins. The address is looked up again if the device's context
+ * changed since (after cudaDeviceReset, for example). The array is held by
+ * every GPU that loads the library until the process exits.
  *
  * Sharing: every call uses the same array, which keeps the previous call's
  * contents (nothing in it needs to start at zero: each launch writes every
@@ -190,6 +228,21 @@ int nys_attn_version(void);
  * NYS_ERR_CUDA on a CUDA failure.
  */
 int nys_attn_selftest_exp2(float* max_rel_err);
+
+/*
+ * Self-test of the bounded device-side wait (an implementation check with no
+ * counterpart in the pages). Launches one CTA on the current device that
+ * waits on an mbarrier nothing arrives on, with the same bounded wait every
+ * kernel of the library uses but a limit of `limit_ns` nanoseconds (at most
+ * one second) instead of one second; no copy or tensor-core operation is in
+ * flight. The wait runs out, the kernel records NYS_ERR_TIMEOUT in the
+ * device status word (read it with nys_attn_device_status) and returns, so
+ * the context stays usable. Synchronous. *completed (host pointer) is set to
+ * 0 when the wait ran out and 1 if it had completed (which nothing can
+ * cause). NYS_ERR_INVALID_ARG for a null pointer or a limit of 0 or more than
+ * one second, NYS_ERR_CUDA on a CUDA failure.
+ */
+int nys_attn_selftest_wait_timeout(unsigned long long limit_ns, int* completed);
 
 /*
  * Per-kernel timing, for benchmarks. While enabled, each kernel launch of

@@ -26,6 +26,7 @@ DEFAULT_N_ITER = 6
 DEFAULT_NUM_LANDMARKS = 64
 
 F32, BF16 = 0, 1
+INV_INIT_DEFAULT, INV_INIT_EXACT = 0, 1
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape or dtype", -3: "CUDA error",
            -4: "device workspace allocation failed", -5: "bounded device wait timed out",
            -6: "problem exceeds the library's fixed static scratch"}
@@ -49,8 +50,9 @@ def _load() -> ctypes.CDLL:
     lib.nys_attn_forward.argtypes = fwd + [vp]
     lib.nys_attn_forward_host.argtypes = fwd + [vp]
     lib.nys_attn_forward_debug.argtypes = fwd + [vp, vp, vp, vp, vp, vp]
+    lib.nys_attn_forward_ex.argtypes = fwd[:-1] + [i, i, vp, vp, vp]
     for f in ("nys_attn_forward", "nys_attn_forward_host", "nys_attn_forward_debug",
-              "nys_attn_device_status", "nys_attn_version"):
+              "nys_attn_forward_ex", "nys_attn_device_status", "nys_attn_version"):
         getattr(lib, f).restype = ctypes.c_int
     lib.nys_attn_workspace_bytes.argtypes = [i, i, i, i, i, i]
     lib.nys_attn_workspace_bytes.restype = ctypes.c_size_t
@@ -65,6 +67,8 @@ def _load() -> ctypes.CDLL:
     lib.nys_attn_kernel_name.restype = ctypes.c_char_p
     lib.nys_attn_pinv_static.argtypes = [vp, vp, vp, i, i, i, i, vp]
     lib.nys_attn_pinv_static.restype = i
+    lib.nys_attn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_int)]
+    lib.nys_attn_selftest_wait_timeout.restype = i
     lib.nys_attn_selftest_exp2.argtypes = [ctypes.POINTER(ctypes.c_float)]
     lib.nys_attn_selftest_exp2.restype = i
     lib.nys_strerror.argtypes = [i]
@@ -139,6 +143,36 @@ def forward(q, k, v, mask=None, conv_w=None, m: int = DEFAULT_NUM_LANDMARKS,
     return out
 
 
+def takes_exact_path(num_landmarks: int, segment_means_seq_len: int) -> bool:
+    """The layer's branch rule (walkthrough 2.1, 3.1): path A, exact attention, when the
+    number of landmarks equals the segment-means sequence length."""
+    return int(num_landmarks) == int(segment_means_seq_len)
+
+
+def forward_ex(q, k, v, mask=None, conv_w=None, m: int = DEFAULT_NUM_LANDMARKS,
+               n_iter: int = DEFAULT_N_ITER, inv_coeff_init_option: bool = False,
+               exact: bool = False, output_attentions: bool = False, out=None, stream=None):
+    """forward() with the layer's other options (nys_attn_forward_ex): the exact Z_0
+    coefficient, the exact branch (path A), and the returned attention weights
+    ([B, H, n, m], or [B, H, n, n] on the exact path, float32). Returns out, or
+    (out, weights) when output_attentions is set."""
+    import torch
+    (B, H, n, d), mask, conv_w = _prep_device(q, k, v, mask, conv_w)
+    if out is None:
+        out = torch.empty_like(q)
+    probs = None
+    if output_attentions:
+        probs = torch.empty(B, H, n, n if exact else int(m), device=q.device, dtype=torch.float32)
+    s = stream if stream is not None else torch.cuda.current_stream(q.device)
+    with torch.cuda.device(q.device):
+        rc = lib.nys_attn_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(mask), _ptr(conv_w), B, H, n, d,
+                                     int(m), int(n_iter), _dtype_code(q),
+                                     INV_INIT_EXACT if inv_coeff_init_option else INV_INIT_DEFAULT,
+                                     1 if exact else 0, _ptr(out), _ptr(probs), s.cuda_stream)
+    _check(rc, "nys_attn_forward_ex")
+    return (out, probs) if output_attentions else out
+
+
 def forward_debug(q, k, v, mask=None, conv_w=None, m: int = DEFAULT_NUM_LANDMARKS,
                   n_iter: int = DEFAULT_N_ITER):
     """forward() plus the float32 stages: q_l, k_l, z, k3v, w (per head)."""
@@ -192,6 +226,15 @@ def selftest_exp2() -> float:
     return float(err.value)
 
 
+def selftest_wait_timeout(limit_ns: int = 1_000_000) -> int:
+    """Run the bounded-wait self-test (a wait nothing completes, limited to `limit_ns`);
+    returns 0 when the wait ran out (the expected result) and 1 if it completed."""
+    done = ctypes.c_int(-1)
+    _check(lib.nys_attn_selftest_wait_timeout(int(limit_ns), ctypes.byref(done)),
+           "nys_attn_selftest_wait_timeout")
+    return int(done.value)
+
+
 def workspace_bytes(B, H, n, d, m, dtype_code=BF16) -> int:
     return int(lib.nys_attn_workspace_bytes(B, H, n, d, m, dtype_code))
 
@@ -229,12 +272,34 @@ def profile_read() -> dict:
     return out
 
 
+def _check_pinv_static_args(q_l, k_l, out):
+    """Shape, dtype, device and layout checks of pinv_static() (no CUDA call): q_l and k_l
+    float32 [B, H, m, d] on one device, out (if given) a contiguous float32 [B, H, m, m] on
+    the same device. A wrong buffer here would make the kernel read or write out of bounds."""
+    import torch
+    if q_l.dim() != 4 or q_l.dtype != torch.float32:
+        raise ValueError("q_l must be a float32 [B, H, m, d] tensor")
+    if k_l.dtype != torch.float32 or tuple(k_l.shape) != tuple(q_l.shape):
+        raise ValueError("k_l must be a float32 tensor of q_l's shape")
+    if k_l.device != q_l.device:
+        raise ValueError("k_l must be on q_l's device")
+    if out is not None:
+        B, H, m, _ = (int(t) for t in q_l.shape)
+        if out.dtype != torch.float32 or tuple(out.shape) != (B, H, m, m):
+            raise ValueError("out must be a float32 [B, H, m, m] tensor")
+        if not out.is_contiguous():
+            raise ValueError("out must be contiguous")
+        if out.device != q_l.device:
+            raise ValueError("out must be on q_l's device")
+
+
 def pinv_static(q_l, k_l, n_iter: int = DEFAULT_N_ITER, out=None, stream=None):
     """kernel_2 + iterative inverse from float32 landmarks [B, H, m, d] -> Z [B, H, m, m],
     through the allocation-free entry point (scratch is a fixed array inside the library)."""
     import torch
-    if q_l.shape != k_l.shape or q_l.dim() != 4 or q_l.dtype != torch.float32 or not q_l.is_cuda:
-        raise ValueError("q_l, k_l must be float32 CUDA tensors of one [B, H, m, d] shape")
+    _check_pinv_static_args(q_l, k_l, out)
+    if not q_l.is_cuda:
+        raise ValueError("q_l, k_l must be CUDA tensors")
     B, H, m, d = (int(t) for t in q_l.shape)
     q_l, k_l = q_l.contiguous(), k_l.contiguous()
     if out is None:

@@ -78,4 +78,71 @@ landmarks_kernel(const T* __restrict__ q, const T* __restrict__ k, float* __rest
     }
 }
 
+// bf16, when one warp instruction covers whole rows (D = 64: 4 rows, D = 32: 8 rows) and
+// L is a multiple of that: one warp per landmark (grid-stride over the 2 * BH * m landmarks
+// of Q and K), reading the landmark's L contiguous rows as 512-byte warp instructions (lane l
+// takes 16-byte slice l % (D / 8) of row l / (D / 8) of each instruction), eight loads in
+// flight per lane; the lanes holding the same slice are summed with shuffles. Every warp
+// reads contiguous 4 KB runs, and the landmarks are spread over all warps of all SMs.
+template <int D>
+__global__ void __launch_bounds__(256)
+landmarks_warp_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                      float* __restrict__ ql, float* __restrict__ kl, __nv_bfloat16* __restrict__ ql16,
+                      __nv_bfloat16* __restrict__ kl16, int BH, int n, int m) {
+    constexpr int S = D / 8;        // 16-byte slices per row
+    constexpr int R = 32 / S;       // rows per warp instruction
+    constexpr int U = 8;            // loads in flight per lane
+    const int lane = threadIdx.x & 31;
+    const int slice = lane % S, rsub = lane / S;
+    const long long per_tensor = (long long)BH * m;
+    const long long units = 2 * per_tensor;
+    const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+    const int L = n / m;
+    const int instr = L / R;        // warp instructions per landmark
+    const float scale = split_scale(D) / (float)L;
+    for (long long u = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units; u += warps) {
+        const int which = u >= per_tensor;
+        const long long lm = which ? u - per_tensor : u;   // (bh, j) flattened
+        const __nv_bfloat16* src = (which ? k : q) + ((size_t)lm * L + rsub) * D + slice * 8;
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int t = 0; t < instr; t += U) {
+            // a batch of up to U loads, all issued before any is used (the last batch is predicated)
+            uint4 raw[U];
+#pragma unroll
+            for (int e = 0; e < U; ++e)
+                raw[e] = t + e < instr ? __ldg(reinterpret_cast<const uint4*>(src + (size_t)(t + e) * R * D))
+                                       : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int e = 0; e < U; ++e) {
+                const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[e]);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __bfloat1622float2(h2[i]);
+                    acc[2 * i] += f.x;
+                    acc[2 * i + 1] += f.y;
+                }
+            }
+        }
+#pragma unroll
+        for (int off = S; off < 32; off <<= 1)
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+        if (lane < S) {
+            float* dst = (which ? kl : ql) + (size_t)lm * D + slice * 8;
+            const float4 o0 = make_float4(acc[0] * scale, acc[1] * scale, acc[2] * scale, acc[3] * scale);
+            const float4 o1 = make_float4(acc[4] * scale, acc[5] * scale, acc[6] * scale, acc[7] * scale);
+            reinterpret_cast<float4*>(dst)[0] = o0;
+            reinterpret_cast<float4*>(dst)[1] = o1;
+            const __nv_bfloat162 b0 = __floats2bfloat162_rn(o0.x, o0.y), b1 = __floats2bfloat162_rn(o0.z, o0.w);
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(o1.x, o1.y), b3 = __floats2bfloat162_rn(o1.z, o1.w);
+            uint4 pk;
+            pk.x = *reinterpret_cast<const uint32_t*>(&b0);
+            pk.y = *reinterpret_cast<const uint32_t*>(&b1);
+            pk.z = *reinterpret_cast<const uint32_t*>(&b2);
+            pk.w = *reinterpret_cast<const uint32_t*>(&b3);
+            *reinterpret_cast<uint4*>((which ? kl16 : ql16) + (size_t)lm * D + slice * 8) = pk;
+        }
+    }
+}
+
 }  // namespace nys

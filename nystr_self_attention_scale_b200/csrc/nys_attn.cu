@@ -13,15 +13,19 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <vector>
 
 #include "common.cuh"
+#include "exact.cuh"
 #include "landmarks.cuh"
+#include "probs.cuh"
 #include "simt.cuh"
 #include "tc_k3v.cuh"
 #include "tc_output.cuh"
 #include "tc_pinv.cuh"
 #include "tc_pinv_pair.cuh"
+#include "tc_pinv_res.cuh"
 
 namespace nys {
 namespace {
@@ -76,6 +80,7 @@ int device_state(DeviceState** out) {
         cudaFuncSetAttribute(k3v_partial_simt_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
         cudaFuncSetAttribute(output_simt_kernel<float, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
         cudaFuncSetAttribute(output_simt_kernel<float, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)big);
+        cudaFuncSetAttribute(pinv_simt_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPinvSmemBytes);
         if (cudaGetLastError() != cudaSuccess) return NYS_ERR_CUDA;
         st.ready = true;
     }
@@ -153,9 +158,10 @@ bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
 // ---------------------------------------------------------------- per-kernel timing
 // When enabled, every launch is bracketed by two CUDA events on the stream it
 // runs on; nys_attn_profile_read() sums their elapsed times per kernel.
-enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_MASKBITS, K_KERNEL2, K_COUNT };
+enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_MASKBITS, K_KERNEL2, K_PROBS,
+                K_COUNT };
 const char* const kKernelNames[K_COUNT] = {"landmarks", "pinv", "k3v_partial", "k3v_combine",
-                                           "w_product", "output", "mask_bits", "kernel2"};
+                                           "w_product", "output", "mask_bits", "kernel2", "attn_probs"};
 
 struct ProfRecord { int kid; cudaEvent_t a, b; };
 std::mutex g_prof_mu;
@@ -207,6 +213,25 @@ struct Plan {
     int tc_cps, tc_splits;  // tensor-core kernel_3 V: 128-key chunks per split, splits
 };
 
+// Per-call options beyond the spec signature (nys_attn_forward_ex).
+struct Options {
+    int inv_init = NYS_INV_INIT_DEFAULT;   // Z_0 scaling of the iterative inverse
+    bool exact = false;                    // path A: exact softmax attention (m, n_iter unused)
+    float* attn_probs = nullptr;           // optional [B, H, n, m] (or [B, H, n, n] exact) weights
+};
+
+// Argument checks of the exact branch (walkthrough 2.1, path A): no landmarks.
+int validate_exact(const void* q, const void* k, const void* v, const void* out, int B, int H, int n,
+                   int d, int dtype) {
+    if (!q || !k || !v || !out) return NYS_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || n <= 0 || d <= 0) return NYS_ERR_INVALID_ARG;
+    if (dtype != NYS_F32 && dtype != NYS_BF16) return NYS_ERR_UNSUPPORTED;
+    if (d != 32 && d != 64) return NYS_ERR_UNSUPPORTED;
+    if (dtype == NYS_BF16 && n % 128 != 0) return NYS_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1 << 24) || n / 64 >= 65535) return NYS_ERR_UNSUPPORTED;
+    return NYS_OK;
+}
+
 int validate(const void* q, const void* k, const void* v, const void* out, int B, int H, int n,
              int d, int m, int n_iter, int dtype) {
     if (!q || !k || !v || !out) return NYS_ERR_INVALID_ARG;
@@ -219,6 +244,35 @@ int validate(const void* q, const void* k, const void* v, const void* out, int B
         return NYS_ERR_UNSUPPORTED;
     if ((long long)B * H > (1 << 24) || n / 64 >= 65535) return NYS_ERR_UNSUPPORTED;
     return NYS_OK;
+}
+
+// Workspace of the exact branch: the key-split partials of softmax(Qs Ks^T + mask) V over all
+// n query rows, and the packed key-mask bits. The key split depends on n only, as on the
+// Nystrom path: one split up to n = 8192 (the rows already give B*H*n/128 work items).
+Plan make_plan_exact(int B, int H, int n, int d, int dtype) {
+    Plan p{};
+    p.B = B; p.H = H; p.n = n; p.d = d; p.m = n; p.n_iter = 0; p.dtype = dtype;
+    p.BH = B * H;
+    int kps = std::min(((n + 63) / 64) * 64, 1024);
+    int splits = (n + kps - 1) / kps;
+    if (dtype == NYS_BF16) {
+        const int chunks = n / 128;
+        p.tc_cps = std::min(chunks, 64);
+        p.tc_splits = (chunks + p.tc_cps - 1) / p.tc_cps;
+        splits = p.tc_splits;
+        kps = p.tc_cps * 128;
+    }
+    p.splits = splits;
+    p.keys_per_split = kps;
+    const size_t BH = p.BH;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+    p.off_po = take(BH * splits * (size_t)n * d * 4);
+    p.off_pm = take(BH * splits * (size_t)n * 4);
+    p.off_pl = take(BH * splits * (size_t)n * 4);
+    p.off_mbits = take((size_t)B * ((n + 31) / 32) * 4);
+    p.total = o;
+    return p;
 }
 
 Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_count) {
@@ -273,7 +327,7 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
 
 template <typename T, int D>
 int launch_simt(const Plan& p, const DeviceState& st, const T* q, const T* k, const T* v,
-               const uint8_t* mask, const float* conv_w, T* out, char* ws, cudaStream_t s) {
+               const uint8_t* mask, const float* conv_w, T* out, char* ws, int inv_init, cudaStream_t s) {
     float* ql = reinterpret_cast<float*>(ws + p.off_ql);
     float* kl = reinterpret_cast<float*>(ws + p.off_kl);
     float* k3v = reinterpret_cast<float*>(ws + p.off_k3v);
@@ -296,7 +350,10 @@ int launch_simt(const Plan& p, const DeviceState& st, const T* q, const T* k, co
     if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
     {
         ProfScope ps(K_PINV, st.aux);
-        pinv_simt_kernel<<<BH, 256, 0, st.aux>>>(ql, kl, z, pinv, m, D, p.n_iter);
+        if (m <= 64)
+            pinv_simt_smem_kernel<<<BH, 256, kPinvSmemBytes, st.aux>>>(ql, kl, z, m, D, p.n_iter, inv_init);
+        else
+            pinv_simt_kernel<<<BH, 256, 0, st.aux>>>(ql, kl, z, pinv, m, D, p.n_iter, inv_init);
     }
     if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
     {
@@ -304,7 +361,7 @@ int launch_simt(const Plan& p, const DeviceState& st, const T* q, const T* k, co
         {
             ProfScope ps(K_K3V, s);
             k3v_partial_simt_kernel<T, D><<<grid, 256, k3v_simt_smem_bytes<D>(), s>>>(
-                ql, k, v, mask, po, pm, pl, p.H, n, m, p.splits, p.keys_per_split);
+                ql, k, v, mask, po, pm, pl, p.H, n, m, p.splits, p.keys_per_split, 1.f);
         }
         const long long threads = (long long)BH * m * (D / 4);
         ProfScope ps(K_COMBINE, s);
@@ -347,25 +404,41 @@ int launch_output_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* 
             return NYS_ERR_CUDA;
         attr_set[dev] = true;
     }
+    // programmatic dependent launch: the kernel may start while W (the kernel before it on this
+    // stream) finishes; it waits for W's completion before loading W^T
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(480);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     ProfScope ps(K_OUTPUT, s);
-    output_tc_kernel<D, M><<<grid, 480, C::kSmemBytes, s>>>(mq, mv, mo, mkl, mwt, prm);
+    if (cudaLaunchKernelEx(&cfg, output_tc_kernel<D, M>, mq, mv, mo, mkl, mwt, prm) != cudaSuccess)
+        return NYS_ERR_CUDA;
     return NYS_OK;
 }
 
+// kernel_3 V on the tensor cores; `rows` is the row operand [BH, p.m, D] bf16: the landmarks
+// Q_l (scaled by d^-1/4 already, so the exponent carries K's d^-1/4) or, on the exact branch,
+// the raw queries (p.m = n; the exponent carries the whole d^-1/2).
 template <int D>
-int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql16, const __nv_bfloat16* k,
+int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* rows, const __nv_bfloat16* k,
                   const __nv_bfloat16* v, const uint32_t* mbits, float* po, float* pm, float* pl, int sms,
-                  cudaStream_t s) {
+                  float score_scale, cudaStream_t s) {
     using C = K3vTc<D>;
     CUtensorMap mql, mk, mv;
     const CUtensorMapSwizzle sw = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const uint64_t BH = p.BH, n = p.n, m = p.m;
-    if (!map_bf16_3d(&mql, ql16, D, m, BH, D, 128, sw) || !map_bf16_3d(&mk, k, D, n, BH, D, 128, sw) ||
+    if (!map_bf16_3d(&mql, rows, D, m, BH, D, 128, sw) || !map_bf16_3d(&mk, k, D, n, BH, D, 128, sw) ||
         !map_bf16_3d(&mv, v, D, n, BH, D, 128, sw))
         return NYS_ERR_CUDA;
     const int halves = (p.m + 127) / 128;
     K3vTcParams prm{mbits, po, pm, pl, p.H, p.n, p.m, halves, p.tc_splits, p.tc_cps,
-                    p.BH * halves * p.tc_splits};
+                    p.BH * halves * p.tc_splits, score_scale};
     const int grid = std::min(prm.total_items, sms);
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
@@ -383,7 +456,7 @@ int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* ql1
 
 template <int M>
 int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const float* kl, float* z, char* ws,
-                   cudaStream_t s) {
+                   int inv_init, cudaStream_t s) {
     using C = PinvTc<M>;
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
@@ -412,7 +485,7 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     }
     PinvTcParams prm{k2b, k2tb, reinterpret_cast<uint8_t*>(ws + p.off_zb), reinterpret_cast<uint8_t*>(ws + p.off_ztb),
                      reinterpret_cast<uint8_t*>(ws + p.off_ta),
-                     reinterpret_cast<uint8_t*>(ws + p.off_tb), colsum, rowsum, z, p.n_iter};
+                     reinterpret_cast<uint8_t*>(ws + p.off_tb), colsum, rowsum, z, p.n_iter, inv_init};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.BH * C::kClusterSize);
     cfg.blockDim = dim3(128);
@@ -430,9 +503,47 @@ int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const 
     return NYS_OK;
 }
 
+// m = 64 and 128: kernel_2 and the iterative inverse in one CTA per 128 rows (two heads per CTA
+// at m = 64), every operand on chip. `started` (or null) fires once every CTA has begun.
+template <int MH>
+int launch_pinv_res(const Plan& p, const float* ql, const float* kl, float* z, int inv_init, cudaStream_t s,
+                    cudaEvent_t started) {
+    using C = PinvRes<MH>;
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(pinv_res_kernel<MH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)C::kSmemBytes) != cudaSuccess)
+            return NYS_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    PinvResMaps maps;
+    const uint64_t BH = p.BH;
+    const auto f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (!map_3d(&maps.ql, f32, 4, ql, p.d, MH, BH, 32, MH, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !map_3d(&maps.kl, f32, 4, kl, p.d, MH, BH, 32, MH, CU_TENSOR_MAP_SWIZZLE_128B))
+        return NYS_ERR_CUDA;
+    PinvResParams prm{z, p.BH, p.d, p.n_iter, inv_init};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((p.BH + C::kHeads - 1) / C::kHeads);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeLaunchCompletionEvent;
+    attr[0].val.launchCompletionEvent.event = started;
+    attr[0].val.launchCompletionEvent.flags = 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = started != nullptr ? 1 : 0;
+    ProfScope ps(K_PINV, s);
+    if (cudaLaunchKernelEx(&cfg, pinv_res_kernel<MH>, maps, prm) != cudaSuccess) return NYS_ERR_CUDA;
+    return NYS_OK;
+}
+
 // m = 256: kernel_2 and the iterative inverse in one CTA-pair kernel.
 int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, const float* kl, float* z, char* ws,
-                     cudaStream_t s) {
+                     int inv_init, cudaStream_t s, cudaEvent_t started) {
     using C = PinvPair;
     constexpr int M = 256;
     static bool attr_set[kMaxDevices] = {};
@@ -457,7 +568,7 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
         !map_3d(&maps.k2t, f32, 4, k2t, M, M, BH, 32, 128, sw) ||
         !map_3d(&maps.wt, f32, 4, zs, M, M, BH, 32, 128, sw))
         return NYS_ERR_CUDA;
-    PinvPairParams prm{k2, k2t, zs, z, p.d, p.n_iter};
+    PinvPairParams prm{k2, k2t, zs, z, p.d, p.n_iter, inv_init};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.BH * 2);
     cfg.blockDim = dim3(C::kThreads);
@@ -471,10 +582,10 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
     // `started` fires once every CTA pair has begun: kernel_3 V is held back until then, so
     // that its persistent grid takes the SMs the pairs leave instead of splitting SM pairs
     attr[1].id = cudaLaunchAttributeLaunchCompletionEvent;
-    attr[1].val.launchCompletionEvent.event = st.started;
+    attr[1].val.launchCompletionEvent.event = started;
     attr[1].val.launchCompletionEvent.flags = 0;
     cfg.attrs = attr;
-    cfg.numAttrs = 2;
+    cfg.numAttrs = started != nullptr ? 2 : 1;
     ProfScope ps(K_PINV, s);
     if (cudaLaunchKernelEx(&cfg, pinv_pair_kernel, maps, prm) != cudaSuccess) return NYS_ERR_CUDA;
     return NYS_OK;
@@ -483,7 +594,7 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
 template <int D>
 int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, const __nv_bfloat16* k,
                 const __nv_bfloat16* v, const uint8_t* mask, const float* conv_w, __nv_bfloat16* out, char* ws,
-                cudaStream_t s) {
+                int inv_init, cudaStream_t s) {
     using bf = __nv_bfloat16;
     float* ql = reinterpret_cast<float*>(ws + p.off_ql);
     float* kl = reinterpret_cast<float*>(ws + p.off_kl);
@@ -500,10 +611,16 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     const int BH = p.BH, n = p.n, m = p.m;
     int rc = NYS_OK;
     {
-        long long threads = (long long)BH * m * (D / 8);
-        dim3 grid((unsigned)((threads + 255) / 256), 2);
         ProfScope ps(K_LANDMARKS, s);
-        landmarks_kernel<bf><<<grid, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, D, m);
+        constexpr int rows_per_instr = 32 / (D / 8);
+        if ((n / m) % rows_per_instr == 0) {
+            // eight CTAs of eight warps per SM (the register file's limit), striding over the landmarks
+            landmarks_warp_kernel<D><<<8 * st.sm_count, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, m);
+        } else {
+            long long threads = (long long)BH * m * (D / 8);
+            dim3 grid((unsigned)((threads + 255) / 256), 2);
+            landmarks_kernel<bf><<<grid, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, D, m);
+        }
     }
     // kernel_3 V (+ mask bits, + combine) runs on the auxiliary stream, concurrently with the
     // inverse on the caller's stream: the inverse is the longer branch at the supported sizes,
@@ -511,16 +628,37 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     // released by a cross-stream event. At m = 256 the auxiliary stream waits until every
     // CTA pair of the inverse has started (see launch_pinv_pair); otherwise until the
     // landmarks are done.
-    if (m == 256) {
-        rc = launch_pinv_pair(p, st, ql, kl, z, ws, s);
+    // one wave of CTA pairs: kernel_3 V waits until every pair has started and takes the SMs they
+    // leave; more pairs than SMs (B*H > SMs / 2): "every pair has started" would only come after a
+    // whole wave of the inverse, so kernel_3 V is released with the landmarks instead and its
+    // persistent grid spans every SM, taking SMs as the inverse's waves free them
+    const bool one_wave = m == 256 && 2 * BH <= st.sm_count;
+    if (m == 256 && one_wave) {
+        rc = launch_pinv_pair(p, st, ql, kl, z, ws, inv_init, s, st.started);
         if (rc != NYS_OK) return rc;
         if (cudaStreamWaitEvent(st.aux, st.started, 0) != cudaSuccess) return NYS_ERR_CUDA;
-    } else {
+    } else if (m == 256) {
         if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
         if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
-        rc = m == 64 ? launch_pinv_tc<64>(p, st, ql, kl, z, ws, s)
-           : m == 128 ? launch_pinv_tc<128>(p, st, ql, kl, z, ws, s) : NYS_ERR_UNSUPPORTED;
+        rc = launch_pinv_pair(p, st, ql, kl, z, ws, inv_init, s, nullptr);
         if (rc != NYS_OK) return rc;
+    } else {
+        // m = 64 / 128: the resident inverse is much shorter than kernel_3 V; kernel_3 V is released
+        // once every inverse CTA has started (one wave) and takes every SM, those of the inverse as
+        // they free up; with more inverse CTAs than SMs it is released with the landmarks
+        const int res_ctas = m == 128 ? BH : (BH + 1) / 2;
+        if (res_ctas <= st.sm_count) {
+            rc = m == 64 ? launch_pinv_res<64>(p, ql, kl, z, inv_init, s, st.started)
+               : m == 128 ? launch_pinv_res<128>(p, ql, kl, z, inv_init, s, st.started) : NYS_ERR_UNSUPPORTED;
+            if (rc != NYS_OK) return rc;
+            if (cudaStreamWaitEvent(st.aux, st.started, 0) != cudaSuccess) return NYS_ERR_CUDA;
+        } else {
+            if (cudaEventRecord(st.fork, s) != cudaSuccess) return NYS_ERR_CUDA;
+            if (cudaStreamWaitEvent(st.aux, st.fork, 0) != cudaSuccess) return NYS_ERR_CUDA;
+            rc = m == 64 ? launch_pinv_res<64>(p, ql, kl, z, inv_init, s, nullptr)
+               : m == 128 ? launch_pinv_res<128>(p, ql, kl, z, inv_init, s, nullptr) : NYS_ERR_UNSUPPORTED;
+            if (rc != NYS_OK) return rc;
+        }
     }
     if (mask) {
         const int words = p.B * (n / 32);
@@ -530,8 +668,10 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     // the inverse runs concurrently on its own SMs (one CTA per SM, one per 128 landmark
     // rows of each head); the persistent kernel_3 V grid takes the rest
     const int pinv_ctas = BH * ((m + 127) / 128);
-    const int k3v_sms = std::max(st.sm_count / 4, st.sm_count - pinv_ctas);
-    rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, k3v_sms, st.aux);
+    // one wave of CTA pairs at m = 256 (as long as kernel_3 V): the SMs the pairs leave; otherwise
+    // (several waves, or the short resident inverse at m <= 128) every SM
+    const int k3v_sms = m == 256 && one_wave ? std::max(st.sm_count / 4, st.sm_count - pinv_ctas) : st.sm_count;
+    rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, k3v_sms, split_scale(D) * kLog2e, st.aux);
     if (rc != NYS_OK) return rc;
     {
         const long long threads = (long long)BH * m * (D / 4);
@@ -542,8 +682,18 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
     if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;
     {
+        static bool attr_set[kMaxDevices] = {};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (!attr_set[dev]) {
+            if (cudaFuncSetAttribute(w_tile_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)WTile<D>::bytes(256)) != cudaSuccess)
+                return NYS_ERR_CUDA;
+            attr_set[dev] = true;
+        }
         ProfScope ps(K_W, s);
-        w_kernel<D><<<dim3(BH, (m + 63) / 64), 256, 0, s>>>(z, k3v, w, wt16, m);
+        w_tile_kernel<D><<<dim3(m / WTile<D>::kRows, BH), WTile<D>::kThreads, WTile<D>::bytes(m), s>>>(
+            z, k3v, w, wt16, m);
     }
     switch (m) {
         case 64: rc = launch_output_tc<D, 64>(p, st, q, v, conv_w, out, kl16, wt16, s); break;
@@ -555,14 +705,107 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
 }
 
+// Exact branch (walkthrough 2.1, path A): softmax(Qs Ks^T + mask) V over all n query rows on
+// the kernel_3 V machinery (tensor cores for bf16, CUDA cores for float32), then the split
+// merge, normalisation and conv; optionally the n x n weights.
+template <typename T, int D>
+int launch_exact(const Plan& p, const DeviceState& st, const T* q, const T* k, const T* v,
+                 const uint8_t* mask, const float* conv_w, T* out, float* attn_probs, char* ws, cudaStream_t s) {
+    float* po = reinterpret_cast<float*>(ws + p.off_po);
+    float* pm = reinterpret_cast<float*>(ws + p.off_pm);
+    float* pl = reinterpret_cast<float*>(ws + p.off_pl);
+    const int BH = p.BH, n = p.n;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+        uint32_t* mbits = mask ? reinterpret_cast<uint32_t*>(ws + p.off_mbits) : nullptr;
+        if (mask) {
+            const int words = p.B * (n / 32);
+            ProfScope ps(K_MASKBITS, s);
+            mask_bits_kernel<<<(words + 255) / 256, 256, 0, s>>>(mask, mbits, p.B, n);
+        }
+        const float sc = split_scale(D) * split_scale(D) * kLog2e;   // Q and K both raw
+        const int rc = launch_k3v_tc<D>(p, st, q, k, v, mbits, po, pm, pl, st.sm_count, sc, s);
+        if (rc != NYS_OK) return rc;
+    } else {
+        dim3 grid(BH, (n + 63) / 64, p.splits);
+        ProfScope ps(K_K3V, s);
+        k3v_partial_simt_kernel<T, D><<<grid, 256, k3v_simt_smem_bytes<D>(), s>>>(
+            q, k, v, mask, po, pm, pl, p.H, n, n, p.splits, p.keys_per_split, split_scale(D));
+    }
+    {
+        ProfScope ps(K_OUTPUT, s);
+        exact_finish_kernel<T, D><<<dim3((n + 63) / 64, BH), 256, 0, s>>>(po, pm, pl, v, conv_w, out, p.H, n,
+                                                                          p.splits);
+    }
+    if (attn_probs) {
+        ProfScope ps(K_PROBS, s);
+        exact_probs_kernel<T, D><<<dim3((n + 63) / 64, BH), 256, 0, s>>>(q, k, mask, attn_probs, p.H, n);
+    }
+    return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
+
+// kernel_1 Z (walkthrough 2.7) from the call's float32 K_l and Z, after the forward.
+template <typename T, int D>
+int launch_nystrom_probs(const Plan& p, const T* q, float* attn_probs, char* ws, cudaStream_t s) {
+    const float* kl = reinterpret_cast<const float*>(ws + p.off_kl);
+    const float* z = reinterpret_cast<const float*>(ws + p.off_z);
+    const size_t smem = ProbsSmem<D>::bytes(p.m);
+    static bool attr_set[kMaxDevices] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(nystrom_probs_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)ProbsSmem<D>::bytes(256)) != cudaSuccess)
+            return NYS_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    ProfScope ps(K_PROBS, s);
+    nystrom_probs_kernel<T, D><<<dim3((p.n + 63) / 64, p.BH), 256, smem, s>>>(q, kl, z, attn_probs, p.n, p.m);
+    return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
+
+int run_exact(const void* q, const void* k, const void* v, const uint8_t* mask, const float* conv_w,
+              int B, int H, int n, int d, int dtype, void* out, float* attn_probs, cudaStream_t s) {
+    int rc = validate_exact(q, k, v, out, B, H, n, d, dtype);
+    if (rc != NYS_OK) return rc;
+    DeviceState* st = nullptr;
+    rc = device_state(&st);
+    if (rc != NYS_OK) return rc;
+    cudaGetLastError();   // an earlier, unrelated launch error is not this call's
+    const Plan p = make_plan_exact(B, H, n, d, dtype);
+    void* ws = nullptr;
+    if (cudaMallocAsync(&ws, p.total, s) != cudaSuccess) {
+        cudaGetLastError();
+        return NYS_ERR_NOMEM;
+    }
+    char* w = static_cast<char*>(ws);
+    std::unique_lock<std::mutex> launch_lock(st->launch_mu);
+    using bf = __nv_bfloat16;
+    if (dtype == NYS_F32)
+        rc = d == 64 ? launch_exact<float, 64>(p, *st, (const float*)q, (const float*)k, (const float*)v, mask,
+                                               conv_w, (float*)out, attn_probs, w, s)
+                     : launch_exact<float, 32>(p, *st, (const float*)q, (const float*)k, (const float*)v, mask,
+                                               conv_w, (float*)out, attn_probs, w, s);
+    else
+        rc = d == 64 ? launch_exact<bf, 64>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask, conv_w,
+                                            (bf*)out, attn_probs, w, s)
+                     : launch_exact<bf, 32>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask, conv_w,
+                                            (bf*)out, attn_probs, w, s);
+    if (cudaFreeAsync(ws, s) != cudaSuccess && rc == NYS_OK) rc = NYS_ERR_CUDA;
+    return rc;
+}
+
 int run(const void* q, const void* k, const void* v, const uint8_t* mask, const float* conv_w,
         int B, int H, int n, int d, int m, int n_iter, int dtype, void* out, float* dbg_ql,
-        float* dbg_kl, float* dbg_z, float* dbg_k3v, float* dbg_w, cudaStream_t s) {
+        float* dbg_kl, float* dbg_z, float* dbg_k3v, float* dbg_w, cudaStream_t s,
+        const Options& opt = Options()) {
+    if (opt.exact) return run_exact(q, k, v, mask, conv_w, B, H, n, d, dtype, out, opt.attn_probs, s);
+    if (opt.inv_init != NYS_INV_INIT_DEFAULT && opt.inv_init != NYS_INV_INIT_EXACT) return NYS_ERR_INVALID_ARG;
     int rc = validate(q, k, v, out, B, H, n, d, m, n_iter, dtype);
     if (rc != NYS_OK) return rc;
     DeviceState* st = nullptr;
     rc = device_state(&st);
     if (rc != NYS_OK) return rc;
+    cudaGetLastError();   // an earlier, unrelated launch error is not this call's
     const Plan p = make_plan(B, H, n, d, m, n_iter, dtype, st->sm_count);
     void* ws = nullptr;
     if (cudaMallocAsync(&ws, p.total, s) != cudaSuccess) {
@@ -571,17 +814,25 @@ int run(const void* q, const void* k, const void* v, const uint8_t* mask, const 
     }
     char* w = static_cast<char*>(ws);
     std::unique_lock<std::mutex> launch_lock(st->launch_mu);
+    using bf = __nv_bfloat16;
     if (dtype == NYS_F32) {
         rc = d == 64 ? launch_simt<float, 64>(p, *st, (const float*)q, (const float*)k, (const float*)v,
-                                              mask, conv_w, (float*)out, w, s)
+                                              mask, conv_w, (float*)out, w, opt.inv_init, s)
                      : launch_simt<float, 32>(p, *st, (const float*)q, (const float*)k, (const float*)v,
-                                              mask, conv_w, (float*)out, w, s);
+                                              mask, conv_w, (float*)out, w, opt.inv_init, s);
     } else {
-        using bf = __nv_bfloat16;
         rc = d == 64 ? launch_bf16<64>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask, conv_w,
-                                       (bf*)out, w, s)
+                                       (bf*)out, w, opt.inv_init, s)
                      : launch_bf16<32>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask, conv_w,
-                                       (bf*)out, w, s);
+                                       (bf*)out, w, opt.inv_init, s);
+    }
+    if (rc == NYS_OK && opt.attn_probs) {
+        if (dtype == NYS_F32)
+            rc = d == 64 ? launch_nystrom_probs<float, 64>(p, (const float*)q, opt.attn_probs, w, s)
+                         : launch_nystrom_probs<float, 32>(p, (const float*)q, opt.attn_probs, w, s);
+        else
+            rc = d == 64 ? launch_nystrom_probs<bf, 64>(p, (const bf*)q, opt.attn_probs, w, s)
+                         : launch_nystrom_probs<bf, 32>(p, (const bf*)q, opt.attn_probs, w, s);
     }
     if (rc == NYS_OK) {
         const size_t BH = p.BH, md = (size_t)m * d, mm = (size_t)m * m;
@@ -604,25 +855,54 @@ int run(const void* q, const void* k, const void* v, const uint8_t* mask, const 
 // the array until the process exits. In host code the name below is only a
 // host-side stand-in: its device address comes from cudaGetSymbolAddress().
 constexpr size_t kStaticScratchFloats = (8u << 20) / sizeof(float);
+constexpr int kStaticMaxM = 256;   // the largest m any entry point accepts
+static_assert((size_t)5 * kStaticMaxM * kStaticMaxM <= kStaticScratchFloats,
+              "one head of the largest supported m must fit the static scratch");
 static __device__ __align__(256) float g_static_scratch[kStaticScratchFloats];
 
-std::mutex g_static_mu;
-float* g_static_ptr[kMaxDevices];   // device address of g_static_scratch, per device
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+    static CtxGetCurrentFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
 
-// Once per device, with that device current: look up the array's address.
+std::mutex g_static_mu;
+// device address of g_static_scratch per device, with the context it was looked up in: a
+// device reset (or any teardown of the context) reloads the module, so the address is looked
+// up again when the current context is not the one recorded
+struct StaticScratchAddr { CUcontext ctx = nullptr; float* ptr = nullptr; };
+StaticScratchAddr g_static_addr[kMaxDevices];
+
+// Once per device (and context), with that device current: look up the array's address.
 int static_scratch(float** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return NYS_ERR_CUDA;
+    CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+    if (!get_ctx) return NYS_ERR_CUDA;
+    CUcontext ctx = nullptr;   // null before the runtime has made its context current
+    if (get_ctx(&ctx) != CUDA_SUCCESS) return NYS_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (g_static_ptr[dev] == nullptr) {
+    StaticScratchAddr& a = g_static_addr[dev];
+    if (a.ptr == nullptr || ctx == nullptr || a.ctx != ctx) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) {
             cudaGetLastError();
             return NYS_ERR_CUDA;
         }
-        g_static_ptr[dev] = static_cast<float*>(p);
+        if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return NYS_ERR_CUDA;
+        a.ctx = ctx;
+        a.ptr = static_cast<float*>(p);
     }
-    *out = g_static_ptr[dev];
+    *out = a.ptr;
     return NYS_OK;
 }
 
@@ -644,6 +924,17 @@ int nys_attn_forward_debug(const void* q, const void* k, const void* v, const ui
                            float* w, void* stream) {
     return nys::run(q, k, v, key_mask, conv_w, B, H, n, d, m, n_iter, dtype, out, q_l, k_l, z, k3v,
                     w, static_cast<cudaStream_t>(stream));
+}
+
+int nys_attn_forward_ex(const void* q, const void* k, const void* v, const uint8_t* key_mask,
+                        const float* conv_w, int B, int H, int n, int d, int m, int n_iter, int dtype,
+                        int inv_init, int exact, void* out, float* attn_probs, void* stream) {
+    nys::Options opt;
+    opt.inv_init = inv_init;
+    opt.exact = exact != 0;
+    opt.attn_probs = attn_probs;
+    return nys::run(q, k, v, key_mask, conv_w, B, H, n, d, m, n_iter, dtype, out, nullptr, nullptr,
+                    nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream), opt);
 }
 
 int nys_attn_host_plan(int B, int H, int* chunks, int max_chunks) {
@@ -797,6 +1088,37 @@ __global__ void exp2_selftest_kernel(int n, float lo, float hi, unsigned int* wo
 }
 }  // namespace nys
 
+namespace nys {
+// One CTA waits on an mbarrier that nothing arrives on, with the bounded wait every kernel
+// uses (limit given here instead of the kernels' one second); no copy or MMA is in flight.
+__global__ void wait_timeout_selftest_kernel(uint64_t limit_ns, int* result) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(&bar, 1);
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = sm100::warp_all(sm100::mbar_wait_limit(&bar, 0, limit_ns));
+    if (threadIdx.x == 0) *result = ok ? 1 : 0;
+}
+}  // namespace nys
+
+int nys_attn_selftest_wait_timeout(unsigned long long limit_ns, int* completed) {
+    if (!completed || limit_ns == 0 || limit_ns > 1000000000ull) return NYS_ERR_INVALID_ARG;
+    int* d = nullptr;
+    if (cudaMalloc(&d, sizeof(int)) != cudaSuccess) return NYS_ERR_CUDA;
+    int h = -1, rc = NYS_OK;
+    if (cudaMemset(d, 0xFF, sizeof(int)) != cudaSuccess) rc = NYS_ERR_CUDA;
+    if (rc == NYS_OK) {
+        nys::wait_timeout_selftest_kernel<<<1, 32>>>((uint64_t)limit_ns, d);
+        if (cudaGetLastError() != cudaSuccess || cudaMemcpy(&h, d, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess)
+            rc = NYS_ERR_CUDA;
+    }
+    cudaFree(d);
+    *completed = h;
+    return rc;
+}
+
 int nys_attn_selftest_exp2(float* max_rel_err) {
     if (!max_rel_err) return NYS_ERR_INVALID_ARG;
     unsigned int* d = nullptr;
@@ -818,20 +1140,23 @@ int nys_attn_pinv_static(const float* q_l, const float* k_l, float* z, int BH, i
                          int n_iter, void* stream) {
     if (!q_l || !k_l || !z) return NYS_ERR_INVALID_ARG;
     if (BH <= 0 || m <= 0 || d <= 0 || n_iter < 0) return NYS_ERR_INVALID_ARG;
-    if ((d != 32 && d != 64) || m > 256) return NYS_ERR_UNSUPPORTED;
+    if ((d != 32 && d != 64) || m > nys::kStaticMaxM) return NYS_ERR_UNSUPPORTED;
     const size_t per_head = (size_t)5 * m * m;   // k2, X, T, U and the second Z buffer
-    if (per_head > nys::kStaticScratchFloats) return NYS_ERR_SCRATCH_LIMIT;
+    if (per_head > nys::kStaticScratchFloats) return NYS_ERR_SCRATCH_LIMIT;   // unreachable at m <= 256
     float* scratch = nullptr;
     int rc = nys::static_scratch(&scratch);
     if (rc != NYS_OK) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaGetLastError();   // an earlier, unrelated launch error is not this call's
     const int per_launch = (int)(nys::kStaticScratchFloats / per_head);
     for (int h0 = 0; h0 < BH; h0 += per_launch) {
         const int nh = BH - h0 < per_launch ? BH - h0 : per_launch;
         const size_t md = (size_t)h0 * m * d, mm = (size_t)h0 * m * m;
-        nys::pinv_simt_kernel<<<nh, 256, 0, s>>>(q_l + md, k_l + md, z + mm, scratch, m, d, n_iter);
+        nys::pinv_simt_kernel<<<nh, 256, 0, s>>>(q_l + md, k_l + md, z + mm, scratch, m, d, n_iter,
+                                                 NYS_INV_INIT_DEFAULT);
+        if (cudaGetLastError() != cudaSuccess) return NYS_ERR_CUDA;   // stop at the first failed launch
     }
-    return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+    return NYS_OK;
 }
 
 int nys_attn_profile_enable(int on) {

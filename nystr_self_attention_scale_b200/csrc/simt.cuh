@@ -87,13 +87,14 @@ __device__ void block_gemm(float* __restrict__ C, int ldc, const float* __restri
 
 // ------------------------------------------------------------------ kernel_2 + iterative inverse
 // Walkthrough 2.4 (kernel_2 = softmax(Q_l K_l^T)) and 2.5 (iterative inverse):
-//   Z_0 = c k2^T, c = 1 / (max column sum * max row sum)
+//   Z_0 = c k2^T, c = 1 / (max column sum * max row sum) (or 1 / max column sum with
+//   the exact-coefficient option, walkthrough 2.5 second bullet)
 //   repeat: X = k2 Z; T = 7I - X; U = 15I - X T; T = 13I - X U; Z = Z T / 4
 // One CTA per (batch, head); the m x m matrices live in global scratch
 // (L2-resident), 5 per head: k2, X, T, U, and the second Z buffer.
 __global__ void __launch_bounds__(256)
 pinv_simt_kernel(const float* __restrict__ ql, const float* __restrict__ kl, float* __restrict__ z_out,
-                 float* __restrict__ scratch, int m, int d, int n_iter) {
+                 float* __restrict__ scratch, int m, int d, int n_iter, int inv_init) {
     __shared__ GemmSmem sm;
     __shared__ float red[2][8];
     const int bh = blockIdx.x;
@@ -140,7 +141,8 @@ pinv_simt_kernel(const float* __restrict__ ql, const float* __restrict__ kl, flo
     __syncthreads();
     float c_mc = red[0][0], c_mr = red[1][0];
     for (int w = 1; w < 8; ++w) { c_mc = fmaxf(c_mc, red[0][w]); c_mr = fmaxf(c_mr, red[1][w]); }
-    const float coeff = 1.f / (c_mc * c_mr);
+    // default: 1 / (max column sum * max row sum); exact-coefficient option: 1 / max column sum
+    const float coeff = inv_init == NYS_INV_INIT_EXACT ? 1.f / c_mc : 1.f / (c_mc * c_mr);
     for (size_t e = tid; e < mm; e += 256) {
         size_t r = e / m, c = e % m;
         Z[e] = coeff * A[c * m + r];
@@ -169,11 +171,135 @@ pinv_simt_kernel(const float* __restrict__ ql, const float* __restrict__ kl, flo
     }
 }
 
+// ------------------------------------------------------------------ kernel_2 + inverse, m <= 64
+// The same computation as pinv_simt_kernel with every m x m matrix in shared memory (six
+// 64 x 68 float buffers, 104 KB), for m <= 64: no operand goes through L2 between products.
+// Each product C = alpha (L R) + diag I is computed by the 256 threads in 4 x 4 blocks
+// (rows 4 ty .., columns 4 tx ..), the left factor read as scalars (the two row groups of a
+// warp fall in different banks), the right factor as 16-byte rows; entries outside m x m stay
+// zero, so the padding never contributes.
+constexpr int kPinvSmemLd = 68;
+constexpr size_t kPinvSmemBytes = sizeof(float) * 6 * 64 * kPinvSmemLd;
+
+__device__ __forceinline__ void smem_gemm64(float* __restrict__ C, const float* __restrict__ Lm,
+                                            const float* __restrict__ Rm, int inner, int m, float alpha,
+                                            float diag) {
+    constexpr int LD = kPinvSmemLd;
+    const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+    float acc[4][4] = {};
+#pragma unroll 4
+    for (int k = 0; k < inner; ++k) {
+        const float4 b = *reinterpret_cast<const float4*>(Rm + k * LD + 4 * tx);
+        const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float a = Lm[(4 * ty + i) * LD + k];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a, bv[j], acc[i][j]);
+        }
+    }
+    __syncthreads();   // every thread has read its operands before any result is stored
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = 4 * ty + i;
+        float4 o;
+        float* ov = reinterpret_cast<float*>(&o);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = 4 * tx + j;
+            ov[j] = (r < m && c < m) ? alpha * acc[i][j] + (r == c ? diag : 0.f) : 0.f;
+        }
+        *reinterpret_cast<float4*>(C + r * LD + 4 * tx) = o;
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(256)
+pinv_simt_smem_kernel(const float* __restrict__ ql, const float* __restrict__ kl, float* __restrict__ z_out,
+                      int m, int d, int n_iter, int inv_init) {
+    constexpr int LD = kPinvSmemLd;
+    extern __shared__ __align__(16) float psm[];
+    float* A = psm;                 // k2
+    float* Zc = A + 64 * LD;        // Z (current)
+    float* Zn = Zc + 64 * LD;       // Z (next)
+    float* X = Zn + 64 * LD;
+    float* T = X + 64 * LD;
+    float* U = T + 64 * LD;
+    __shared__ float red[2][8];
+    const int bh = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // landmarks: Q_l rows into X ([r][k]), K_l transposed into T ([k][c]), zero-padded to 64 x 64
+    for (int e = tid; e < 64 * 64; e += 256) {
+        const int r = e >> 6, c = e & 63;
+        X[r * LD + c] = (r < m && c < d) ? ql[((size_t)bh * m + r) * d + c] : 0.f;
+        T[c * LD + r] = (r < m && c < d) ? kl[((size_t)bh * m + r) * d + c] : 0.f;
+    }
+    __syncthreads();
+    smem_gemm64(A, X, T, d, m, 1.f, 0.f);    // S2 = Q_l K_l^T (sum over the d columns)
+    // walkthrough 2.4: k2 = softmax_row(S2), one warp per row
+    for (int r = warp; r < m; r += 8) {
+        float* row = A + r * LD;
+        float mx = -INFINITY;
+        for (int c = lane; c < m; c += 32) mx = fmaxf(mx, row[c]);
+        mx = warp_max(mx);
+        float sum = 0.f;
+        for (int c = lane; c < m; c += 32) {
+            const float e = __expf(row[c] - mx);
+            row[c] = e;
+            sum += e;
+        }
+        sum = warp_sum(sum);
+        const float inv = 1.f / sum;
+        for (int c = lane; c < m; c += 32) row[c] *= inv;
+    }
+    __syncthreads();
+    // walkthrough 2.5: c = 1 / (max column sum * max row sum), or 1 / max column sum (exact option)
+    float mcol = -INFINITY, mrow = -INFINITY;
+    if (tid < m) {
+        float cs = 0.f, rs = 0.f;
+        for (int j = 0; j < m; ++j) {
+            cs += A[j * LD + tid];
+            rs += A[tid * LD + j];
+        }
+        mcol = cs;
+        mrow = rs;
+    }
+    mcol = warp_max(mcol);
+    mrow = warp_max(mrow);
+    if (lane == 0) { red[0][warp] = mcol; red[1][warp] = mrow; }
+    __syncthreads();
+    float c_mc = red[0][0], c_mr = red[1][0];
+    for (int w = 1; w < 8; ++w) { c_mc = fmaxf(c_mc, red[0][w]); c_mr = fmaxf(c_mr, red[1][w]); }
+    const float coeff = inv_init == NYS_INV_INIT_EXACT ? 1.f / c_mc : 1.f / (c_mc * c_mr);
+    for (int e = tid; e < 64 * 64; e += 256) {
+        const int r = e >> 6, c = e & 63;
+        Zc[r * LD + c] = (r < m && c < m) ? coeff * A[c * LD + r] : 0.f;   // Z_0 = c k2^T
+    }
+    __syncthreads();
+    for (int it = 0; it < n_iter; ++it) {
+        smem_gemm64(X, A, Zc, m, m, 1.f, 0.f);     // X = A Z
+        for (int e = tid; e < 64 * 64; e += 256) {
+            const int r = e >> 6, c = e & 63;
+            T[r * LD + c] = (r < m && c < m) ? (r == c ? 7.f : 0.f) - X[r * LD + c] : 0.f;   // T = 7I - X
+        }
+        __syncthreads();
+        smem_gemm64(U, X, T, m, m, -1.f, 15.f);    // U = 15I - X T
+        smem_gemm64(T, X, U, m, m, -1.f, 13.f);    // T = 13I - X U
+        smem_gemm64(Zn, Zc, T, m, m, 0.25f, 0.f);  // Z = Z T / 4
+        float* t = Zc; Zc = Zn; Zn = t;
+    }
+    float* Z = z_out + (size_t)bh * m * m;
+    for (int e = tid; e < m * m; e += 256) Z[e] = Zc[(e / m) * LD + (e % m)];
+}
+
 // ------------------------------------------------------------------ kernel_3 V, split over keys
 // Walkthrough 2.4: k3 = softmax_row(Q_l Ks^T + mask), new_value = k3 V.
 // CTA (bh, 64-landmark block, key split) runs an online softmax over its key
 // range in 64-key chunks and writes unnormalised partials: O (64 x D), the
-// running max M and the running sum l per landmark row.
+// running max M and the running sum l per landmark row. The rows are scaled by
+// q_scale on load: 1 for the landmarks (already scaled by d^-1/4), d^-1/4 when
+// the rows are the raw queries of the exact branch (walkthrough 2.1, path A),
+// which runs the same online softmax over all n query rows.
 template <int D>
 constexpr size_t k3v_simt_smem_bytes() { return sizeof(float) * (2 * D * 68 + 64 * (D + 4) + 64 * 68); }
 
@@ -182,7 +308,7 @@ __global__ void __launch_bounds__(256)
 k3v_partial_simt_kernel(const float* __restrict__ ql, const T* __restrict__ k, const T* __restrict__ v,
                         const uint8_t* __restrict__ mask, float* __restrict__ part_o,
                         float* __restrict__ part_m, float* __restrict__ part_l, int H, int n, int m,
-                        int splits, int keys_per_split) {
+                        int splits, int keys_per_split, float q_scale) {
     constexpr int CW = D / 16;  // output columns per thread
     extern __shared__ float smem[];
     float (*sQ)[68] = reinterpret_cast<float (*)[68]>(smem);                  // [D][68]
@@ -196,7 +322,7 @@ k3v_partial_simt_kernel(const float* __restrict__ ql, const T* __restrict__ k, c
     const float s = split_scale(D);
     for (int e = tid; e < 64 * D; e += 256) {
         int r = e / D, c = e % D;
-        sQ[c][r] = (j0 + r < m) ? ql[((size_t)bh * m + j0 + r) * D + c] : 0.f;
+        sQ[c][r] = (j0 + r < m) ? q_scale * ql[((size_t)bh * m + j0 + r) * D + c] : 0.f;
     }
     float o[4][CW], mrun[4], lrun[4];
 #pragma unroll
@@ -439,6 +565,105 @@ w_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __re
             pk.y = *reinterpret_cast<uint32_t*>(&hi);
             *reinterpret_cast<uint2*>(wt16 + ((size_t)bh * D + c) * m + r0 + ty * 4) = pk;
         }
+    }
+}
+
+// W = Z (k3 V) for the bf16 path (m a multiple of 32): one CTA of 128 threads per 32-row
+// tile of one head, so that the 256 tiles of the headline shape spread over every SM. The
+// tile's 32 Z rows (contiguous in memory) and the head's whole k3 V are staged in shared
+// memory with 16-byte asynchronous copies, all in flight at once; then each thread
+// accumulates a 4 x 4 block over all m in float32, reading four Z values of one row and four
+// k3 V values of one k as 16-byte shared loads. Writes W (float32) and W^T (bf16, [d, m] per
+// head, through a shared-memory transpose so that the stores are coalesced).
+template <int D>
+struct WTile {
+    static constexpr int kRows = 32, kThreads = 128;
+    static constexpr size_t bytes(int m) {   // sZ [32][m + 4] + sK [m][D] + sW [D][36]
+        return sizeof(float) * ((size_t)32 * (m + 4) + (size_t)m * D + (size_t)D * 36);
+    }
+};
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void sm100_griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(128)
+w_tile_kernel(const float* __restrict__ z, const float* __restrict__ k3v, float* __restrict__ w,
+              __nv_bfloat16* __restrict__ wt16, int m) {
+    constexpr int CG = D / 4;                         // column groups of 4
+    constexpr int RG = 128 / CG;                      // row groups (4 rows each): 8 (D=64) or 16 (D=32)
+    static_assert(RG * 4 >= WTile<D>::kRows, "tile rows");
+    extern __shared__ __align__(16) float wsm[];
+    const int ldz = m + 4;                                                  // padded row: 4 rows hit 4 bank groups
+    float* sZ = wsm;                                                        // [32][m + 4]
+    float* sK = wsm + (size_t)32 * ldz;                                     // [m][D]
+    float (*sW)[36] = reinterpret_cast<float (*)[36]>(sK + (size_t)m * D);  // [D][36]: W^T tile
+    const int bh = blockIdx.y, r0 = blockIdx.x * WTile<D>::kRows;
+    const int tid = threadIdx.x;
+    // the output pass launched after this kernel may start its set-up now; it waits for this
+    // kernel's completion before it reads W^T
+    sm100_griddep_launch_dependents();
+    const float* zb = z + ((size_t)bh * m + r0) * m;
+    const float* kb = k3v + (size_t)bh * m * D;
+    const int zc = m / 4;                             // 16-byte chunks per Z row
+    for (int e = tid; e < 32 * zc; e += 128)
+        cp_async16(sZ + (size_t)(e / zc) * ldz + 4 * (e % zc), zb + 4 * (size_t)e);
+    for (int e = tid; e < m * D / 4; e += 128) cp_async16(sK + 4 * (size_t)e, kb + 4 * (size_t)e);
+    cp_async_wait_all();
+    __syncthreads();
+    const int cg = tid % CG, rg = tid / CG;           // columns 4 cg .. 4 cg + 3, rows 4 rg .. 4 rg + 3
+    if (4 * rg < WTile<D>::kRows) {
+        float acc[4][4] = {};
+        const float* zr = sZ + (size_t)(4 * rg) * ldz;
+#pragma unroll 2
+        for (int k = 0; k < m; k += 4) {
+            float4 a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(zr + (size_t)i * ldz + k);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = *reinterpret_cast<const float4*>(sK + (size_t)(k + j) * D + 4 * cg);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float ai[4] = {a[i].x, a[i].y, a[i].z, a[i].w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[i][0] = fmaf(ai[j], b[j].x, acc[i][0]);
+                    acc[i][1] = fmaf(ai[j], b[j].y, acc[i][1]);
+                    acc[i][2] = fmaf(ai[j], b[j].z, acc[i][2]);
+                    acc[i][3] = fmaf(ai[j], b[j].w, acc[i][3]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int r = 4 * rg + i;
+            *reinterpret_cast<float4*>(w + ((size_t)bh * m + r0 + r) * D + 4 * cg) =
+                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sW[4 * cg + j][r] = acc[i][j];
+        }
+    }
+    if (wt16 == nullptr) return;
+    __syncthreads();
+    // W^T tile: D rows of 32 bf16 (64 bytes) each, written as 16-byte chunks
+    for (int e = tid; e < D * 4; e += 128) {
+        const int c = e / 4, q = e % 4;               // column c of W, rows 8 q .. 8 q + 7 of the tile
+        uint32_t pk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(sW[c][8 * q + 2 * j], sW[c][8 * q + 2 * j + 1]);
+            pk[j] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(wt16 + ((size_t)bh * D + c) * m + r0 + 8 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
 }
 

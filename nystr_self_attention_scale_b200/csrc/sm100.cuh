@@ -51,19 +51,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Waits for the completion of the phase with parity `parity`. Bounded.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Waits for the completion of the phase with parity `parity`, for at most `limit_ns` of
+// global time; a wait that runs out records NYS_ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             record_status(NYS_ERR_TIMEOUT);
             return false;
         }
     }
+}
+// The kernels' wait: bounded by kWaitLimitNs.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    return mbar_wait_limit(bar, parity, kWaitLimitNs);
 }
 
 // Warp-uniform and group-uniform decisions, so that warp-collective tcgen05
@@ -92,6 +97,15 @@ __device__ __forceinline__ bool group_any(bool v, int bar_id, int nthreads) {
     return r != 0;
 }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the kernel before
+// it in the stream is still running; it must wait (griddep_wait) before reading anything that
+// kernel writes. The earlier kernel lets it start by triggering (griddep_launch_dependents).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(m) : "memory");
@@ -101,6 +115,27 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
     asm volatile(
         "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
         ::"r"(smem_u32(dst)), "l"(m), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+// L2 eviction-priority policies for cache hints (createpolicy): data read once and streamed
+// (evict first) and data read again soon (evict last).
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+// tma_load_3d with an L2 cache-policy hint.
+__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1,
+                                                 int c2, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+        ::"r"(smem_u32(dst)), "l"(m), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
         : "memory");
 }
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int c0, int c1, int c2) {
@@ -227,8 +262,18 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // ---------------------------------------------------------------- descriptors
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading and
 // stride byte offsets (16-byte units), version 1, swizzle/layout code
-// (0 none, 2 = 128-byte swizzle, 4 = 64-byte, 6 = 32-byte).
-enum : uint32_t { kLayoutNone = 0, kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6 };
+// (0 none, 2 = 128-byte swizzle, 4 = 64-byte, 6 = 32-byte, 1 = 128-byte swizzle of
+// 32-byte granules, the one layout an MN-major tf32 operand can take).
+enum : uint32_t { kLayoutNone = 0, kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6, kLayoutSw128B32 = 1 };
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside an MN-major tf32 operand
+// atom of the 32-byte-granule 128-byte swizzle: rows (K) of 128 bytes (32 tf32 along MN),
+// 4 rows per 512-byte atom, the 32-byte granule index XORed with row % 4. Atoms of 4 rows sit
+// 512 bytes apart here, so an 8-row K group is 1 KB (one MMA K step reads two atoms: SBO 512).
+__device__ __forceinline__ uint32_t mn32_chunk(int row, int chunk) {
+    return (uint32_t)(row & 7) * 128u + ((((uint32_t)chunk >> 1) ^ ((uint32_t)row & 3u)) << 5) +
+           (((uint32_t)chunk & 1u) << 4);
+}
 
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
                                               uint32_t layout) {

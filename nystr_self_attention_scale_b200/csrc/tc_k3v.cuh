@@ -1,7 +1,9 @@
 // tc_k3v.cuh -- bf16 kernel_3 V pass on the 5th-generation tensor cores.
 //
 // Walkthrough (blog.gitcode.com) 2.4: k3 = softmax_row(Q_l Ks^T + mask), new_value = k3 V.
-// A work item is (batch*head, 128-landmark block, key split). For each
+// The same kernel runs the exact branch (walkthrough 2.1, path A) with the raw queries
+// as its rows: softmax_row(Qs Ks^T + mask) V over all n query rows.
+// A work item is (batch*head, 128-row block, key split). For each
 // 128-key chunk of the split:
 //   S = Q_l_block . K_chunk^T          tcgen05 bf16 MMA into TMEM (K unscaled;
 //                                      the d^-1/4 of K is applied in the exponent)
@@ -77,6 +79,8 @@ struct K3vTcParams {
     float* part_m;         // [BH, splits, m]  running max (natural-log units)
     float* part_l;         // [BH, splits, m]  running sum
     int H, n, m, halves, splits, chunks_per_split, total_items;
+    float score_scale;     // exponent scale of the raw S (log2 units): d^-1/4 log2(e) for the
+                           // landmark rows (K's share of the scaling), d^-1/2 log2(e) for raw queries
 };
 
 template <int D>
@@ -146,6 +150,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
 
     if (warp == 0) {
         if (lane == 0) {
+            const uint64_t stream_policy = l2_policy_evict_first();
             int g = 0, it = 0;
             int last_stage_use[C::kStages];
             for (int s = 0; s < C::kStages; ++s) last_stage_use[s] = -1;
@@ -163,8 +168,10 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                     if (!mbar_wait(&kv_empty[st], ((g / C::kStages) & 1) ^ 1)) { *abort_flag = 1; break; }
                     mbar_arrive_expect_tx(&kv_full[st], 2 * C::kTileBytes);
                     const int key0 = (c0 + c) * C::kChunk;
-                    tma_load_3d(sm + C::kOffK + st * C::kTileBytes, &map_k, &kv_full[st], 0, key0, bh);
-                    tma_load_3d(sm + C::kOffV + st * C::kTileBytes, &map_v, &kv_full[st], 0, key0, bh);
+                    // K and V stream through once: evict them first, so that they do not push
+                    // the inverse's operands (re-read every iteration, on other SMs) out of L2
+                    tma_load_3d_hint(sm + C::kOffK + st * C::kTileBytes, &map_k, &kv_full[st], 0, key0, bh, stream_policy);
+                    tma_load_3d_hint(sm + C::kOffV + st * C::kTileBytes, &map_v, &kv_full[st], 0, key0, bh, stream_policy);
                     last_stage_use[st] = g / C::kStages;
                 }
             }
@@ -256,7 +263,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-        const float sc = split_scale(D) * kLog2e;   // exponent scale of the raw S = Q_l . K^T
+        const float sc = prm.score_scale;           // exponent scale of the raw S = Q_rows . K^T
         constexpr float kSlack = 8.f;               // log2 units: P stays below 2^8
         constexpr int kT = C::kTeamThreads;
         const int bar_id = 1 + t;                   // this stream's named barrier

@@ -160,6 +160,11 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     if (i > 0) {
                         if (!mbar_wait(const_empty, ce_phase)) { *abort_flag = 1; break; }
                         ce_phase ^= 1;
+                    } else {
+                        // W^T comes from the kernel launched just before this one, and this kernel
+                        // may start before that one ends (programmatic dependent launch): the set-up,
+                        // the Toeplitz build and the V loads go ahead, the constants wait here
+                        griddep_wait();
                     }
                     mbar_arrive_expect_tx(const_full, C::kKlBytes + C::kWtLoadBytes);
                     tma_load_3d(sm + C::kOffKl, &map_kl, const_full, 0, 0, bh);

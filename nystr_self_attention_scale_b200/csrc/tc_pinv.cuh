@@ -234,6 +234,7 @@ struct PinvTcParams {
     const float* rowsum;       // [BH][m]
     float* z_out;              // [BH][m][m] row-major
     int n_iter;
+    int inv_init;              // NYS_INV_INIT_DEFAULT or NYS_INV_INIT_EXACT
 };
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -293,7 +294,8 @@ __global__ void __launch_bounds__(128, 1) pinv_tc_kernel(const PinvTcParams prm)
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
-    // c = 1 / (max column sum * max row sum) of this head's kernel_2
+    // c = 1 / (max column sum * max row sum) of this head's kernel_2 (default), or
+    // 1 / max column sum (the exact-coefficient option)
     float mc = -INFINITY, mr = -INFINITY;
     for (int c = tid; c < M; c += 128) {
         float s = 0.f;
@@ -310,8 +312,11 @@ __global__ void __launch_bounds__(128, 1) pinv_tc_kernel(const PinvTcParams prm)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // the exact-coefficient option drops the row factor (the row sums of a softmax are 1)
     const float coeff = 1.f / (fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3])) *
-                               fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7])));
+                               (prm.inv_init == NYS_INV_INIT_EXACT
+                                    ? 1.f
+                                    : fmaxf(fmaxf(red[4], red[5]), fmaxf(red[6], red[7]))));
     const uint32_t tmem = *tmem_slot;
     const uint32_t tX = tmem, tOut = tmem + M;      // accumulator regions (columns)
     const uint32_t lane_base = (uint32_t)(32 * warp) << 16;

@@ -118,13 +118,13 @@ __device__ __forceinline__ void commit2(uint64_t* bar, uint16_t mask) {
         : "memory");
 }
 // TMA tile load into this CTA's shared memory whose completion is counted on the
-// barrier at `bar_cluster_addr` (the pair's first CTA).
+// barrier at `bar_cluster_addr` (the pair's first CTA), with an L2 cache-policy hint.
 __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster_addr,
-                                                 int c0, int c1, int c2) {
+                                                 int c0, int c1, int c2, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];"
-        ::"r"(sm100::smem_u32(dst)), "l"(m), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2)
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%3, %4, %5}], [%2], %6;"
+        ::"r"(sm100::smem_u32(dst)), "l"(m), "r"(bar_cluster_addr), "r"(c0), "r"(c1), "r"(c2), "l"(policy)
         : "memory");
 }
 
@@ -144,6 +144,7 @@ struct PinvPairParams {
     float* wt;         // [BH][256][256] W^T scratch (row g = column g of W)
     float* z_out;      // [BH][256][256]
     int d, n_iter;
+    int inv_init;      // NYS_INV_INIT_DEFAULT or NYS_INV_INIT_EXACT
 };
 
 struct PinvPair {
@@ -244,6 +245,8 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 tma_load_3d(bbuf + C::kOffBhi + a * C::kAtomBytes, &maps.kl, pro_full, 32 * a, r0, bh);
             }
             const uint32_t bfull0 = mapa(smem_u32(bfull), 0);
+            // k2 and W^T are streamed in again every iteration: keep them in L2
+            const uint64_t keep_policy = l2_policy_evict_last();
             bool ok = true;
             for (int it = 0; it < n_iter && ok; ++it) {
                 for (int part = 0; part < 2 && ok; ++part) {
@@ -263,7 +266,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                         ok = mbar_wait(&bfree[kc], p == 3 ? 0u : 1u);
                         if (!ok) break;
                         if (leader) mbar_arrive_expect_tx(&bfull[kc], 2 * C::kAtomBytes);
-                        tma_load_3d_pair(bbuf + kc * C::kAtomBytes, mp, bfull0 + 8 * kc, 32 * kc, r0, bh);
+                        tma_load_3d_pair(bbuf + kc * C::kAtomBytes, mp, bfull0 + 8 * kc, 32 * kc, r0, bh, keep_policy);
                     }
                 }
             }
@@ -507,7 +510,8 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 float mc = wmax[0];
 #pragma unroll
                 for (int w = 1; w < 8; ++w) mc = fmaxf(mc, wmax[w]);
-                coeff = 1.f / (mc * fmaxf(rmax[0], rmax[1]));
+                // the exact-coefficient option drops the row factor (softmax rows sum to 1)
+                coeff = 1.f / (mc * (prm.inv_init == NYS_INV_INIT_EXACT ? 1.f : fmaxf(rmax[0], rmax[1])));
             }
             if (et == 0) tma_store_wait_all<0>();
             if (n_iter == 0 && !failed) {

@@ -18,3 +18,16 @@ def oracle_mod():
     import oracle
     oracle.build()
     return oracle
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the errors the parity comparisons measured (what, max-abs, rel-F)."""
+    try:
+        from parity import MEASURED
+    except ImportError:
+        return
+    if not MEASURED:
+        return
+    terminalreporter.write_sep("-", "measured errors (max-abs, rel-F)")
+    for what, max_abs, rel_f in MEASURED:
+        terminalreporter.write_line(f"{what}: max-abs {max_abs:.3e}  rel-F {rel_f:.3e}")

@@ -12,6 +12,14 @@ import numpy as np
 
 TOL = {"f32": dict(max_abs=2e-3, rel_f=1e-4), "bf16": dict(max_abs=None, rel_f=2e-2)}
 
+# (what, max-abs, rel-F) of every comparison made in this session, printed at the end of the
+# run (tests/conftest.py), so that a GPU run's log records the measured errors.
+MEASURED = []
+
+
+def note(what, max_abs, rel_f):
+    MEASURED.append((what, float(max_abs), float(rel_f)))
+
 
 def to_device(x, torch):
     dt = torch.float32 if x["dtype"] == "f32" else torch.bfloat16
@@ -63,6 +71,7 @@ def errors(got, ref):
 def assert_close(got, ref, dtype, what=""):
     tol = TOL[dtype]
     max_abs, rel_f = errors(got, ref)
+    note(what, max_abs, rel_f)
     assert np.all(np.isfinite(got)), f"{what}: non-finite output"
     assert rel_f <= tol["rel_f"], f"{what}: rel-F {rel_f:.3e} > {tol['rel_f']:.1e} (max-abs {max_abs:.3e})"
     if tol["max_abs"] is not None:

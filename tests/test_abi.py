@@ -135,3 +135,47 @@ def test_host_plan_covers_every_slice_once(lib):
     assert lib.nys_attn_host_plan(0, 1, buf, 8) == -1
     assert lib.nys_attn_host_plan(1, 1, buf, 7) == -1
     assert lib.nys_attn_host_plan(1, 1, None, 8) == -1
+
+
+def test_pinv_static_binding_rejects_bad_buffers():
+    """pinv_static() checks its buffers before calling the library: a k_l of another dtype,
+    shape or device, or an `out` of the wrong shape, dtype, layout or device, would make the
+    kernel read or write out of bounds (checked here on CPU tensors: no CUDA call is made)."""
+    import torch
+    import nystr_self_attention_scale_b200 as nys
+    check = nys._check_pinv_static_args
+    q = torch.zeros(2, 3, 64, 32)
+    check(q, q.clone(), None)
+    check(q, q.clone(), torch.zeros(2, 3, 64, 64))
+    bad = [
+        (q.double(), q, None),                              # q_l not float32
+        (q[0], q[0], None),                                 # not 4-D
+        (q, q.to(torch.bfloat16), None),                    # k_l dtype
+        (q, torch.zeros(2, 3, 64, 64), None),               # k_l shape
+        (q, q, torch.zeros(2, 3, 64, 32)),                  # out shape
+        (q, q, torch.zeros(2, 3, 64, 64, dtype=torch.float64)),   # out dtype
+        (q, q, torch.zeros(2, 3, 64, 128)[..., ::2]),       # out strided
+        (q, q, torch.zeros(2, 3, 64, 64, device="meta")),   # out on another device
+        (q, q.to("meta"), None),                            # k_l on another device
+    ]
+    for args in bad:
+        with pytest.raises(ValueError):
+            check(*args)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(inv_init=2), -1),                      # neither Z_0 option
+    (dict(inv_init=-1), -1),
+    (dict(exact=1, null=True), -1),
+    (dict(exact=1, d=48), -2),
+    (dict(exact=1, dtype=1, n=192), -2),         # bf16 exact branch: n % 128 == 0
+    (dict(exact=1, B=0), -1),
+    (dict(n=500, m=64), -1),                     # Nystrom path checks as nys_attn_forward
+])
+def test_forward_ex_rejects_before_launch(lib, kw, code):
+    p = None if kw.pop("null", False) else ctypes.c_void_p(16)
+    a = dict(B=1, H=1, n=512, d=64, m=64, n_iter=6, dtype=0, inv_init=0, exact=0)
+    a.update(kw)
+    assert lib.nys_attn_forward_ex(p, p, p, None, None, a["B"], a["H"], a["n"], a["d"], a["m"],
+                                   a["n_iter"], a["dtype"], a["inv_init"], a["exact"], p, None,
+                                   None) == code

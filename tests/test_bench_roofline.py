@@ -79,3 +79,26 @@ def test_pipe_aware_bound_charges_the_inverse_at_tf32():
     assert t > bench.roofline_bound_time(w, PEAKS)[0]          # never below the plain bound here
     wf = WORKLOADS["default_f32_masked"]                       # fp32: both bounds are the same
     assert bench.roofline_bound_time_pipes(wf, PEAKS) == bench.roofline_bound_time(wf, PEAKS)[0]
+
+
+def test_exponential_bound_charges_two_softmaxes_to_the_mufu():
+    """2 B H n m exponentials (kernel_1 and kernel_3) at 16 per clock per SM: about 58 us at
+    the headline shape, just under the pipe-aware bound."""
+    w = WORKLOADS["n16384_bf16_corr"]
+    t, t_exp = bench.roofline_bound_time_exp(w, PEAKS)
+    assert bench.step_exponentials(w) == 2 * 32 * 16384 * 256
+    assert t_exp == pytest.approx(2 * 32 * 16384 * 256 / (148 * 16 * 1965e6), rel=1e-12)
+    assert 57e-6 < t_exp < 58.5e-6
+    assert t == max(t_exp, bench.roofline_bound_time_pipes(w, PEAKS))
+
+
+def test_exact_branch_bound_counts_n_squared_work():
+    """Path A: 4 n^2 d flops per head (Q K^T and P V) plus the conv, n^2 exponentials."""
+    w = WORKLOADS["longcls_bf16_masked"]
+    t, nbytes, flops = bench.roofline_bound_time_exact(w, PEAKS)
+    assert flops == w.BH * (4 * w.n ** 2 * w.d + 2 * 65 * w.n * w.d)
+    assert nbytes == 4 * w.BH * w.n * w.d * 2
+    assert t == max(nbytes / (PEAKS["hbm_gbs"] * 1e9), flops / (PEAKS["bf16_tflops"] * 1e12))
+    assert bench.step_exponentials(w, "exact") == w.BH * w.n * w.n
+    nb, fl, unit = bench.kernel_work(w, "k3v_partial", "exact")
+    assert fl == w.BH * 4 * w.n * w.n * w.d and unit == "tensor"

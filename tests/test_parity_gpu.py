@@ -6,13 +6,19 @@ then recomputes a sample of heads and query rows (the sampled rows of the
 oracle are exact, not approximations: every output row depends on the whole
 head, which the oracle processes in full).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 
-from parity import assert_close, errors, gpu_forward, oracle_heads, sample_rows
+from parity import assert_close, errors, gpu_forward, note, oracle_heads, sample_rows
 from workloads import WORKLOADS, make_inputs
 
 pytestmark = pytest.mark.gpu
+
+# Relative Frobenius bound on Z of the bf16 path (tf32 tensor-core inverse) against the fp64
+# oracle's Z for the same inputs: about twice the measured 7.9e-3 .. 9.3e-3 (m = 128 and 256).
+Z_STAGE_BF16 = 2e-2
 
 torch = pytest.importorskip("torch")
 
@@ -39,8 +45,10 @@ def _full_check(nys, oracle_mod, x, what):
 
 
 def _sampled_check(nys, oracle_mod, x, heads, rows, what):
+    """Selected heads (and rows; None = every row) of a full-size forward against the oracle."""
     out = gpu_forward(x, nys, torch)
-    got = np.stack([out[b, h, rows].double().cpu().numpy() for b, h in heads])
+    sel = slice(None) if rows is None else rows
+    got = np.stack([out[b, h, sel].double().cpu().numpy() for b, h in heads])
     ref = oracle_heads(x, oracle_mod, heads, rows=rows)
     return assert_close(got, ref, x["dtype"], what)
 
@@ -71,11 +79,39 @@ def test_longcls_bf16_masked_small_full(nys, oracle_mod):
     _full_check(nys, oracle_mod, x, "longcls_bf16_masked B=3")
 
 
+def test_longcls_bf16_masked_noconv_full_size_sampled(nys, oracle_mod):
+    """The long-sequence shape without the conv: at m = 128 the conv term is most of the
+    output's norm, so only here is the attention term held to the bf16 bar on its own."""
+    w = dataclasses.replace(WORKLOADS["longcls_bf16_masked"], conv=False)
+    x = make_inputs(w)
+    heads = [(0, 0), (5, 1), (17, 0), (31, 1)]
+    rows = sample_rows(w.n, lengths=[x["lengths"][b] for b, _ in heads])
+    _sampled_check(nys, oracle_mod, x, heads, rows, "longcls_bf16_masked, no conv")
+
+
+def test_longcls_bf16_masked_noconv_small_full(nys, oracle_mod):
+    """The same recipe without the conv at B=3, every row compared."""
+    w = dataclasses.replace(WORKLOADS["longcls_bf16_masked"], conv=False)
+    x = make_inputs(w, seed=1, B=3)
+    _full_check(nys, oracle_mod, x, "longcls_bf16_masked B=3, no conv")
+
+
 def test_n16384_bf16_corr_full_size_sampled(nys, oracle_mod):
+    """Full size, as the benchmark launches it; three heads compared on every row (every
+    128-row tile of the output pass and every key split of kernel_3 V)."""
     w = WORKLOADS["n16384_bf16_corr"]
     x = make_inputs(w)
     heads = [(0, 0), (2, 5), (3, 7)]
-    _sampled_check(nys, oracle_mod, x, heads, sample_rows(w.n), "n16384_bf16_corr")
+    _sampled_check(nys, oracle_mod, x, heads, None, "n16384_bf16_corr")
+
+
+def test_n16384_bf16_corr_bh128_sampled(nys, oracle_mod):
+    """B*H = 128 at m = 256: more CTA pairs of the inverse than one wave of the GPU (kernel_3 V
+    then runs beside the inverse's waves); two heads compared on every row, one of them in the
+    second wave."""
+    w = WORKLOADS["n16384_bf16_corr_bh128"]
+    x = make_inputs(w, seed=4)
+    _sampled_check(nys, oracle_mod, x, [(0, 1), (15, 6)], None, "n16384_bf16_corr B*H=128")
 
 
 def test_n16384_bf16_corr_small_full(nys, oracle_mod):
@@ -90,7 +126,7 @@ def test_sweep_full_size_sampled(nys, oracle_mod, n, conv):
     w = WORKLOADS[f"sweep_n{n}_{'conv' if conv else 'noconv'}"]
     x = make_inputs(w)
     heads = [(0, 0), (7, 7)] if n >= 16384 else [(0, 0), (3, 4), (7, 7)]
-    _sampled_check(nys, oracle_mod, x, heads, sample_rows(n), w.name)
+    _sampled_check(nys, oracle_mod, x, heads, None if n == 65536 else sample_rows(n), w.name)
 
 
 def test_sweep_n1024_full(nys, oracle_mod):
@@ -164,15 +200,18 @@ def test_stages_against_oracle(nys, oracle_mod, name):
     _, ost = oracle_heads(x, oracle_mod, heads, rows=[0], stages=True)
     for idx, (b, h) in enumerate(heads):
         for g, o in (("q_l", "ql"), ("k_l", "kl")):
-            _, rel = errors(st[g][b, h], ost[idx][o])
+            ma, rel = errors(st[g][b, h], ost[idx][o])
+            note(f"stage {g} {name} head {idx}", ma, rel)
             assert rel < 1e-6, (g, rel)
-        _, rel = errors(st["k3v"][b, h], ost[idx]["k3v"])
+        ma, rel = errors(st["k3v"][b, h], ost[idx]["k3v"])
+        note(f"stage k3v {name} head {idx}", ma, rel)
         assert rel < (1e-5 if w.dtype == "f32" else 2e-2), ("k3v", rel)
-        # The bf16 path runs the iterative inverse with tf32 operands; Z itself is
-        # ill-conditioned (its small singular directions carry most of its norm), so its
-        # relative error is ~1e-2 while the output stays within bf16 rounding.
-        _, rel = errors(st["z"][b, h], ost[idx]["z"])
-        assert rel < (1e-4 if w.dtype == "f32" else 5e-2), ("z", rel)
+        # The bf16 path runs the iterative inverse with tf32 operands (the landmarks, and so
+        # kernel_2, come from bf16 inputs but are float32); Z's error is recorded here and
+        # bounded by the Z stage bar of the bf16 path.
+        ma, rel = errors(st["z"][b, h], ost[idx]["z"])
+        note(f"stage z {name} head {idx}", ma, rel)
+        assert rel < (1e-4 if w.dtype == "f32" else Z_STAGE_BF16), ("z", rel)
 
 
 def test_mask_padded_keys_do_not_contribute(nys):
@@ -209,12 +248,13 @@ def test_mask_padded_keys_do_not_contribute(nys):
     ("bf16", 1, 1, 256, 64, 256),   # m = n = 256 on the bf16 path
     ("bf16", 1, 3, 384, 32, 64),    # n = 3 tiles of 128
 ])
-def test_edge_shapes(nys, oracle_mod, dtype, B, H, n, d, m):
+@pytest.mark.parametrize("conv", [True, False])
+def test_edge_shapes(nys, oracle_mod, dtype, B, H, n, d, m, conv):
     w = WORKLOADS["tiny_f32"]
-    import dataclasses
-    w = dataclasses.replace(w, dtype=dtype, d=d, m=m, lengths=(max(1, n // 3), n), zero_pad=True)
+    w = dataclasses.replace(w, dtype=dtype, d=d, m=m, lengths=(max(1, n // 3), n), zero_pad=True,
+                            conv=conv)
     x = make_inputs(w, seed=5, B=B, H=H, n=n)
-    _full_check(nys, oracle_mod, x, f"edge {dtype} B{B} H{H} n{n} d{d} m{m}")
+    _full_check(nys, oracle_mod, x, f"edge {dtype} B{B} H{H} n{n} d{d} m{m} conv{conv}")
 
 
 @pytest.mark.parametrize("d,n_iter,lengths,n", [
@@ -224,18 +264,18 @@ def test_edge_shapes(nys, oracle_mod, dtype, B, H, n, d, m):
     (32, 3, (300, 2048), 2048),    # d = 32, masked, ragged lengths
     (64, 6, (1, 1024), 1024),      # masked, some sequences with a single valid key
 ])
-def test_pair_inverse_variants(nys, oracle_mod, d, n_iter, lengths, n):
+@pytest.mark.parametrize("conv", [True, False])
+def test_pair_inverse_variants(nys, oracle_mod, d, n_iter, lengths, n, conv):
     """m = 256 on the bf16 path: the CTA-pair inverse with kernel_2 in its prologue, over
-    head dimensions, iteration counts and masks the headline workload does not reach."""
-    import dataclasses
+    head dimensions, iteration counts and masks the headline workload does not reach; with
+    the conv off the attention term alone is held to the bf16 bar."""
     w = dataclasses.replace(WORKLOADS["n16384_bf16_corr"], d=d, n_iter=n_iter, lengths=lengths,
-                            zero_pad=lengths is not None)
+                            zero_pad=lengths is not None, conv=conv)
     x = make_inputs(w, seed=13, B=2, H=2, n=n)
-    _full_check(nys, oracle_mod, x, f"pair inverse d{d} n_iter{n_iter} lengths{lengths} n{n}")
+    _full_check(nys, oracle_mod, x, f"pair inverse d{d} n_iter{n_iter} lengths{lengths} n{n} conv{conv}")
 
 
 def test_single_valid_key(nys, oracle_mod):
-    import dataclasses
     w = dataclasses.replace(WORKLOADS["default_f32_masked"], lengths=(1, 1))
     x = make_inputs(w, seed=6, B=2, H=2, n=512)
     _full_check(nys, oracle_mod, x, "one valid key per sequence")
@@ -310,3 +350,24 @@ def test_profile_mask_times_only_selected_kernels(nys):
     finally:
         nys.profile_enable(False)
         nys.profile_mask(None)
+
+
+# ------------------------------------------------------------------ failure detection
+
+def test_bounded_wait_runs_out_and_reports_timeout(nys):
+    """A device-side wait that nothing completes ends after its limit (1 ms here), records
+    NYS_ERR_TIMEOUT in the status word, and leaves the context usable: a forward right
+    after it still matches the oracle's bar and leaves the status clean."""
+    import time
+    assert nys.device_status() == 0
+    t0 = time.perf_counter()
+    completed = nys.selftest_wait_timeout(1_000_000)
+    dt = time.perf_counter() - t0
+    assert completed == 0
+    assert dt >= 1e-3
+    assert nys.device_status() == -5          # NYS_ERR_TIMEOUT, read and cleared
+    assert nys.device_status() == 0
+    x = make_inputs(WORKLOADS["tiny_f32"])
+    out = gpu_forward(x, nys, torch)
+    assert torch.isfinite(out).all()
+    assert nys.device_status() == 0

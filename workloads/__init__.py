@@ -76,6 +76,9 @@ WORKLOADS = {
                                     lengths=(1024, 4096), zero_pad=True),
     "n16384_bf16_corr": Workload("n16384_bf16_corr", "bf16", 4, 8, 16384, 64, 256,
                                  dist="correlated"),
+    # the headline shape at B*H = 128: more CTA pairs of the m = 256 inverse than one wave
+    "n16384_bf16_corr_bh128": Workload("n16384_bf16_corr_bh128", "bf16", 16, 8, 16384, 64, 256,
+                                       dist="correlated"),
     "degenerate_f32_it24": Workload("degenerate_f32_it24", "f32", 1, 1, 256, 64, 256,
                                     n_iter=24, conv=False),
     "degenerate_f32_it6": Workload("degenerate_f32_it6", "f32", 1, 1, 256, 64, 256,
