@@ -69,10 +69,10 @@ def load_peaks():
 # forward's orchestration depends on that whole function
 KERNEL_SOURCES = {
     "landmarks": (["landmarks.cuh"], ["launch_bf16", "launch_simt"]),
-    "pinv": (["tc_pinv_pair.cuh", "tc_pinv.cuh", "sm100.cuh"], ["launch_pinv_pair", "launch_pinv_tc"]),
+    "pinv": (["tc_pinv_pair.cuh", "tc_pinv_res.cuh", "sm100.cuh"], ["launch_pinv_pair", "launch_pinv_res"]),
     "k3v_partial": (["tc_k3v.cuh", "sm100.cuh"], ["launch_k3v_tc"]),
     "k3v_combine": (["simt.cuh"], ["launch_bf16", "launch_simt"]),
-    "w_product": (["simt.cuh"], ["launch_bf16", "launch_simt"]),
+    "w_product": (["simt.cuh", "tc_w.cuh", "sm100.cuh"], ["launch_bf16", "launch_simt"]),
     "output": (["tc_output.cuh", "sm100.cuh"], ["launch_output_tc"]),
 }
 
@@ -136,14 +136,14 @@ def kernel_work(w, kernel, path="nystrom"):
             "alu" if w.dtype == "f32" else "tensor_tf32"
     if kernel == "k3v_partial":
         return 2 * tensor + BH * m * d * 4, BH * 4 * n * m * d, unit
-    if kernel == "kernel2":
-        return BH * (2 * m * d * 4 + 2 * m * m * 4), BH * 2 * m * m * d, "alu"
     if kernel == "mask_bits":
         return w.B * n + w.B * n // 8, 0, "alu"
     if kernel == "k3v_combine":
         return BH * m * d * 8, 0, "alu"
     if kernel == "w_product":
-        return BH * (m * m + 2 * m * d) * 4, BH * 2 * m * m * d, "alu"
+        # tf32 tensor cores for bf16 inputs at m = 128 / 256, fp32 FMAs otherwise
+        return BH * (m * m + 2 * m * d) * 4, BH * 2 * m * m * d, \
+            "tensor_tf32" if (w.dtype == "bf16" and m % 128 == 0) else "alu"
     if kernel == "output":
         return 3 * tensor + BH * 2 * m * d * 4, BH * (4 * n * m * d + (2 * 65 * n * d if w.conv else 0)), unit
     raise KeyError(kernel)
@@ -158,7 +158,7 @@ def compute_peak_tflops(unit, peaks, kernel_impl_simt):
     return peaks["bf16_tflops"]
 
 
-SIMT_KERNELS = {"landmarks", "k3v_combine", "w_product", "kernel2", "mask_bits"}
+SIMT_KERNELS = {"landmarks", "k3v_combine", "mask_bits"}
 
 
 def roofline_for(w, kernel, avg_ms, peaks, simt_set, traffic, path="nystrom"):
@@ -554,7 +554,9 @@ def main():
             traffic = ent.get("bytes_per_launch")
     simt = set(SIMT_KERNELS)
     if w.dtype == "f32":  # the float32 path runs every stage on CUDA cores
-        simt |= {"pinv", "k3v_partial", "output"}
+        simt |= {"pinv", "k3v_partial", "output", "w_product"}
+    elif w.m % 128 != 0:
+        simt.add("w_product")   # W on CUDA cores at m = 64
     if args.path == "exact":
         traffic = None   # the ncu traffic figures are for the Nystrom path's kernels
     roof = roofline_for(w, dom, prof[dom][1] / max(1, prof[dom][0]), peaks, simt, traffic, args.path)

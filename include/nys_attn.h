@@ -67,7 +67,8 @@ typedef enum {
     NYS_ERR_CUDA = -3,         /* a CUDA call failed                                           */
     NYS_ERR_NOMEM = -4,        /* workspace allocation failed                                  */
     NYS_ERR_TIMEOUT = -5,      /* a bounded device-side wait ran out                           */
-    NYS_ERR_SCRATCH_LIMIT = -6 /* needs more than the fixed static scratch (nys_attn_pinv_static) */
+    NYS_ERR_SCRATCH_LIMIT = -6, /* needs more than the fixed static scratch (nys_attn_pinv_static) */
+    NYS_ERR_GUARD = -7          /* a workspace guard zone was overwritten (guard mode only)    */
 } nys_status_t;
 
 /*
@@ -206,7 +207,8 @@ int nys_attn_pinv_static(const float* q_l, const float* k_l, float* z, int BH, i
                          int n_iter, void* stream);
 
 /* Synchronises the current device, then returns and clears the device status
- * word (NYS_OK or NYS_ERR_TIMEOUT); NYS_ERR_CUDA if the synchronisation fails. */
+ * word (NYS_OK, NYS_ERR_TIMEOUT or NYS_ERR_GUARD); NYS_ERR_CUDA if the
+ * synchronisation fails. */
 int nys_attn_device_status(void);
 
 /* Bytes of device scratch nys_attn_forward takes for this shape (0 if invalid). */
@@ -243,6 +245,37 @@ int nys_attn_selftest_exp2(float* max_rel_err);
  * one second, NYS_ERR_CUDA on a CUDA failure.
  */
 int nys_attn_selftest_wait_timeout(unsigned long long limit_ns, int* completed);
+
+/*
+ * nys_attn_set_workspace_guard -- a checking mode for the workspace of
+ * nys_attn_forward / _ex / _debug / _host (an implementation check with no
+ * counterpart in the pages). enable = 1 turns it on for every later call in
+ * the process, 0 turns it off; returns the previous setting, or
+ * NYS_ERR_INVALID_ARG for any other value. While it is on, each workspace
+ * buffer lies between 4 KiB guard zones, the whole workspace is set to 0xFF
+ * bytes before the first kernel (a NaN in float32 and bf16, so a read of an
+ * element that no kernel wrote makes the result non-finite), and after the
+ * last kernel a check records NYS_ERR_GUARD in the device status word (read
+ * it with nys_attn_device_status) if any guard byte changed. The calls stay
+ * asynchronous; the workspace grows by at most 17 zones (68 KiB) and each
+ * call adds one memset and one small kernel. nys_attn_workspace_bytes
+ * reports the size for the current setting.
+ */
+int nys_attn_set_workspace_guard(int enable);
+
+/*
+ * Self-test of the guard check (an implementation check with no counterpart
+ * in the pages). Allocates a 12 KiB buffer holding two guard zones around a
+ * 4 KiB region, fills it as the guard mode does, overwrites the region in
+ * the middle (which is allowed) and, with corrupt = 1, one byte of the second
+ * zone from the host (cudaMemset, inside the allocation), then runs the
+ * check. *status (host pointer) receives what the device status word then
+ * holds: NYS_OK for corrupt = 0, NYS_ERR_GUARD for corrupt = 1. Synchronous;
+ * the status word is read and cleared. NYS_ERR_INVALID_ARG for a null
+ * pointer, a corrupt value other than 0 / 1, or a status word that already
+ * held an error when the call began; NYS_ERR_CUDA on a CUDA failure.
+ */
+int nys_attn_selftest_guard(int corrupt, int* status);
 
 /*
  * Per-kernel timing, for benchmarks. While enabled, each kernel launch of

@@ -29,7 +29,9 @@ F32, BF16 = 0, 1
 INV_INIT_DEFAULT, INV_INIT_EXACT = 0, 1
 _STATUS = {0: "ok", -1: "invalid argument", -2: "unsupported shape or dtype", -3: "CUDA error",
            -4: "device workspace allocation failed", -5: "bounded device wait timed out",
-           -6: "problem exceeds the library's fixed static scratch"}
+           -6: "problem exceeds the library's fixed static scratch",
+           -7: "a workspace guard zone was overwritten (guard mode)"}
+OK, ERR_TIMEOUT, ERR_GUARD = 0, -5, -7
 
 
 class NysError(RuntimeError):
@@ -69,6 +71,10 @@ def _load() -> ctypes.CDLL:
     lib.nys_attn_pinv_static.restype = i
     lib.nys_attn_selftest_wait_timeout.argtypes = [ctypes.c_ulonglong, ctypes.POINTER(ctypes.c_int)]
     lib.nys_attn_selftest_wait_timeout.restype = i
+    lib.nys_attn_set_workspace_guard.argtypes = [i]
+    lib.nys_attn_set_workspace_guard.restype = i
+    lib.nys_attn_selftest_guard.argtypes = [i, ctypes.POINTER(ctypes.c_int)]
+    lib.nys_attn_selftest_guard.restype = i
     lib.nys_attn_selftest_exp2.argtypes = [ctypes.POINTER(ctypes.c_float)]
     lib.nys_attn_selftest_exp2.restype = i
     lib.nys_strerror.argtypes = [i]
@@ -233,6 +239,25 @@ def selftest_wait_timeout(limit_ns: int = 1_000_000) -> int:
     _check(lib.nys_attn_selftest_wait_timeout(int(limit_ns), ctypes.byref(done)),
            "nys_attn_selftest_wait_timeout")
     return int(done.value)
+
+
+def set_workspace_guard(enable: bool) -> bool:
+    """Turn the workspace guard mode on or off for later calls; returns the previous setting.
+
+    While it is on, every workspace buffer lies between guard zones, the workspace starts as
+    0xFF bytes (NaN), and a check after each call records ERR_GUARD in the device status word
+    if a guard byte changed (read it with device_status())."""
+    prev = int(lib.nys_attn_set_workspace_guard(1 if enable else 0))
+    _check(min(prev, 0), "nys_attn_set_workspace_guard")
+    return bool(prev)
+
+
+def selftest_guard(corrupt: bool) -> int:
+    """Run the guard check on a small buffer, with one guard byte changed from the host if
+    `corrupt`; returns the status word it left (OK, or ERR_GUARD when corrupt)."""
+    st = ctypes.c_int(1)
+    _check(lib.nys_attn_selftest_guard(1 if corrupt else 0, ctypes.byref(st)), "nys_attn_selftest_guard")
+    return int(st.value)
 
 
 def workspace_bytes(B, H, n, d, m, dtype_code=BF16) -> int:

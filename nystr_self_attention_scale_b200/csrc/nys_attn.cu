@@ -12,6 +12,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <type_traits>
 #include <vector>
@@ -23,9 +24,9 @@
 #include "simt.cuh"
 #include "tc_k3v.cuh"
 #include "tc_output.cuh"
-#include "tc_pinv.cuh"
 #include "tc_pinv_pair.cuh"
 #include "tc_pinv_res.cuh"
+#include "tc_w.cuh"
 
 namespace nys {
 namespace {
@@ -89,6 +90,28 @@ int device_state(DeviceState** out) {
 }
 
 size_t align_up(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------- workspace guard mode
+// With the guard mode on (nys_attn_set_workspace_guard), every workspace buffer sits between
+// guard zones, the whole workspace is filled with 0xFF bytes before the first launch (a NaN
+// in fp32 and bf16, so a read of an element no kernel wrote poisons the result), and after
+// the last launch one CTA per zone checks that every guard byte is still 0xFF; a changed
+// byte records NYS_ERR_GUARD in the device status word.
+constexpr size_t kGuardBytes = 4096;
+constexpr int kMaxGuards = 17;   // make_plan takes at most 16 buffers, + a trailing zone
+std::atomic<int> g_guard_mode{0};
+
+struct GuardList {
+    unsigned long long off[kMaxGuards];
+    int n;
+};
+
+__global__ void guard_check_kernel(const uint32_t* __restrict__ ws, const GuardList zones) {
+    const uint32_t* z = ws + zones.off[blockIdx.x] / 4;
+    bool bad = false;
+    for (int i = threadIdx.x; i < (int)(kGuardBytes / 4); i += blockDim.x) bad |= z[i] != 0xFFFFFFFFu;
+    if (__syncthreads_or(bad) && threadIdx.x == 0) record_status(NYS_ERR_GUARD);
+}
 
 // [B, n] uint8 key mask -> [B, n / 32] validity bits (bit i of word w = key 32 w + i).
 __global__ void mask_bits_kernel(const uint8_t* __restrict__ mask, uint32_t* __restrict__ bits, int B, int n) {
@@ -158,10 +181,10 @@ bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
 // ---------------------------------------------------------------- per-kernel timing
 // When enabled, every launch is bracketed by two CUDA events on the stream it
 // runs on; nys_attn_profile_read() sums their elapsed times per kernel.
-enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_MASKBITS, K_KERNEL2, K_PROBS,
+enum KernelId { K_LANDMARKS = 0, K_PINV, K_K3V, K_COMBINE, K_W, K_OUTPUT, K_MASKBITS, K_PROBS,
                 K_COUNT };
 const char* const kKernelNames[K_COUNT] = {"landmarks", "pinv", "k3v_partial", "k3v_combine",
-                                           "w_product", "output", "mask_bits", "kernel2", "attn_probs"};
+                                           "w_product", "output", "mask_bits", "attn_probs"};
 
 struct ProfRecord { int kid; cudaEvent_t a, b; };
 std::mutex g_prof_mu;
@@ -209,8 +232,9 @@ struct Plan {
     int BH, splits, keys_per_split;
     size_t off_ql, off_kl, off_ql16, off_kl16, off_k3v, off_w, off_wt16, off_z, off_pinv;
     size_t off_po, off_pm, off_pl, off_mbits, total;
-    size_t off_k2b, off_k2tb, off_zb, off_ztb, off_ta, off_tb, off_colsum, off_rowsum;  // tensor-core inverse
+    size_t off_k2b, off_k2tb, off_zb;   // CTA-pair inverse (m = 256): k2, k2^T and W^T scratch
     int tc_cps, tc_splits;  // tensor-core kernel_3 V: 128-key chunks per split, splits
+    GuardList guards;       // guard zones (guard mode only; guards.n == 0 otherwise)
 };
 
 // Per-call options beyond the spec signature (nys_attn_forward_ex).
@@ -266,11 +290,23 @@ Plan make_plan_exact(int B, int H, int n, int d, int dtype) {
     p.keys_per_split = kps;
     const size_t BH = p.BH;
     size_t o = 0;
-    auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+    const bool guard = g_guard_mode.load() != 0;
+    p.guards.n = 0;
+    auto zone = [&]() {
+        if (p.guards.n < kMaxGuards) p.guards.off[p.guards.n++] = o;
+        o += kGuardBytes;
+    };
+    auto take = [&](size_t bytes) {
+        if (guard) zone();
+        size_t r = o;
+        o = align_up(o + bytes);
+        return r;
+    };
     p.off_po = take(BH * splits * (size_t)n * d * 4);
     p.off_pm = take(BH * splits * (size_t)n * 4);
     p.off_pl = take(BH * splits * (size_t)n * 4);
     p.off_mbits = take((size_t)B * ((n + 31) / 32) * 4);
+    if (guard) zone();
     p.total = o;
     return p;
 }
@@ -297,7 +333,18 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
     p.keys_per_split = kps;
     const size_t BH = p.BH, md = (size_t)m * d, mm = (size_t)m * m;
     size_t o = 0;
-    auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes); return r; };
+    const bool guard = g_guard_mode.load() != 0;
+    p.guards.n = 0;
+    auto zone = [&]() {
+        if (p.guards.n < kMaxGuards) p.guards.off[p.guards.n++] = o;
+        o += kGuardBytes;
+    };
+    auto take = [&](size_t bytes) {
+        if (guard) zone();
+        size_t r = o;
+        o = align_up(o + bytes);
+        return r;
+    };
     p.off_ql = take(BH * md * 4);
     p.off_kl = take(BH * md * 4);
     p.off_ql16 = take(BH * md * 2);
@@ -311,18 +358,26 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
     p.off_pm = take(BH * splits * (size_t)m * 4);
     p.off_pl = take(BH * splits * (size_t)m * 4);
     p.off_mbits = take((size_t)B * ((n + 31) / 32) * 4);
-    if (dtype == NYS_BF16) {
+    if (dtype == NYS_BF16 && m == 256) {
         p.off_k2b = take(BH * mm * 4);
         p.off_k2tb = take(BH * mm * 4);
         p.off_zb = take(BH * mm * 4);
-        p.off_ztb = take(BH * mm * 4);
-        p.off_ta = take(BH * mm * 4);
-        p.off_tb = take(BH * mm * 4);
-        p.off_colsum = take(BH * ((m + 31) / 32) * (size_t)m * 4);
-        p.off_rowsum = take(BH * (size_t)m * 4);
     }
+    if (guard) zone();
     p.total = o;
     return p;
+}
+
+// Guard mode: fill the workspace before the first launch, check its guard zones after the last.
+int guard_fill(const Plan& p, void* ws, cudaStream_t s) {
+    if (p.guards.n == 0) return NYS_OK;
+    return cudaMemsetAsync(ws, 0xFF, p.total, s) == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+}
+
+int guard_check(const Plan& p, const void* ws, cudaStream_t s) {
+    if (p.guards.n == 0) return NYS_OK;
+    guard_check_kernel<<<p.guards.n, 256, 0, s>>>(static_cast<const uint32_t*>(ws), p.guards);
+    return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
 }
 
 template <typename T, int D>
@@ -454,55 +509,6 @@ int launch_k3v_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* row
     return NYS_OK;
 }
 
-template <int M>
-int launch_pinv_tc(const Plan& p, const DeviceState& st, const float* ql, const float* kl, float* z, char* ws,
-                   int inv_init, cudaStream_t s) {
-    using C = PinvTc<M>;
-    static bool attr_set[kMaxDevices] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    const size_t smem2 = (size_t)(32 + M) * (p.d + 1) * sizeof(float);
-    if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(pinv_tc_kernel<M>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)C::kSmemBytes) != cudaSuccess ||
-            cudaFuncSetAttribute(kernel2_kernel<32, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 96 * 1024) != cudaSuccess ||
-            cudaFuncSetAttribute(kernel2_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 96 * 1024) != cudaSuccess)
-            return NYS_ERR_CUDA;
-        attr_set[dev] = true;
-    }
-    uint8_t* k2b = reinterpret_cast<uint8_t*>(ws + p.off_k2b);
-    uint8_t* k2tb = reinterpret_cast<uint8_t*>(ws + p.off_k2tb);
-    float* colsum = reinterpret_cast<float*>(ws + p.off_colsum);
-    float* rowsum = reinterpret_cast<float*>(ws + p.off_rowsum);
-    {
-        ProfScope ps(K_KERNEL2, s);
-        if (p.d == 64)
-            kernel2_kernel<64, false><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
-        else
-            kernel2_kernel<32, false><<<dim3(p.BH, M / 32), 256, smem2, s>>>(ql, kl, k2b, k2tb, colsum, rowsum, M);
-    }
-    PinvTcParams prm{k2b, k2tb, reinterpret_cast<uint8_t*>(ws + p.off_zb), reinterpret_cast<uint8_t*>(ws + p.off_ztb),
-                     reinterpret_cast<uint8_t*>(ws + p.off_ta),
-                     reinterpret_cast<uint8_t*>(ws + p.off_tb), colsum, rowsum, z, p.n_iter, inv_init};
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.BH * C::kClusterSize);
-    cfg.blockDim = dim3(128);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = C::kClusterSize;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    ProfScope ps(K_PINV, s);
-    if (cudaLaunchKernelEx(&cfg, pinv_tc_kernel<M>, prm) != cudaSuccess) return NYS_ERR_CUDA;
-    return NYS_OK;
-}
-
 // m = 64 and 128: kernel_2 and the iterative inverse in one CTA per 128 rows (two heads per CTA
 // at m = 64), every operand on chip. `started` (or null) fires once every CTA has begun.
 template <int MH>
@@ -614,8 +620,13 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
         ProfScope ps(K_LANDMARKS, s);
         constexpr int rows_per_instr = 32 / (D / 8);
         if ((n / m) % rows_per_instr == 0) {
-            // eight CTAs of eight warps per SM (the register file's limit), striding over the landmarks
-            landmarks_warp_kernel<D><<<8 * st.sm_count, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, m);
+            // at most eight CTAs of eight warps per SM (the register file's limit), striding over
+            // the landmarks, and just enough of them that every warp takes the same number of
+            // landmarks (no partly-filled last round)
+            const long long units = 2LL * BH * m, slots = 64LL * st.sm_count;
+            const long long per_warp = (units + slots - 1) / slots;
+            const int ctas = (int)((units + 8 * per_warp - 1) / (8 * per_warp));
+            landmarks_warp_kernel<D><<<ctas, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, m);
         } else {
             long long threads = (long long)BH * m * (D / 8);
             dim3 grid((unsigned)((threads + 255) / 256), 2);
@@ -687,13 +698,23 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
         cudaGetDevice(&dev);
         if (!attr_set[dev]) {
             if (cudaFuncSetAttribute(w_tile_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     (int)WTile<D>::bytes(256)) != cudaSuccess)
+                                     (int)WTile<D>::bytes(256)) != cudaSuccess ||
+                cudaFuncSetAttribute(w_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)WTc<D>::bytes(256)) != cudaSuccess)
                 return NYS_ERR_CUDA;
             attr_set[dev] = true;
         }
         ProfScope ps(K_W, s);
-        w_tile_kernel<D><<<dim3(m / WTile<D>::kRows, BH), WTile<D>::kThreads, WTile<D>::bytes(m), s>>>(
-            z, k3v, w, wt16, m);
+        if (m % 128 == 0) {
+            // tensor cores: one CTA per 128 rows of W, Z rows by TMA
+            CUtensorMap map_z;
+            if (!map_3d(&map_z, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, z, m, m, BH, 32, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                return NYS_ERR_CUDA;
+            w_tc_kernel<D><<<dim3(m / 128, BH), WTc<D>::kThreads, WTc<D>::bytes(m), s>>>(map_z, k3v, w, wt16, m);
+        } else {
+            w_tile_kernel<D><<<dim3(m / WTile<D>::kRows, BH), WTile<D>::kThreads, WTile<D>::bytes(m), s>>>(
+                z, k3v, w, wt16, m);
+        }
     }
     switch (m) {
         case 64: rc = launch_output_tc<D, 64>(p, st, q, v, conv_w, out, kl16, wt16, s); break;
@@ -780,6 +801,11 @@ int run_exact(const void* q, const void* k, const void* v, const uint8_t* mask, 
     char* w = static_cast<char*>(ws);
     std::unique_lock<std::mutex> launch_lock(st->launch_mu);
     using bf = __nv_bfloat16;
+    rc = guard_fill(p, ws, s);
+    if (rc != NYS_OK) {
+        cudaFreeAsync(ws, s);
+        return rc;
+    }
     if (dtype == NYS_F32)
         rc = d == 64 ? launch_exact<float, 64>(p, *st, (const float*)q, (const float*)k, (const float*)v, mask,
                                                conv_w, (float*)out, attn_probs, w, s)
@@ -790,6 +816,7 @@ int run_exact(const void* q, const void* k, const void* v, const uint8_t* mask, 
                                             (bf*)out, attn_probs, w, s)
                      : launch_exact<bf, 32>(p, *st, (const bf*)q, (const bf*)k, (const bf*)v, mask, conv_w,
                                             (bf*)out, attn_probs, w, s);
+    if (rc == NYS_OK) rc = guard_check(p, ws, s);
     if (cudaFreeAsync(ws, s) != cudaSuccess && rc == NYS_OK) rc = NYS_ERR_CUDA;
     return rc;
 }
@@ -815,6 +842,11 @@ int run(const void* q, const void* k, const void* v, const uint8_t* mask, const 
     char* w = static_cast<char*>(ws);
     std::unique_lock<std::mutex> launch_lock(st->launch_mu);
     using bf = __nv_bfloat16;
+    rc = guard_fill(p, ws, s);
+    if (rc != NYS_OK) {
+        cudaFreeAsync(ws, s);
+        return rc;
+    }
     if (dtype == NYS_F32) {
         rc = d == 64 ? launch_simt<float, 64>(p, *st, (const float*)q, (const float*)k, (const float*)v,
                                               mask, conv_w, (float*)out, w, opt.inv_init, s)
@@ -844,6 +876,7 @@ int run(const void* q, const void* k, const void* v, const uint8_t* mask, const 
             if (c.dst && cudaMemcpyAsync(c.dst, w + c.off, c.bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess)
                 rc = NYS_ERR_CUDA;
     }
+    if (rc == NYS_OK) rc = guard_check(p, ws, s);
     if (cudaFreeAsync(ws, s) != cudaSuccess && rc == NYS_OK) rc = NYS_ERR_CUDA;
     return rc;
 }
@@ -1067,6 +1100,7 @@ const char* nys_strerror(int status) {
         case NYS_ERR_NOMEM: return "device workspace allocation failed";
         case NYS_ERR_TIMEOUT: return "bounded device wait timed out";
         case NYS_ERR_SCRATCH_LIMIT: return "problem exceeds the library's fixed static scratch";
+        case NYS_ERR_GUARD: return "a workspace guard zone was overwritten (guard mode)";
         default: return "unknown status";
     }
 }
@@ -1117,6 +1151,40 @@ int nys_attn_selftest_wait_timeout(unsigned long long limit_ns, int* completed) 
     cudaFree(d);
     *completed = h;
     return rc;
+}
+
+int nys_attn_set_workspace_guard(int enable) {
+    if (enable != 0 && enable != 1) return NYS_ERR_INVALID_ARG;
+    return nys::g_guard_mode.exchange(enable);
+}
+
+int nys_attn_selftest_guard(int corrupt, int* status) {
+    if (!status || (corrupt != 0 && corrupt != 1)) return NYS_ERR_INVALID_ARG;
+    nys::Plan p{};
+    p.guards.n = 2;
+    p.guards.off[0] = 0;
+    p.guards.off[1] = 2 * nys::kGuardBytes;   // a 4 KiB "buffer" between the zones
+    p.total = 3 * nys::kGuardBytes;
+    void* ws = nullptr;
+    if (cudaMalloc(&ws, p.total) != cudaSuccess) return NYS_ERR_CUDA;
+    int rc = cudaDeviceSynchronize() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
+    int prior = 0;
+    if (rc == NYS_OK && cudaMemcpyFromSymbol(&prior, nys::g_status, sizeof(int)) != cudaSuccess) rc = NYS_ERR_CUDA;
+    if (rc == NYS_OK && prior != NYS_OK) rc = NYS_ERR_INVALID_ARG;   // the caller must read the word first
+    if (rc == NYS_OK) rc = nys::guard_fill(p, ws, 0);
+    // the buffer itself may be written freely; with corrupt = 1 one byte of the second zone changes
+    if (rc == NYS_OK && cudaMemset(static_cast<char*>(ws) + nys::kGuardBytes, 0, nys::kGuardBytes) != cudaSuccess)
+        rc = NYS_ERR_CUDA;
+    if (rc == NYS_OK && corrupt &&
+        cudaMemset(static_cast<char*>(ws) + 2 * nys::kGuardBytes + 1000, 0x7F, 1) != cudaSuccess)
+        rc = NYS_ERR_CUDA;
+    if (rc == NYS_OK) rc = nys::guard_check(p, ws, 0);
+    if (rc == NYS_OK && cudaDeviceSynchronize() != cudaSuccess) rc = NYS_ERR_CUDA;
+    cudaFree(ws);
+    if (rc == NYS_OK) rc = nys_attn_device_status();
+    if (rc < 0 && rc != NYS_ERR_GUARD) return rc;
+    *status = rc;
+    return NYS_OK;
 }
 
 int nys_attn_selftest_exp2(float* max_rel_err) {

@@ -266,6 +266,24 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
 // 32-byte granules, the one layout an MN-major tf32 operand can take).
 enum : uint32_t { kLayoutNone = 0, kLayoutSw128 = 2, kLayoutSw64 = 4, kLayoutSw32 = 6, kLayoutSw128B32 = 1 };
 
+// fp32 -> tf32 (round to nearest, ties away from zero), kept in an fp32 register: the value a
+// kind::tf32 MMA operand holds
+__device__ __forceinline__ float tf32_rna(float x) {
+    uint32_t y;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(y) : "f"(x));
+    return __uint_as_float(y);
+}
+
+// ---------------------------------------------------------------- clusters
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside an MN-major tf32 operand
 // atom of the 32-byte-granule 128-byte swizzle: rows (K) of 128 bytes (32 tf32 along MN),
 // 4 rows per 512-byte atom, the 32-byte granule index XORed with row % 4. Atoms of 4 rows sit

@@ -36,7 +36,7 @@
 // chunk max through shared memory. Each SM sub-partition runs four softmax
 // warps, two per stream. Each group writes its P (bf16 pairs) into its half
 // of the stream's P buffer.
-// K/V chunks use a 4-stage shared-memory ring.
+// K/V chunks use a 6-stage shared-memory ring (three chunks of lookahead per stream).
 #pragma once
 
 #include "sm100.cuh"
@@ -49,7 +49,7 @@ struct K3vTc {
     static constexpr int kSpan = D * 2;
     static constexpr uint32_t kLayout = D == 64 ? sm100::kLayoutSw128 : sm100::kLayoutSw64;
     static constexpr uint32_t kSbo = 8 * kSpan;
-    static constexpr int kStages = 4;
+    static constexpr int kStages = 6;
     static constexpr uint32_t kTileBytes = 128 * kSpan;
     static constexpr uint32_t kOffQl = 0;
     static constexpr uint32_t kOffK = kOffQl + kTileBytes;
@@ -351,17 +351,17 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 // bf16 (nearest even); the running sum adds the fp32 values.
                 const uint64_t sc2 = f2(sc, sc), nmo2 = f2(-mo, -mo);
                 uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-#pragma unroll 1
+                // pass 2: this group's 64 scores again, with one wait; then the S buffer is released
+                // to the stream's next S MMA
+                uint32_t vv[2][32];
+                tmem_ld32(sbuf, vv[0]);
+                tmem_ld32(sbuf + 32, vv[1]);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(&s_free[t]);
+#pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    // pass 2, 32 keys per TMEM load; after the last load the S buffer is released
-                    // to the stream's next S MMA
-                    uint32_t v[32];
-                    tmem_ld32(sbuf + 32 * h, v);
-                    tmem_ld_wait();
-                    if (h == 1) {
-                        tc_fence_before();
-                        mbar_arrive(&s_free[t]);
-                    }
+                    uint32_t* v = vv[h];
                     if (!full) {
 #pragma unroll
                         for (int e = 0; e < 32; ++e)

@@ -19,11 +19,13 @@
 // warps 10-13 epilogue (and the Toeplitz build), warp 14 TMA producer of the
 // V halos. A warp w reaches TMEM lanes 32 (w % 4) .. +31, so each group of four
 // warps covers all 128 rows. Two TMEM slots alternate between consecutive
-// tiles, and softmax group g owns slot g: it takes every other tile, whole
-// rows (all landmark columns), so neither group waits for the other and the
-// two, at different points of their tiles, hide each other's TMEM latency on
-// each SM sub-partition. P is written, packed, over the first M/2 columns of
-// the slot, where the P.W MMA reads its A operand. Every wait is bounded.
+// tiles. Both softmax groups work on every tile, group g on the landmark
+// columns [g M/2, (g+1) M/2) of each row, and exchange the row max through
+// shared memory: a tile's softmax takes half as long on the chain that
+// reuses its slot (S MMA, softmax, O MMAs, epilogue read), and each SM
+// sub-partition runs one warp of each group on it. Each group writes its P,
+// packed, over the first half of its own columns, where the P.W MMA reads its
+// A operand. Every wait is bounded.
 #pragma once
 
 #include "sm100.cuh"
@@ -47,22 +49,29 @@ struct OutTc {
     static constexpr uint32_t kTBlock = 128 * 128;    // [128][64] bf16 K-block of T
     static constexpr uint32_t kTBytes = 3 * kTBlock;
     static constexpr uint32_t kOutBytes = kRows * kSpan;
-    // TMEM slot (256 columns): S in [0, M); P (bf16 pairs) over [0, M/2); O_att and O_conv
-    // after P, in S columns the softmax has finished reading before the O MMAs are issued
+    // TMEM slot (256 columns): S in [0, M). Softmax group g reads S's columns [g M/2, (g+1) M/2)
+    // and writes its P (bf16 pairs) over the first half of that range, columns it has already
+    // read. For M = 256 the O accumulators take the second halves of the two ranges (read by
+    // then); for M <= 128 they sit after S.
     static constexpr int kSlot = 256;
     static constexpr int kTmemCols = 2 * kSlot;
-    static constexpr int kColP = 0;
-    static constexpr int kColOatt = M == 256 ? M / 2 : M;
-    static constexpr int kColOconv = kColOatt + D;
-    static_assert(kColOconv + D <= kSlot, "TMEM slot layout");
+    static constexpr int kHalfCols = M / 2;           // S columns per softmax group
+    static constexpr int kColOatt = M == 256 ? 64 : M;
+    static constexpr int kColOconv = M == 256 ? 192 : M + D;
+    static_assert(kColOconv + D <= kSlot && (M != 256 || kColOatt + D <= 128), "TMEM slot layout");
+    // TMEM column of the packed P pair holding landmark `c` (even)
+    __host__ __device__ static constexpr int p_col(int c) {
+        return c < kHalfCols ? c / 2 : kHalfCols + (c - kHalfCols) / 2;
+    }
     static constexpr uint32_t kOffQ = 0;
     static constexpr uint32_t kOffV = kOffQ + kStages * kQBytes;
     static constexpr uint32_t kOffKl = kOffV + kStages * kVBytes;
     static constexpr uint32_t kOffWt = kOffKl + kKlBytes;
     static constexpr uint32_t kOffT = kOffWt + kWtBytes;
     static constexpr uint32_t kOffOut = kOffT + kTBytes;
-    static constexpr uint32_t kOffPsum = kOffOut + kOutBytes;   // [2 slots][128] float row sums
-    static constexpr uint32_t kOffBar = kOffPsum + 2 * 128 * 4;
+    static constexpr uint32_t kOffPsum = kOffOut + kOutBytes;   // [2 slots][2 groups][128] partial row sums
+    static constexpr uint32_t kOffXch = kOffPsum + 2 * 2 * 128 * 4;   // [2 slots][2 groups][128] partial row maxima
+    static constexpr uint32_t kOffBar = kOffXch + 2 * 2 * 128 * 4;
     static constexpr int kNumBars = 20;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -92,7 +101,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint64_t* q_full = bars + 0;     // [2] Q tile landed
     uint64_t* q_empty = bars + 2;    // [2] Q stage reusable (its S MMA completed)
     uint64_t* s_full = bars + 4;     // [2] S in TMEM
-    uint64_t* p_full = bars + 6;     // [2] P in TMEM, S fully read (128 arrivals)
+    uint64_t* p_full = bars + 6;     // [2] P in TMEM, S fully read (256 arrivals)
     uint64_t* o_full = bars + 8;     // [2] O_att, O_conv ready
     uint64_t* slot_free = bars + 10; // [2] epilogue done with the slot (128 arrivals)
     uint64_t* const_full = bars + 12;
@@ -104,6 +113,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
     float* psum = reinterpret_cast<float*>(sm + C::kOffPsum);
+    float* pmax = reinterpret_cast<float*>(sm + C::kOffXch);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // contiguous tile range of this CTA
@@ -118,7 +128,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mbar_init(&q_full[b], 1);
             mbar_init(&q_empty[b], 1);
             mbar_init(&s_full[b], 1);
-            mbar_init(&p_full[b], 128);
+            mbar_init(&p_full[b], 256);
             mbar_init(&o_full[b], 1);
             mbar_init(&slot_free[b], 128);
             mbar_init(&v_full[b], 1);
@@ -247,7 +257,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             if (elect_one()) {
 #pragma unroll
                 for (int k = 0; k < M / 16; ++k)   // landmarks 16k .. 16k+15: 8 packed P columns
-                    mma_bf16_ts(slot + C::kColOatt, slot + C::kColP + k * 8, descWt(k), C::kIdPW, k > 0);
+                    mma_bf16_ts(slot + C::kColOatt, slot + C::p_col(16 * k), descWt(k), C::kIdPW, k > 0);
             }
             if (prm.conv_w != nullptr) {
                 if (!wait(&v_full[st], (j / C::kStages) & 1)) return false;
@@ -287,75 +297,87 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         mma_commit(mma_done);
         mbar_wait(mma_done, 0);
     } else if (warp >= 2 && warp < 10) {
-        // ------------------------------------------------ softmax: group g takes the tiles i with
-        // i % 2 == g (TMEM slot g), one whole row of S per thread
+        // ------------------------------------------------ softmax: both groups take every tile, group g
+        // the landmark columns [g M/2, (g+1) M/2) of each row (one row per thread); the row max is
+        // exchanged through shared memory
         const int g = (warp - 2) >> 2;
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
         const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
         const float sc = split_scale(D) * kLog2e;  // S holds Q . K_l^T with K_l already scaled
-        constexpr int kB = M < 64 ? M : 64;        // S columns per TMEM wait
-        for (int i = g; i < count && !warp_any(*abort_flag != 0); i += 2) {
-            const int s = g;
-            if (!warp_all(mbar_wait(&s_full[s], (i >> 1) & 1))) { *abort_flag = 1; break; }
+        constexpr int kB = C::kHalfCols < 64 ? C::kHalfCols : 64;   // S columns per TMEM wait
+        const int cbase = g * C::kHalfCols;
+        // one named barrier per tile (the max exchange): a group can only reach tile i + 2's
+        // exchange, which reuses tile i's maxima slots, after both groups left tile i + 1's
+        for (int i = 0; i < count; ++i) {
+            const int s = i & 1;
+            const bool ok = warp_all(mbar_wait(&s_full[s], (i >> 1) & 1));
             tc_fence_after();
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
-            // pass 1: the row max, kB columns per wait
+            // pass 1: this half-row's max, kB columns per wait
             float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four short max chains
+            if (ok) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < M; c0 += kB) {
-                uint32_t v[kB / 32][32];
+                for (int c0 = cbase; c0 < cbase + C::kHalfCols; c0 += kB) {
+                    uint32_t v[kB / 32][32];
 #pragma unroll
-                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(slot + c0 + bq * 32, v[bq]);
-                tmem_ld_wait();
+                    for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(slot + c0 + bq * 32, v[bq]);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int bq = 0; bq < kB / 32; ++bq)
+                    for (int bq = 0; bq < kB / 32; ++bq)
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        mq[j & 3] = max3(mq[j & 3], __uint_as_float(v[bq][2 * j]), __uint_as_float(v[bq][2 * j + 1]));
+                        for (int j = 0; j < 16; ++j)
+                            mq[j & 3] = max3(mq[j & 3], __uint_as_float(v[bq][2 * j]), __uint_as_float(v[bq][2 * j + 1]));
+                }
             }
-            const float mo = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sc;
-            // pass 2: P over the first M/2 columns, in increasing column order, so it only
-            // overwrites scores this thread has already read.
+            pmax[(s * 2 + g) * 128 + r] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            // also publishes the maxima; a wait that ran out in either group, or an abort by another
+            // role, stops both groups together
+            if (group_any(!ok || *abort_flag != 0, 3, 256)) { *abort_flag = 1; break; }
+            const float mo = fmaxf(pmax[(s * 2) * 128 + r], pmax[(s * 2 + 1) * 128 + r]) * sc;
+            // pass 2: P over the first half of this group's columns, in increasing column order, so
+            // it only overwrites scores this thread has already read.
             // exponentials on packed fp32 pairs: the MUFU unit takes 10 of every 16 pairs, the FMA
             // pipe the other 6 (polynomial 2^x), so neither pipe alone bounds the loop. P is rounded
             // to bf16 (nearest even); the row sum adds the fp32 values.
+            // 32 columns per TMEM load, two register buffers: the load of the next 32 scores is in
+            // flight while the current 32 are exponentiated (tcgen05.wait::ld then waits for it alone)
             const uint64_t sc2 = f2(sc, sc), nmo2 = f2(-mo, -mo);
             uint64_t acc[2] = {f2(0.f, 0.f), f2(0.f, 0.f)};
-#pragma unroll 1
-            for (int c0 = 0; c0 < M; c0 += kB) {
-                uint32_t v[kB / 32][32];
+            constexpr int kChunks = C::kHalfCols / 32;
+            uint32_t vb[2][32];
+            tmem_ld32(slot + cbase, vb[0]);
+            tmem_ld_wait();
 #pragma unroll
-                for (int bq = 0; bq < kB / 32; ++bq) tmem_ld32(slot + c0 + bq * 32, v[bq]);
-                tmem_ld_wait();
+            for (int cc = 0; cc < kChunks; ++cc) {
+                if (cc + 1 < kChunks) tmem_ld32(slot + cbase + 32 * (cc + 1), vb[(cc + 1) & 1]);
+                const uint32_t* v = vb[cc & 1];
+                uint32_t pk[16];
 #pragma unroll
-                for (int bq = 0; bq < kB / 32; ++bq) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const uint64_t x2 = f2_fma(f2(__uint_as_float(v[bq][2 * j]), __uint_as_float(v[bq][2 * j + 1])),
-                                                   sc2, nmo2);
-                        float e0, e1;
-                        if ((j & 7) == 2 || (j & 7) == 5 || (j & 7) == 7) {
-                            exp2_poly_pair(x2, e0, e1);
-                        } else {
-                            float x0, x1;
-                            f2_split(x2, x0, x1);
-                            e0 = ex2(x0);
-                            e1 = ex2(x1);
-                        }
-                        pk[j] = pack_bf16_rn(e0, e1);
-                        acc[j & 1] = f2_add(acc[j & 1], f2(e0, e1));
+                for (int j = 0; j < 16; ++j) {
+                    const uint64_t x2 = f2_fma(f2(__uint_as_float(v[2 * j]), __uint_as_float(v[2 * j + 1])), sc2, nmo2);
+                    float e0, e1;
+                    if ((j & 7) == 2 || (j & 7) == 5 || (j & 7) == 7) {
+                        exp2_poly_pair(x2, e0, e1);
+                    } else {
+                        float x0, x1;
+                        f2_split(x2, x0, x1);
+                        e0 = ex2(x0);
+                        e1 = ex2(x1);
                     }
-                    tmem_st16(slot + C::kColP + (c0 + bq * 32) / 2, pk);
+                    pk[j] = pack_bf16_rn(e0, e1);
+                    acc[j & 1] = f2_add(acc[j & 1], f2(e0, e1));
                 }
+                // P of these 32 columns lands on scores this thread has already read (and waited for)
+                tmem_st16(slot + C::p_col(cbase + 32 * cc), pk);
+                if (cc + 1 < kChunks) tmem_ld_wait();
             }
             tmem_st_wait();
             {
                 float a0, a1, b0, b1;
                 f2_split(acc[0], a0, a1);
                 f2_split(acc[1], b0, b1);
-                psum[s * 128 + r] = (a0 + a1) + (b0 + b1);
+                psum[(s * 2 + g) * 128 + r] = (a0 + a1) + (b0 + b1);
             }
             tc_fence_before();
             mbar_arrive(&p_full[s]);
@@ -408,7 +430,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 break;
             }
             tc_fence_after();
-            const float li = 1.f / psum[s * 128 + r];
+            const float li = 1.f / (psum[(s * 2) * 128 + r] + psum[(s * 2 + 1) * 128 + r]);
             const uint32_t slot = tmem + s * C::kSlot + lane_base;
             uint32_t outp[D / 2];
 #pragma unroll

@@ -7,18 +7,22 @@
 // X, so they commute with X. (2) Transposing the update gives W = Z^T with
 // W_0 = c k2, X^T = W k2^T and W <- T5(X^T) W / 4, where T5(X^T) is the same
 // polynomial taken in X^T. The kernel iterates in X^T (called X below)
-//   P1: X = W k2^T    P2: U = T1 X    P3: V = T3 X    P4: W = T5 W / 4
+//   P1: X = W k2^T    P2: -U = T1 (-X)    P3: -V = T3 (-X)    P4: W = T5 W / 4
 // (equal to the page's sequence in real arithmetic) and takes every left
-// factor from TMEM: W is the raw accumulator of the previous P4, and each T is
-// written back to TMEM by the epilogue that forms it (tf32-rounded). The right
-// factors live in shared memory as K-major lines: X, written once per
+// factor from TMEM: W is the raw accumulator of the previous P4; T1 = 7I - X
+// is written back over P1's accumulator by its epilogue (tf32-rounded); since
+// P2 and P3 multiply by -X, their accumulators -U and -V differ from
+// T3 = 15I - U and T5 = 13I - V only on the diagonal, which is all their
+// epilogues change (the other entries reach the MMA as fp32 bits). The right
+// factors live in shared memory as K-major lines: -X, written once per
 // iteration by the P1 epilogue column by column into the B half of the CTA
 // that owns the column (its own or, through distributed shared memory, the
 // peer's) -- X is symmetric only in exact arithmetic, and using its rows as
 // its columns loses accuracy on ill-conditioned k2 -- and, streamed from L2 one
-// 32-wide K atom at a time behind the previous product's MMAs, the rows of k2
-// (for P1) and the columns of W (for P4; the P4 epilogue writes W^T row-major
-// to scratch).
+// 32-wide K atom at a time behind the previous product's MMAs, the columns of W
+// (for P4; the P4 epilogue writes W^T row-major to scratch) and the last three
+// K atoms of k2's rows (for P1; its first five K atoms stay in shared memory
+// for the whole kernel).
 //
 // One head per cluster of two CTAs, one 2-CTA tcgen05 MMA per K step
 // (cta_group::2, kind::tf32, M = N = 256): CTA r holds rows 128r .. 128r+127 of
@@ -36,7 +40,6 @@
 #pragma once
 
 #include "sm100.cuh"
-#include "tc_pinv.cuh"
 
 namespace nys {
 namespace pair2 {
@@ -161,7 +164,11 @@ struct PinvPair {
     // barriers: bfull[8], bfree[8], mma_done, mma4_done, e_ready, wl_ready, drain, pro_full, cs_ready,
     // e_step[2]
     static constexpr uint32_t kOffMisc = kOffBar + 26 * 8;
-    static constexpr uint32_t kSmemNeed = kOffMisc + 64 + 1024;
+    // K atoms 0 .. kK2Resident - 1 of k2 (this CTA's B lines) stay in shared memory for every
+    // P1; the later P1s stream only the other atoms through the B buffer
+    static constexpr int kK2Resident = 5;
+    static constexpr uint32_t kOffK2r = (kOffMisc + 64 + 1023) / 1024 * 1024;
+    static constexpr uint32_t kSmemNeed = kOffK2r + kK2Resident * kAtomBytes + 1024;
     // more than half of the SM's shared memory: no other CTA (and no other TMEM user) shares the SM
     static constexpr uint32_t kSmemBytes = kSmemNeed < 200 * 1024 ? 200 * 1024 : kSmemNeed;
     static constexpr int kThreads = 320;
@@ -258,13 +265,17 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                         ok = wait_acq_cluster(wl_ready, (uint32_t)it & 1u);
                         fence_proxy_async_global();
                     }
-                    for (int kc = 0; kc < 8 && ok; ++kc) {
+                    for (int i = 0; i < 8 && ok; ++i) {
                         // K atom kc is free once the previous product (P3 before P4, P4 before the
-                        // next P1) has read it. bfree[kc] completes twice per iteration, after
-                        // P3 and after P4, and never runs ahead of these loads by more than one
-                        // phase, so its parity is exact.
+                        // next P1) has read it; the atoms are taken in the order those products
+                        // free them. bfree[kc] completes twice per iteration, after P3 and after
+                        // P4, and never runs ahead of these waits by more than one phase, so its
+                        // parity is exact: every completion is waited for, also for the resident
+                        // k2 atoms that the P1s do not stream.
+                        const int kc = (i & 1) ? 4 + (i >> 1) : (i >> 1);
                         ok = mbar_wait(&bfree[kc], p == 3 ? 0u : 1u);
                         if (!ok) break;
+                        if (p == 0 && kc < C::kK2Resident) continue;
                         if (leader) mbar_arrive_expect_tx(&bfull[kc], 2 * C::kAtomBytes);
                         tma_load_3d_pair(bbuf + kc * C::kAtomBytes, mp, bfull0 + 8 * kc, 32 * kc, r0, bh, keep_policy);
                     }
@@ -278,7 +289,8 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         if (leader) {
             const uint32_t bs = smem_u32(bbuf);
             bool ok = true;
-            uint32_t ne = 0, nf = 0;   // e_ready phases waited, streamed products issued
+            uint32_t ne = 0;        // e_ready phases waited
+            uint32_t fph = 0;       // bit kc: the parity of the next bfull[kc] phase to wait for
             // kernel_2: S2 = Q_l K_l^T from split tf32 operands, hi.hi + hi.lo + lo.hi
             ok = warp_all(wait_acq_cluster(e_ready, ne & 1u));
             ++ne;
@@ -317,14 +329,18 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                     }
                     tc_fence_after();
                     for (int i = 0; i < 8; ++i) {
-                        const int kc = (i & 1) ? 4 + (i >> 1) : (i >> 1);   // atoms 0, 4, 1, 5, ...
+                        // atoms 0, 4, 1, 5, ... (the later P1s: 0 .. 7, the resident ones first)
+                        const bool resident_p1 = p == 0 && it > 0;
+                        const int kc = resident_p1 ? i : ((i & 1) ? 4 + (i >> 1) : (i >> 1));
+                        const bool resident = resident_p1 && kc < C::kK2Resident;
                         if (stepped && (i & 3) == 0) {
                             ok = warp_all(wait_acq_cluster(&e_step[i >> 2], ns & 1u));
                             if (!ok) break;
                             tc_fence_after();
                         }
-                        if (streamed) {
-                            ok = warp_all(mbar_wait(&bfull[kc], nf & 1u));
+                        if (streamed && !resident) {
+                            ok = warp_all(mbar_wait(&bfull[kc], (fph >> kc) & 1u));
+                            fph ^= 1u << kc;
                             if (!ok) break;
                             tc_fence_after();
                         }
@@ -332,13 +348,13 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
 #pragma unroll
                             for (int kk = 0; kk < 4; ++kk)
                                 mma2_ts(d_col, a_col + kc * 32 + kk * 8,
-                                        smem_desc(bs + kc * C::kAtomBytes + kk * 32, 16, 1024, kLayoutSw128),
+                                        smem_desc((resident ? bs + C::kOffK2r : bs) + kc * C::kAtomBytes + kk * 32, 16,
+                                                  1024, kLayoutSw128),
                                         C::kIdesc, (i | kk) != 0 ? 1u : 0u);
                             if (p >= 2) commit2(&bfree[kc], 3);   // the producer refills this atom next
                         }
                     }
                     if (stepped) ++ns;
-                    if (streamed) ++nf;
                     if (ok && elect_one()) commit2(p == 3 ? mma4_done : mma_done, 3);
                 }
             }
@@ -395,16 +411,25 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         float coeff = 0.f;
         if (!failed) {
             // split Q_l and K_l into tf32 hi + lo in place (fp32 accuracy from three tf32 products)
+            // four independent chunks per step (2 * chunks is a multiple of 1024)
             const int chunks = nka * (int)(C::kAtomBytes / 16);   // 16-byte chunks per tile
-            for (int e = et; e < 2 * chunks; e += 256) {
-                const uint32_t base = e < chunks ? C::kOffAhi : C::kOffBhi;
-                const uint32_t off = base + (uint32_t)(e % chunks) * 16u;
-                float4* hi = reinterpret_cast<float4*>(bbuf + off);
-                float4* lo = reinterpret_cast<float4*>(bbuf + off + (C::kOffAlo - C::kOffAhi));
-                const float4 x = *hi;
-                const float4 xh = make_float4(tf32_rna(x.x), tf32_rna(x.y), tf32_rna(x.z), tf32_rna(x.w));
-                *hi = xh;
-                *lo = make_float4(x.x - xh.x, x.y - xh.y, x.z - xh.z, x.w - xh.w);
+#pragma unroll 1
+            for (int e0 = et; e0 < 2 * chunks; e0 += 4 * 256) {
+                uint32_t off[4];
+                float4 x[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + 256 * u;
+                    off[u] = (e < chunks ? C::kOffAhi : C::kOffBhi) + (uint32_t)(e % chunks) * 16u;
+                    x[u] = *reinterpret_cast<const float4*>(bbuf + off[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 xh = make_float4(tf32_rna(x[u].x), tf32_rna(x[u].y), tf32_rna(x[u].z), tf32_rna(x[u].w));
+                    *reinterpret_cast<float4*>(bbuf + off[u]) = xh;
+                    *reinterpret_cast<float4*>(bbuf + off[u] + (C::kOffAlo - C::kOffAhi)) =
+                        make_float4(x[u].x - xh.x, x[u].y - xh.y, x[u].z - xh.z, x[u].w - xh.w);
+                }
             }
             fence_proxy_async_shared();
             arrive_e();
@@ -467,9 +492,12 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 }
                 tmem_st32(R0 + lane_base + 32 * a, v);
 #pragma unroll
-                for (int c = 0; c < 8; ++c)
-                    *reinterpret_cast<uint4*>(bbuf + stage_off(a, c)) =
-                        make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 w4 = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                    *reinterpret_cast<uint4*>(bbuf + stage_off(a, c)) = w4;
+                    // the resident copy of k2's first K atoms (this CTA's B lines), for the later P1s
+                    if (a < C::kK2Resident) *reinterpret_cast<uint4*>(sm + C::kOffK2r + stage_off(a, c)) = w4;
+                }
             }
             rx[h * 128 + lrow] = rsum;   // rx is free: every thread read its row max before the last barrier
             fence_proxy_async_shared();   // the staged k2 rows feed the MMA and a TMA store
@@ -477,12 +505,13 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             // column sums over this CTA's rows (thread et: column et), max row sum of this CTA
             {
                 const int a = et >> 5, j = et & 31;
-                float cs = 0.f;
+                float c4[4] = {0.f, 0.f, 0.f, 0.f};   // four independent chains
 #pragma unroll 8
                 for (int l = 0; l < 128; ++l)
-                    cs += *reinterpret_cast<const float*>(
+                    c4[l & 3] += *reinterpret_cast<const float*>(
                         bbuf + (uint32_t)a * C::kAtomBytes + (uint32_t)l * 128u +
                         ((((uint32_t)j >> 2) ^ (uint32_t)(l & 7)) << 4) + (uint32_t)(j & 3) * 4u);
+                const float cs = (c4[0] + c4[1]) + (c4[2] + c4[3]);
                 cs_own[et] = cs;
                 st_remote(mapa(smem_u32(cs_peer + et), rank ^ 1u), cs);
                 const float rs = warp_max(et < 128 ? rx[et] + rx[128 + et] : 0.f);
@@ -548,8 +577,23 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 if (failed) break;
                 tc_fence_after();
                 const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
-                const float alpha = p == 0 ? -sigma : -1.f;
-                const float diag = p == 0 ? 7.f : (p == 1 ? 15.f : 13.f);
+                if (p == 1 || p == 2) {
+                    // the accumulator holds -U (-V): T3 = 15I - U (T5 = 13I - V) differs from it on
+                    // the diagonal only, which lies in atom diag_atom of this CTA's own column half
+                    if (diag_half) {
+                        uint32_t v[32];
+                        const uint32_t addr = d_col + lane_base + 32 * diag_atom;
+                        tmem_ld32(addr, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i == lane) v[i] = __float_as_uint(__uint_as_float(v[i]) + (p == 1 ? 15.f : 13.f));
+                        tmem_st32(addr, v);
+                    }
+                    arrive_step(0);   // P3 / P4 may start on every atom
+                    arrive_step(1);
+                    continue;
+                }
 #pragma unroll 1
                 for (int jj = 0; jj < 4; ++jj) {
                     const int a = 4 * h + jj;   // 32-column atom
@@ -568,38 +612,28 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                         }
                         continue;
                     }
+                    // p == 0: -X = -sigma D is the right factor of P2 and P3 as K-major lines:
+                    // column g = 32 a + i of X is line 32 (a % 4) + i of CTA a / 4 (= h), and this
+                    // thread's row is K position `row` of every line
                     float e[32];
-                    if (p == 0) {
-                        // X = sigma D is the right factor of P2 and P3 as K-major lines: column
-                        // g = 32 a + i of X is line 32 (a % 4) + i of CTA a / 4 (= h), and this
-                        // thread's row is K position `row` of every line
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) e[i] = sigma * __uint_as_float(v[i]);
-                        const uint32_t base = x_dst + k_off + (uint32_t)(a & 3) * 4096u;
-                        if (x_local) {
+                    for (int i = 0; i < 32; ++i) e[i] = tf32_rna(-sigma * __uint_as_float(v[i]));
+                    const uint32_t base = x_dst + k_off + (uint32_t)(a & 3) * 4096u;
+                    if (x_local) {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                st_local(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), tf32_rna(e[i]));
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                st_remote(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), tf32_rna(e[i]));
-                        }
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) e[i] = -e[i];
+                        for (int i = 0; i < 32; ++i) st_local(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), e[i]);
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) e[i] = alpha * __uint_as_float(v[i]);
+                        for (int i = 0; i < 32; ++i) st_remote(base + i * 128 + ((xl ^ (uint32_t)(i & 7)) << 4), e[i]);
                     }
-                    // T = diag I + alpha D, back into TMEM as the next left factor
+                    // T1 = 7I - X, back into TMEM as P2's left factor
                     if (diag_half && a == diag_atom) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) e[i] += i == lane ? diag : 0.f;
+                        for (int i = 0; i < 32; ++i) e[i] += i == lane ? 7.f : 0.f;
                     }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(tf32_rna(e[i]));
                     tmem_st32(d_col + lane_base + 32 * a, v);
-                    if ((p == 1 || p == 2) && (jj & 1)) arrive_step(jj >> 1);   // P3 / P4 may start on these atoms
                 }
                 if (p == 3) {
                     if (!last_it) arrive_wl();

@@ -12,10 +12,15 @@
 //
 // The iteration runs on W = Z^T, as in the CTA-pair kernel for m = 256 (the page's sequence
 // transposed; equal in real arithmetic):
-//   P1: X = W k2^T     A = W (TMEM, the raw previous P4 accumulator), B = k2 as K-major lines
-//   P2: -U = T1 (-X)   A = T1 (TMEM, written by the P1 epilogue), B = -X, MN-major
-//   P3: -V = T3 (-X)   A = T3 = -U + 15 I (the P2 accumulator, diagonal added in place)
-//   P4: W' = T5 W / 4  A = T5 = -V + 13 I, B = W's rows, MN-major
+//   P1: X = W k2^T          A = W (R0: the raw previous P4 accumulator), B = k2 as K-major
+//                           lines, D -> R1
+//   P2: T3 = 15I + T1 (-X)  A = T1 (R1, written over P1's accumulator by its epilogue),
+//                           B = -X, MN-major; D -> R2, which holds 15 I beforehand
+//   P3: T5 = 13I + T3 (-X)  A = R2, B = -X; D -> R3, which holds 13 I beforehand
+//   P4: W' = T5 W / 4       A = R3, B = W's rows, MN-major; D -> R0
+// so only P1 has an epilogue on the chain: P2 -> P3 -> P4 wait only for the previous
+// product to complete. The P1 epilogue also sets R2 and R3 to 15 I and 13 I; the P4
+// epilogue, which runs beside the next P1, writes W's rows.
 // k2 stays in shared memory for all P1s; -X is written by the P1 epilogue, W's rows by the
 // P4 epilogue of the iteration before (or by the prologue: k2's rows, W_0 = c k2 with c folded
 // into the scales). Nothing is streamed through L2. Scales are folded into the epilogues as
@@ -27,7 +32,6 @@
 #pragma once
 
 #include "sm100.cuh"
-#include "tc_pinv.cuh"
 
 namespace nys {
 
@@ -83,6 +87,7 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
     uint64_t* mma_done = bars + 2;    // kernel_2, P1..P3 accumulators complete
     uint64_t* mma4_done = bars + 3;   // P4 accumulator complete
     uint64_t* drain = bars + 4;       // every MMA issued has completed (32 lanes)
+    uint64_t* chain_done = bars + 5;  // P2 / P3 complete (waited by the MMA warp)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -96,17 +101,18 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
         mbar_init(mma_done, 1);
         mbar_init(mma4_done, 1);
         mbar_init(drain, 32);
+        mbar_init(chain_done, 1);
         fence_mbar_init();
     }
     if (warp == 9) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t R0 = tmem, R1 = tmem + 128;
+    const uint32_t R0 = tmem, R1 = tmem + 128, R2 = tmem + 256, R3 = tmem + 384;
 
     if (warp == 8) {
         // ------------------------------------------------ TMA producer: this CTA's landmarks
@@ -149,23 +155,29 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
             }
             if (elect_one()) mma_commit(mma_done);
         }
+        uint32_t nc = 0;   // chain_done phases waited
         for (int it = 0; it < n_iter && ok; ++it) {
             for (int p = 0; p < 4 && ok; ++p) {
-                // P2, P3, P4 (and the first P1) wait for their left factor and right factor
-                if (p != 0 || it == 0) {
+                // the first P1 waits for the prologue, P2 for the P1 epilogue (T1, -X, and R2 / R3
+                // preset); P3 and P4 for the product before them
+                if ((p == 0 && it == 0) || p == 1) {
                     ok = warp_all(mbar_wait(e_ready, ne & 1u));
                     ++ne;
-                    if (!ok) break;
+                } else if (p >= 2) {
+                    ok = warp_all(mbar_wait(chain_done, nc & 1u));
+                    ++nc;
                 }
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t a_col = (p == 0 || p == 2) ? R0 : R1;
-                const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
+                const uint32_t a_col = p == 0 ? R0 : (p == 1 ? R1 : (p == 2 ? R2 : R3));
+                const uint32_t d_col = p == 0 ? R1 : (p == 1 ? R2 : (p == 2 ? R3 : R0));
+                const bool preset = p == 1 || p == 2;   // accumulate onto 15 I / 13 I
                 if (elect_one()) {
 #pragma unroll 1
                     for (int ka = 0; ka < 4; ++ka)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t acc = (ka | kk) != 0 ? 1u : 0u;
+                            const uint32_t acc = (preset || (ka | kk) != 0) ? 1u : 0u;
                             if (p == 0) {
                                 mma_tf32_ts(d_col, a_col + ka * 32 + kk * 8,
                                             smem_desc(bs + C::kOffK2 + ka * C::kAtom + kk * 32, 16, 1024, kLayoutSw128),
@@ -179,7 +191,7 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
                             }
                         }
                 }
-                if (elect_one()) mma_commit(p == 3 ? mma4_done : mma_done);
+                if (elect_one()) mma_commit(p == 0 ? mma_done : (p == 3 ? mma4_done : chain_done));
             }
         }
         // every MMA issued here has completed before the TMEM is released: one commit per lane
@@ -197,6 +209,18 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
         // the diagonal element (lrow, lrow) lies in this half, in 32-column atom diag_jj of it
         const bool diag_half = (lrow >> 6) == h;
         const int diag_jj = (lrow >> 5) & 1;
+        // v I into this thread's row of TMEM region `base` (its 64 columns): the accumulator
+        // preset of P2 (15 I) and P3 (13 I)
+        auto preset_diag = [&](uint32_t base, float val) {
+#pragma unroll 1
+            for (int jj = 0; jj < 2; ++jj) {
+                uint32_t v[32];
+                const bool here = diag_half && jj == diag_jj;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = (here && i == lane) ? __float_as_uint(val) : 0u;
+                tmem_st32(base + lane_base + 64 * h + 32 * jj, v);
+            }
+        };
         auto arrive_e = [&]() {
             tc_fence_before();
             __syncwarp();
@@ -216,17 +240,26 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
         float coeff = 0.f;
         if (!failed) {
             // split Q_l and K_l into tf32 hi + lo in place (fp32 accuracy from three tf32 products)
+            // four independent chunks per step (2 * chunks is a multiple of 1024)
             const int chunks = nka * (int)(C::kAtom / 16);
-            for (int e = et; e < 2 * chunks; e += 256) {
-                const uint32_t base = e < chunks ? C::kOffQhi : C::kOffKhi;
-                const uint32_t lo_off = e < chunks ? C::kOffQlo - C::kOffQhi : C::kOffKlo - C::kOffKhi;
-                const uint32_t off = base + (uint32_t)(e % chunks) * 16u;
-                float4* hi = reinterpret_cast<float4*>(sm + off);
-                float4* lo = reinterpret_cast<float4*>(sm + off + lo_off);
-                const float4 x = *hi;
-                const float4 xh = make_float4(tf32_rna(x.x), tf32_rna(x.y), tf32_rna(x.z), tf32_rna(x.w));
-                *hi = xh;
-                *lo = make_float4(x.x - xh.x, x.y - xh.y, x.z - xh.z, x.w - xh.w);
+            static_assert(C::kOffQlo - C::kOffQhi == C::kOffKlo - C::kOffKhi, "hi / lo distance");
+#pragma unroll 1
+            for (int e0 = et; e0 < 2 * chunks; e0 += 4 * 256) {
+                uint32_t off[4];
+                float4 x[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + 256 * u;
+                    off[u] = (e < chunks ? C::kOffQhi : C::kOffKhi) + (uint32_t)(e % chunks) * 16u;
+                    x[u] = *reinterpret_cast<const float4*>(sm + off[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float4 xh = make_float4(tf32_rna(x[u].x), tf32_rna(x[u].y), tf32_rna(x[u].z), tf32_rna(x[u].w));
+                    *reinterpret_cast<float4*>(sm + off[u]) = xh;
+                    *reinterpret_cast<float4*>(sm + off[u] + (C::kOffQlo - C::kOffQhi)) =
+                        make_float4(x[u].x - xh.x, x[u].y - xh.y, x[u].z - xh.z, x[u].w - xh.w);
+                }
             }
             fence_proxy_async_shared();
             arrive_e();
@@ -308,12 +341,14 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
             // per head: the largest of each
             if (et < 128) {
                 const int a = et >> 5, j = et & 31;
-                float s = 0.f;
+                float c4[4] = {0.f, 0.f, 0.f, 0.f};   // four independent chains
 #pragma unroll 8
                 for (int l = 0; l < 128; ++l)
-                    s += *reinterpret_cast<const float*>(sm + C::kOffK2 + (uint32_t)a * C::kAtom + (uint32_t)l * 128u +
-                                                        ((((uint32_t)j >> 2) ^ (uint32_t)(l & 7)) << 4) +
-                                                        (uint32_t)(j & 3) * 4u);
+                    c4[l & 3] += *reinterpret_cast<const float*>(sm + C::kOffK2 + (uint32_t)a * C::kAtom +
+                                                                (uint32_t)l * 128u +
+                                                                ((((uint32_t)j >> 2) ^ (uint32_t)(l & 7)) << 4) +
+                                                                (uint32_t)(j & 3) * 4u);
+                const float s = (c4[0] + c4[1]) + (c4[2] + c4[3]);
                 const float rs = rx[et] + rx[128 + et];
                 // warps 0-3 hold columns / rows 32 w .. 32 w + 31
                 const float wc = warp_max(s), wr = warp_max(rs);
@@ -362,28 +397,12 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
             const float sigma = it == 0 ? coeff : (it == 1 ? 0.25f * coeff : 0.25f);
             const float lambda = it == 0 ? 0.25f * coeff : 0.25f;
             const bool last_it = it + 1 == n_iter;
-            for (int p = 0; p < 4 && !failed; ++p) {
+            for (int p = 0; p < 4 && !failed; p += 3) {   // the P1 and P4 epilogues
                 const bool ok = p == 3 ? mbar_wait(mma4_done, (n4++) & 1u) : mbar_wait(mma_done, (nd++) & 1u);
                 failed = group_any(!ok, 3, 256);
                 if (failed) break;
                 tc_fence_after();
-                const uint32_t d_col = (p == 0 || p == 2) ? R1 : R0;
-                if (p == 1 || p == 2) {
-                    // the accumulator holds -U (-V): T3 = 15I - U (T5 = 13I - V) needs only its diagonal
-                    if (diag_half) {
-                        uint32_t v[32];
-                        const uint32_t addr = d_col + lane_base + 64 * h + 32 * diag_jj;
-                        tmem_ld32(addr, v);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            if (i == lane) v[i] = __float_as_uint(__uint_as_float(v[i]) + (p == 1 ? 15.f : 13.f));
-                        tmem_st32(addr, v);
-                        tmem_st_wait();
-                    }
-                    arrive_e();
-                    continue;
-                }
+                const uint32_t d_col = p == 0 ? R1 : R0;
                 if (p == 3) {
                     // W' = lambda D: the next P4's right factor (this thread's row, MN-major) or, at
                     // the end, Z = W'^T (column lrow of Z's head block)
@@ -437,6 +456,11 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
                     for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(tf32_rna(e[i]));
                     tmem_st32(addr, v);
                 }
+                // R2 / R3 back to 15 I / 13 I: their last readers, the previous P3 and P4, completed
+                // before this P1 (the tensor pipe runs in issue order). Written here, while the
+                // tensor pipe is idle: stores that overlap an MMA run several times slower
+                preset_diag(R2, 15.f);
+                preset_diag(R3, 13.f);
                 tmem_st_wait();
                 fence_proxy_async_shared();   // -X (and the previous P4 epilogue's W rows) feed the MMA
                 arrive_e();
@@ -448,7 +472,7 @@ pinv_res_kernel(const __grid_constant__ PinvResMaps maps, const PinvResParams pr
     __syncthreads();
     if (warp == 9) {
         tc_fence_after();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, 512);
     }
 }
 

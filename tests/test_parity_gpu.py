@@ -212,6 +212,15 @@ def test_stages_against_oracle(nys, oracle_mod, name):
         ma, rel = errors(st["z"][b, h], ost[idx]["z"])
         note(f"stage z {name} head {idx}", ma, rel)
         assert rel < (1e-4 if w.dtype == "f32" else Z_STAGE_BF16), ("z", rel)
+        # W = Z k3V, the output pass's factor (walkthrough 2.6, reassociated): against the fp64
+        # product of this run's own Z and k3V, relative to the product of their magnitudes, so
+        # that it measures the W kernel alone (fp32 FMAs at m = 64; tf32 operands, 2^-11
+        # relative rounding each, on the tensor-core W kernel at m = 128 / 256)
+        zk = st["z"][b, h] @ st["k3v"][b, h]
+        scale = np.linalg.norm(np.abs(st["z"][b, h]) @ np.abs(st["k3v"][b, h]))
+        werr = float(np.linalg.norm(st["w"][b, h] - zk) / scale)
+        note(f"stage w {name} head {idx}", float(np.max(np.abs(st["w"][b, h] - zk))), werr)
+        assert werr < (1e-6 if w.dtype == "f32" else 2e-3), ("w", werr)
 
 
 def test_mask_padded_keys_do_not_contribute(nys):
