@@ -685,10 +685,21 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
     rc = launch_k3v_tc<D>(p, st, ql16, k, v, mbits, po, pm, pl, k3v_sms, split_scale(D) * kLog2e, st.aux);
     if (rc != NYS_OK) return rc;
     {
+        // a programmatic dependent of kernel_3 V: launched while its last CTAs finish
         const long long threads = (long long)BH * m * (D / 4);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)((threads + 255) / 256));
+        cfg.blockDim = dim3(256);
+        cfg.stream = st.aux;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
         ProfScope ps(K_COMBINE, st.aux);
-        k3v_combine_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st.aux>>>(po, pm, pl, k3v, BH, m, D,
-                                                                                   p.splits);
+        if (cudaLaunchKernelEx(&cfg, k3v_combine_kernel, (const float*)po, (const float*)pm, (const float*)pl, k3v,
+                               BH, m, (int)D, p.splits) != cudaSuccess)
+            return NYS_ERR_CUDA;
     }
     if (cudaEventRecord(st.join, st.aux) != cudaSuccess) return NYS_ERR_CUDA;
     if (cudaStreamWaitEvent(s, st.join, 0) != cudaSuccess) return NYS_ERR_CUDA;

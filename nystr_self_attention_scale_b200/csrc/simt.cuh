@@ -424,13 +424,16 @@ k3v_partial_simt_kernel(const float* __restrict__ ql, const T* __restrict__ k, c
 
 // Merge the key-split partials: k3v[j] = sum_s e^{M_s - M} O_s / sum_s e^{M_s - M} l_s.
 // One thread per (head, landmark row, 4 columns), one pass: the splits are taken
-// eight at a time with all their loads in flight together, and the running sums
+// four at a time with all their loads in flight together, and the running sums
 // are rescaled when a later group raises the maximum. The split order is fixed,
-// so the result is deterministic.
-__global__ void __launch_bounds__(256)
+// so the result is deterministic. Four CTAs fit per SM, so the grid of the
+// supported sizes runs in one wave. May be launched as a programmatic dependent of
+// the kernel that writes the partials: it waits for that grid before reading them.
+__global__ void __launch_bounds__(256, 4)
 k3v_combine_kernel(const float* __restrict__ part_o, const float* __restrict__ part_m,
                    const float* __restrict__ part_l, float* __restrict__ k3v, int BH, int m, int d, int splits) {
-    constexpr int G = 8;
+    constexpr int G = 4;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int q = d / 4;
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= (long long)BH * m * q) return;

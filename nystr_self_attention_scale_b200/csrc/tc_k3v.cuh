@@ -477,6 +477,8 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         }
     }
 
+    // the split merge may launch now (it waits for this grid's completion before reading)
+    griddep_launch_dependents();
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

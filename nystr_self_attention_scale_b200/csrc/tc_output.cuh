@@ -72,7 +72,7 @@ struct OutTc {
     static constexpr uint32_t kOffPsum = kOffOut + kOutBytes;   // [2 slots][2 groups][128] partial row sums
     static constexpr uint32_t kOffXch = kOffPsum + 2 * 2 * 128 * 4;   // [2 slots][2 groups][128] partial row maxima
     static constexpr uint32_t kOffBar = kOffXch + 2 * 2 * 128 * 4;
-    static constexpr int kNumBars = 20;
+    static constexpr int kNumBars = 22;
     static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;  // tmem base, abort flag
     static constexpr uint32_t kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -110,6 +110,8 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     uint64_t* t_full = bars + 15;    // Toeplitz matrix built (128 arrivals)
     uint64_t* v_full = bars + 16;    // [2] V halo landed
     uint64_t* v_empty = bars + 18;   // [2] V stage reusable (its conv MMA completed)
+    // [2] the second softmax group has loaded the last S columns that O_conv overlaps (m = 256)
+    uint64_t* conv_free = bars + 20;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
     float* psum = reinterpret_cast<float*>(sm + C::kOffPsum);
@@ -133,6 +135,7 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
             mbar_init(&slot_free[b], 128);
             mbar_init(&v_full[b], 1);
             mbar_init(&v_empty[b], 1);
+            mbar_init(&conv_free[b], 128);
         }
         mbar_init(const_full, 1);
         mbar_init(t_full, 128);
@@ -251,15 +254,11 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         auto issue_O = [&](int j) -> bool {
             const int s = j & 1, st = j % C::kStages;
             const uint32_t slot = tmem + s * C::kSlot;
-            // O_conv shares TMEM columns with the second half of S: the conv product waits for P too
-            if (!wait(&p_full[s], (j >> 1) & 1)) return false;
-            tc_fence_after();
-            if (elect_one()) {
-#pragma unroll
-                for (int k = 0; k < M / 16; ++k)   // landmarks 16k .. 16k+15: 8 packed P columns
-                    mma_bf16_ts(slot + C::kColOatt, slot + C::p_col(16 * k), descWt(k), C::kIdPW, k > 0);
-            }
+            // the conv product first: it does not need P, so it runs while the softmax finishes.
+            // At m = 256 O_conv shares TMEM columns with the last 64 S columns of the second
+            // softmax group, which that group has loaded by the time it arrives on conv_free
             if (prm.conv_w != nullptr) {
+                if (M == 256 && !wait(&conv_free[s], (j >> 1) & 1)) return false;
                 if (!wait(&v_full[st], (j / C::kStages) & 1)) return false;
                 tc_fence_after();
                 if (elect_one()) {
@@ -268,6 +267,13 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                         mma_bf16_ss(slot + C::kColOconv, descT(k), descV(st, k), C::kIdConv, k > 0);
                 }
                 if (elect_one()) mma_commit(&v_empty[st]);
+            }
+            if (!wait(&p_full[s], (j >> 1) & 1)) return false;
+            tc_fence_after();
+            if (elect_one()) {
+#pragma unroll
+                for (int k = 0; k < M / 16; ++k)   // landmarks 16k .. 16k+15: 8 packed P columns
+                    mma_bf16_ts(slot + C::kColOatt, slot + C::p_col(16 * k), descWt(k), C::kIdPW, k > 0);
             }
             if (elect_one()) mma_commit(&o_full[s]);
             return true;
@@ -371,6 +377,11 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 // P of these 32 columns lands on scores this thread has already read (and waited for)
                 tmem_st16(slot + C::p_col(cbase + 32 * cc), pk);
                 if (cc + 1 < kChunks) tmem_ld_wait();
+                if (M == 256 && g == 1 && cc == kChunks - 2) {
+                    // every S column of this group is in registers: O_conv may overwrite the last 64
+                    tc_fence_before();
+                    mbar_arrive(&conv_free[s]);
+                }
             }
             tmem_st_wait();
             {
