@@ -439,15 +439,19 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
         if (!failed) {
             tc_fence_after();
             // row max: this thread's 128 columns, then the other half's through shared memory
+            // (the prologue's passes over the 128 columns take two atoms per TMEM wait)
             float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-            for (int jj = 0; jj < 4; ++jj) {
-                uint32_t v[32];
-                tmem_ld32(R1 + lane_base + 32 * (4 * h + jj), v);
+            for (int jp = 0; jp < 2; ++jp) {
+                uint32_t v[2][32];
+                tmem_ld32(R1 + lane_base + 32 * (4 * h + 2 * jp), v[0]);
+                tmem_ld32(R1 + lane_base + 32 * (4 * h + 2 * jp + 1), v[1]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    mq[i & 3] = max3(mq[i & 3], __uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                for (int e = 0; e < 2; ++e)
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        mq[i & 3] = max3(mq[i & 3], __uint_as_float(v[e][2 * i]), __uint_as_float(v[e][2 * i + 1]));
             }
             rx[h * 128 + lrow] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
             named_barrier(3, 256);
@@ -455,18 +459,22 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             // exponentials, kept in place in TMEM; their row sum
             float ssum = 0.f;
 #pragma unroll 1
-            for (int jj = 0; jj < 4; ++jj) {
-                uint32_t v[32];
-                const uint32_t addr = R1 + lane_base + 32 * (4 * h + jj);
-                tmem_ld32(addr, v);
+            for (int jp = 0; jp < 2; ++jp) {
+                uint32_t v[2][32];
+                const uint32_t addr = R1 + lane_base + 32 * (4 * h + 2 * jp);
+                tmem_ld32(addr, v[0]);
+                tmem_ld32(addr + 32, v[1]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float e = __expf(__uint_as_float(v[i]) - mx);
-                    ssum += e;
-                    v[i] = __float_as_uint(e);
+                for (int e2 = 0; e2 < 2; ++e2) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float e = __expf(__uint_as_float(v[e2][i]) - mx);
+                        ssum += e;
+                        v[e2][i] = __float_as_uint(e);
+                    }
+                    tmem_st32(addr + 32 * e2, v[e2]);
                 }
-                tmem_st32(addr, v);
             }
             tmem_st_wait();
             sx[h * 128 + lrow] = ssum;
@@ -477,26 +485,31 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             float rsum = 0.f;
             float* k2t_col = prm.k2t + (size_t)bh * M * M + row;
 #pragma unroll 1
-            for (int jj = 0; jj < 4; ++jj) {
-                const int a = 4 * h + jj;
-                uint32_t v[32];
-                tmem_ld32(R1 + lane_base + 32 * a, v);
+            for (int jp = 0; jp < 2; ++jp) {
+                uint32_t vv[2][32];
+                tmem_ld32(R1 + lane_base + 32 * (4 * h + 2 * jp), vv[0]);
+                tmem_ld32(R1 + lane_base + 32 * (4 * h + 2 * jp + 1), vv[1]);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float pv = __uint_as_float(v[i]) * inv;
-                    rsum += pv;
-                    const float pr = tf32_rna(pv);
-                    v[i] = __float_as_uint(pr);
-                    k2t_col[(size_t)(32 * a + i) * M] = pr;
-                }
-                tmem_st32(R0 + lane_base + 32 * a, v);
+                for (int e2 = 0; e2 < 2; ++e2) {
+                    const int a = 4 * h + 2 * jp + e2;
+                    uint32_t* v = vv[e2];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    const uint4 w4 = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-                    *reinterpret_cast<uint4*>(bbuf + stage_off(a, c)) = w4;
-                    // the resident copy of k2's first K atoms (this CTA's B lines), for the later P1s
-                    if (a < C::kK2Resident) *reinterpret_cast<uint4*>(sm + C::kOffK2r + stage_off(a, c)) = w4;
+                    for (int i = 0; i < 32; ++i) {
+                        const float pv = __uint_as_float(v[i]) * inv;
+                        rsum += pv;
+                        const float pr = tf32_rna(pv);
+                        v[i] = __float_as_uint(pr);
+                        k2t_col[(size_t)(32 * a + i) * M] = pr;
+                    }
+                    tmem_st32(R0 + lane_base + 32 * a, vv[e2]);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const uint4 w4 = make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                        *reinterpret_cast<uint4*>(bbuf + stage_off(a, c)) = w4;
+                        // the resident copy of k2's first K atoms (this CTA's B lines), for the later P1s
+                        if (a < C::kK2Resident) *reinterpret_cast<uint4*>(sm + C::kOffK2r + stage_off(a, c)) = w4;
+                    }
                 }
             }
             rx[h * 128 + lrow] = rsum;   // rx is free: every thread read its row max before the last barrier
@@ -542,8 +555,8 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 // the exact-coefficient option drops the row factor (softmax rows sum to 1)
                 coeff = 1.f / (mc * (prm.inv_init == NYS_INV_INIT_EXACT ? 1.f : fmaxf(rmax[0], rmax[1])));
             }
-            if (et == 0) tma_store_wait_all<0>();
             if (n_iter == 0 && !failed) {
+                if (et == 0) tma_store_wait_all<0>();
                 // Z = c k2^T, from the staged rows
                 float* zc = prm.z_out + (size_t)bh * M * M + row;
 #pragma unroll 1
@@ -560,8 +573,14 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 }
             } else if (!failed) {
                 tmem_st_wait();
-                arrive_e();     // W_0 in TMEM, k2 lines in the B buffer
+                arrive_e();     // W_0 in TMEM, k2 lines in the B buffer: the first P1 may start
+                // the TMA store of k2's rows only reads the B buffer, as the first P1 does; it is
+                // complete before the producer reads k2 back (wl_ready) and before the P1
+                // epilogue, behind the next named barrier, overwrites the B buffer
+                if (et == 0) tma_store_wait_all<0>();
                 arrive_wl();    // k2 and k2^T in global memory
+            } else if (et == 0) {
+                tma_store_wait_all<0>();
             }
         }
 
