@@ -480,10 +480,9 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             sx[h * 128 + lrow] = ssum;
             named_barrier(3, 256);
             const float inv = 1.f / (sx[lrow] + sx[128 + lrow]);
-            // k2 = e / sum: into TMEM as W_0 (R0), into the B buffer as the first P1's right
-            // factor (this CTA's rows are its own B lines), and transposed into global k2^T
+            // k2 = e / sum: into TMEM as W_0 (R0) and into the B buffer as the first P1's right
+            // factor (this CTA's rows are its own B lines); k2^T goes to global memory later
             float rsum = 0.f;
-            float* k2t_col = prm.k2t + (size_t)bh * M * M + row;
 #pragma unroll 1
             for (int jp = 0; jp < 2; ++jp) {
                 uint32_t vv[2][32];
@@ -500,7 +499,6 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                         rsum += pv;
                         const float pr = tf32_rna(pv);
                         v[i] = __float_as_uint(pr);
-                        k2t_col[(size_t)(32 * a + i) * M] = pr;
                     }
                     tmem_st32(R0 + lane_base + 32 * a, vv[e2]);
 #pragma unroll
@@ -538,11 +536,6 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             }
             __syncwarp();
             if (lane == 0) arrive_cluster(mapa(smem_u32(cs_ready), rank ^ 1u));
-            // the rows of k2 go to global memory for the later P1s (TMA store of the staging)
-            if (et == 0) {
-                for (int a = 0; a < 8; ++a) tma_store_3d(&maps.k2, bbuf + a * C::kAtomBytes, 32 * a, r0, bh);
-                tma_store_commit();
-            }
             const bool ok = wait_acq_cluster(cs_ready, 0);
             failed = group_any(!ok, 3, 256);
             if (!failed) {
@@ -556,7 +549,6 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 coeff = 1.f / (mc * (prm.inv_init == NYS_INV_INIT_EXACT ? 1.f : fmaxf(rmax[0], rmax[1])));
             }
             if (n_iter == 0 && !failed) {
-                if (et == 0) tma_store_wait_all<0>();
                 // Z = c k2^T, from the staged rows
                 float* zc = prm.z_out + (size_t)bh * M * M + row;
 #pragma unroll 1
@@ -574,13 +566,34 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             } else if (!failed) {
                 tmem_st_wait();
                 arrive_e();     // W_0 in TMEM, k2 lines in the B buffer: the first P1 may start
+                // the rows of k2 go to global memory for the later P1s (TMA store of the staging),
+                // issued only now: a cluster-scope release waits for the issuing thread's
+                // outstanding bulk copies, and the first P1's release must not wait for this one
+                if (et == 0) {
+                    for (int a = 0; a < 8; ++a) tma_store_3d(&maps.k2, bbuf + a * C::kAtomBytes, 32 * a, r0, bh);
+                    tma_store_commit();
+                }
+                // k2^T (the first P4's right factor, streamed back by TMA): this thread's row of
+                // k2 from the staged B lines into column `row` of k2^T. Written only now, so that
+                // the cluster-scope release above does not wait for these global stores.
+                float* k2t_col = prm.k2t + (size_t)bh * M * M + row;
+#pragma unroll 1
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int a = 4 * h + jj;
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        const float4 f4 = *reinterpret_cast<const float4*>(bbuf + stage_off(a, c));
+                        k2t_col[(size_t)(32 * a + 4 * c) * M] = f4.x;
+                        k2t_col[(size_t)(32 * a + 4 * c + 1) * M] = f4.y;
+                        k2t_col[(size_t)(32 * a + 4 * c + 2) * M] = f4.z;
+                        k2t_col[(size_t)(32 * a + 4 * c + 3) * M] = f4.w;
+                    }
+                }
                 // the TMA store of k2's rows only reads the B buffer, as the first P1 does; it is
                 // complete before the producer reads k2 back (wl_ready) and before the P1
                 // epilogue, behind the next named barrier, overwrites the B buffer
                 if (et == 0) tma_store_wait_all<0>();
                 arrive_wl();    // k2 and k2^T in global memory
-            } else if (et == 0) {
-                tma_store_wait_all<0>();
             }
         }
 

@@ -7,8 +7,9 @@
 //   B = kernel_3 V [m, d], staged by the threads in the MN-major tf32 layout (rows of 32 values
 //       along d, 32-byte granules swizzled by row % 4), rounded to tf32 (nearest, ties away)
 //   D = [128, d] fp32 in TMEM: m / 8 MMAs of K = 8
-// The epilogue (one thread per row) writes W in fp32 ([m, d] per head) and W^T in bf16
-// ([d, m] per head, the output pass's operand). A and B are rounded to tf32 (10-bit
+// The epilogue (warp w: TMEM lanes 32 (w % 4), columns 32 (w / 4) ..; one thread per row and
+// 32 columns) writes W in fp32 ([m, d] per head) and W^T in bf16 ([d, m] per head, the
+// output pass's operand). A and B are rounded to tf32 (10-bit
 // mantissa); the output pass reads W^T in bf16 (7-bit mantissa).
 //
 // The output pass is launched as a programmatic dependent of this kernel: it starts its
@@ -21,7 +22,7 @@ namespace nys {
 
 template <int D>
 struct WTc {
-    static constexpr int kThreads = 128;
+    static constexpr int kThreads = 512;   // staging: m * D / 4 float4 over all threads, 8 each at most
     static constexpr uint32_t kAtom = 128 * 128;               // 128 rows x 32 fp32 of Z: 16 KB
     static constexpr uint32_t kMnAtom = 1024;                  // 8 K rows x 32 columns of B
     static constexpr uint32_t kKGroup = (D / 32) * kMnAtom;    // 8 K rows x D columns of B
@@ -68,7 +69,7 @@ w_tc_kernel(const __grid_constant__ CUtensorMap map_z, const float* __restrict__
     }
     // B = kernel_3 V of this head: float4 i of the [m, D] matrix is row k = i / (D / 4), columns
     // 4 (i % (D / 4)) .. + 3, i.e. 16-byte chunk (i % 8) of the 32-column atom (i % (D / 4)) / 8
-    // (8 loads in flight per thread: m * D / 4 is 1024, 2048 or 4096, a multiple of 8 * 128)
+    // (up to 8 loads in flight per thread, one round at m * D / 4 = 4096; the tail is predicated)
     {
         constexpr int kBatch = 8;
         const float4* src = reinterpret_cast<const float4*>(k3v + (size_t)bh * m * D);
@@ -77,10 +78,14 @@ w_tc_kernel(const __grid_constant__ CUtensorMap map_z, const float* __restrict__
         for (int i0 = tid; i0 < total; i0 += kBatch * C::kThreads) {
             float4 x[kBatch];
 #pragma unroll
-            for (int u = 0; u < kBatch; ++u) x[u] = __ldg(src + i0 + u * C::kThreads);
+            for (int u = 0; u < kBatch; ++u) {
+                const int i = i0 + u * C::kThreads;
+                x[u] = i < total ? __ldg(src + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
 #pragma unroll
             for (int u = 0; u < kBatch; ++u) {
                 const int i = i0 + u * C::kThreads, k = i / (D / 4), c4 = i % (D / 4);
+                if (i >= total) break;
                 const uint32_t off = C::off_b(m) + (uint32_t)(k >> 3) * C::kKGroup +
                                      (uint32_t)(c4 >> 3) * C::kMnAtom + mn32_chunk(k & 7, c4 & 7);
                 *reinterpret_cast<float4*>(sm + off) =
@@ -114,15 +119,15 @@ w_tc_kernel(const __grid_constant__ CUtensorMap map_z, const float* __restrict__
     griddep_launch_dependents();
     ok = __syncthreads_and(ok) != 0;
     if (ok) ok = mbar_wait(mma_done, 0);
-    if (ok) {
+    if (ok && warp < 4 * (D / 32)) {
         tc_fence_after();
-        const int r = row0 + 32 * warp + lane;   // this thread's row of W (TMEM lane)
+        const int q = warp & 3, j = warp >> 2;      // TMEM lane quadrant, 32-column block
+        const int r = row0 + 32 * q + lane;         // this thread's row of W (TMEM lane)
         float* wr = w + ((size_t)bh * m + r) * D;
         __nv_bfloat16* wtc = wt16 + (size_t)bh * D * m + r;
-#pragma unroll
-        for (int j = 0; j < D / 32; ++j) {
+        {
             uint32_t v[32];
-            tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + 32 * j, v);
+            tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + 32 * j, v);
             tmem_ld_wait();
 #pragma unroll
             for (int c = 0; c < 8; ++c)
