@@ -623,27 +623,20 @@ int launch_bf16(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, co
             // as many CTAs of eight warps per SM as fit, striding over the landmarks, and just
             // enough of them that every warp takes the same number of landmarks (no partly-filled
             // last round)
-            const bool deep = (n / m) / rows_per_instr >= 16;   // 16 loads per lane per round
-            static int per_sm[2][kMaxDevices] = {};
+            static int per_sm[kMaxDevices] = {};
             int dev = 0;
             cudaGetDevice(&dev);
-            int& fit = per_sm[deep ? 1 : 0][dev];
-            if (fit == 0) {
-                const cudaError_t e =
-                    deep ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, landmarks_warp_kernel<D, 16>, 256, 0)
-                         : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fit, landmarks_warp_kernel<D, 8>, 256, 0);
-                if (e != cudaSuccess || fit < 1) {
-                    fit = 0;
-                    return NYS_ERR_CUDA;
-                }
+            if (per_sm[dev] == 0 &&
+                (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm[dev], landmarks_warp_kernel<D>, 256, 0) !=
+                     cudaSuccess ||
+                 per_sm[dev] < 1)) {
+                per_sm[dev] = 0;
+                return NYS_ERR_CUDA;
             }
-            const long long units = 2LL * BH * m, slots = 8LL * fit * st.sm_count;
+            const long long units = 2LL * BH * m, slots = 8LL * per_sm[dev] * st.sm_count;
             const long long per_warp = (units + slots - 1) / slots;
             const int ctas = (int)((units + 8 * per_warp - 1) / (8 * per_warp));
-            if (deep)
-                landmarks_warp_kernel<D, 16><<<ctas, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, m);
-            else
-                landmarks_warp_kernel<D, 8><<<ctas, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, m);
+            landmarks_warp_kernel<D><<<ctas, 256, 0, s>>>(q, k, ql, kl, ql16, kl16, BH, n, m);
         } else {
             long long threads = (long long)BH * m * (D / 8);
             dim3 grid((unsigned)((threads + 255) / 256), 2);
