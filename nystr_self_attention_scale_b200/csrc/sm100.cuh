@@ -303,6 +303,13 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
     d |= (uint64_t)(layout & 7u) << 61;
     return d;
 }
+// The descriptor of the same operand `bytes` further on (a multiple of 16): only the 14-bit
+// start-address field changes, and no shared-memory address overflows it, so the low word is
+// advanced alone.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) {
+    const uint32_t lo = (uint32_t)d + (bytes >> 4), hi = (uint32_t)(d >> 32);
+    return ((uint64_t)hi << 32) | lo;
+}
 
 // Instruction descriptor: fp32 accumulate, operand formats (1 = bf16, 2 = tf32),
 // operand majors (0 = K-major, 1 = MN-major), shape M x N.

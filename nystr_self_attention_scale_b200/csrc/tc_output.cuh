@@ -8,9 +8,12 @@
 //                                    written back into the S columns of TMEM
 //   O_att  = P . W                   MMA with A = P straight from TMEM
 //   O_conv = T . V_halo              the 65-tap conv as a 128 x 192 banded Toeplitz
-//                                    matrix T (built once per head) times the 192
-//                                    V rows around the tile (zero outside [0, n),
-//                                    supplied by the TMA out-of-bounds fill)
+//                                    matrix T times the 192 V rows around the tile
+//                                    (zero outside [0, n), supplied by the TMA
+//                                    out-of-bounds fill). T's three 64-column blocks
+//                                    are windows of one 256 x 64 strip R,
+//                                    R[u][j] = w[j - u + 128], built once per head:
+//                                    block b is rows 128 - 64 b .. 255 - 64 b of R
 //   out    = O_att / rowsum(P) + O_conv, bf16, TMA store
 //
 // Warp roles (480 threads, one persistent CTA per SM over a contiguous range of
@@ -46,8 +49,7 @@ struct OutTc {
     static constexpr uint32_t kWtBlock = D * 128;     // [D][64] bf16 K-block of W^T
     static constexpr uint32_t kWtBytes = (M / 64) * kWtBlock;
     static constexpr uint32_t kWtLoadBytes = kWtBytes;
-    static constexpr uint32_t kTBlock = 128 * 128;    // [128][64] bf16 K-block of T
-    static constexpr uint32_t kTBytes = 3 * kTBlock;
+    static constexpr uint32_t kTBytes = 256 * 128;    // the [256][64] bf16 strip R
     static constexpr uint32_t kOutBytes = kRows * kSpan;
     // TMEM slot (256 columns): S in [0, M). Softmax group g reads S's columns [g M/2, (g+1) M/2)
     // and writes its P (bf16 pairs) over the first half of that range, columns it has already
@@ -220,20 +222,20 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         // the waits; one elected lane issues each MMA group and each commit
         uint32_t cf_phase = 0;
         bool ok = true;
-        auto descQ = [&](int st, int k) {
-            return smem_desc(sbase + C::kOffQ + st * C::kQBytes + k * 32, 16, C::kSbo, C::kLayout);
+        // operand descriptors: each buffer's is built once, and a K step or a stage advances its
+        // start-address field (this warp's instructions are on every tile's critical path)
+        const uint64_t dQ = smem_desc(sbase + C::kOffQ, 16, C::kSbo, C::kLayout);
+        const uint64_t dKl = smem_desc(sbase + C::kOffKl, 16, C::kSbo, C::kLayout);
+        const uint64_t dWt = smem_desc(sbase + C::kOffWt, 16, 1024, kLayoutSw128);
+        const uint64_t dT = smem_desc(sbase + C::kOffT, 16, 1024, kLayoutSw128);
+        const uint64_t dV = smem_desc(sbase + C::kOffV, C::kVBytes, C::kSbo, C::kLayout);
+        auto descQ = [&](int st, int k) { return desc_advance(dQ, st * C::kQBytes + k * 32); };
+        auto descKl = [&](int k) { return desc_advance(dKl, k * 32); };
+        auto descWt = [&](int k) { return desc_advance(dWt, (k >> 2) * C::kWtBlock + (k & 3) * 32); };
+        auto descT = [&](int k) {   // K step k of T: block k / 4 is the strip window from row 128 - 64 (k / 4)
+            return desc_advance(dT, (128 - 64 * (k >> 2)) * 128 + (k & 3) * 32);
         };
-        auto descKl = [&](int k) { return smem_desc(sbase + C::kOffKl + k * 32, 16, C::kSbo, C::kLayout); };
-        auto descWt = [&](int k) {
-            return smem_desc(sbase + C::kOffWt + (k >> 2) * C::kWtBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
-        };
-        auto descT = [&](int k) {
-            return smem_desc(sbase + C::kOffT + (k >> 2) * C::kTBlock + (k & 3) * 32, 16, 1024, kLayoutSw128);
-        };
-        auto descV = [&](int st, int k) {
-            return smem_desc(sbase + C::kOffV + st * C::kVBytes + k * 16 * C::kSpan, C::kVBytes, C::kSbo,
-                             C::kLayout);
-        };
+        auto descV = [&](int st, int k) { return desc_advance(dV, st * C::kVBytes + k * 16 * C::kSpan); };
         auto wait = [&](uint64_t* bar, uint32_t parity) { return warp_all(mbar_wait(bar, parity)); };
         auto issue_S = [&](int j) -> bool {
             const int s = j & 1, st = j % C::kStages;
@@ -411,22 +413,22 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                     ce_phase ^= 1;
                 }
                 if (conv) {
-                    // T[r][j] = w[j - r] for 0 <= j - r < 65: row r of the banded Toeplitz matrix
+                    // R[u][j] = w[j - u + 128] for 0 <= j - u + 128 < 65: rows r and r + 128
                     const float* wh = prm.conv_w + (size_t)(bh % prm.H) * kTaps;
 #pragma unroll 1
-                    for (int blk = 0; blk < 3; ++blk) {
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const int u = r + 128 * hh;
 #pragma unroll 1
                         for (int ch = 0; ch < 8; ++ch) {
                             uint32_t pk[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
-                                const int j0 = blk * 64 + ch * 8 + 2 * e;
-                                const int d0 = j0 - r, d1 = j0 + 1 - r;
+                                const int d0 = ch * 8 + 2 * e - u + 128, d1 = d0 + 1;
                                 const float w0 = (d0 >= 0 && d0 < kTaps) ? __ldg(wh + d0) : 0.f;
                                 const float w1 = (d1 >= 0 && d1 < kTaps) ? __ldg(wh + d1) : 0.f;
                                 pk[e] = pack_bf16(w0, w1);
                             }
-                            *reinterpret_cast<uint4*>(sm + C::kOffT + blk * C::kTBlock + swz<128>(r, ch)) =
+                            *reinterpret_cast<uint4*>(sm + C::kOffT + swz<128>(u, ch)) =
                                 make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
                     }
@@ -450,19 +452,20 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
                 tmem_ld32(slot + C::kColOatt + c * 32, a);
                 if (conv) tmem_ld32(slot + C::kColOconv + c * 32, b);
                 tmem_ld_wait();
+                if (c + 1 == D / 32) {
+                    // every TMEM column of this tile has been read: the slot is released before the
+                    // last 32 columns are combined
+                    tc_fence_before();
+                    mbar_arrive(&slot_free[s]);
+                }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
-                    float o0 = __uint_as_float(a[2 * j]) * li;
-                    float o1 = __uint_as_float(a[2 * j + 1]) * li;
-                    if (conv) {
-                        o0 += __uint_as_float(b[2 * j]);
-                        o1 += __uint_as_float(b[2 * j + 1]);
-                    }
+                    const float x0 = __uint_as_float(a[2 * j]), x1 = __uint_as_float(a[2 * j + 1]);
+                    const float o0 = conv ? fmaf(x0, li, __uint_as_float(b[2 * j])) : x0 * li;
+                    const float o1 = conv ? fmaf(x1, li, __uint_as_float(b[2 * j + 1])) : x1 * li;
                     outp[c * 16 + j] = pack_bf16(o0, o1);
                 }
             }
-            tc_fence_before();
-            mbar_arrive(&slot_free[s]);
             if (leader) tma_store_wait_read<0>();
             named_barrier(1, 128);
             uint8_t* stage = sm + C::kOffOut;
