@@ -187,14 +187,15 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         const int t = warp == 1 ? 0 : 1;
         bool ok = true;
         int g = 0, it = 0, u = 0;   // chunks before this item, items, chunks of this stream
-        auto descQl = [&](int k) { return smem_desc(sbase + C::kOffQl + k * 32, 16, C::kSbo, C::kLayout); };
-        auto descK = [&](int st, int k) {
-            return smem_desc(sbase + C::kOffK + st * C::kTileBytes + k * 32, 16, C::kSbo, C::kLayout);
-        };
-        auto descV = [&](int st, int k) {
-            return smem_desc(sbase + C::kOffV + st * C::kTileBytes + k * 16 * C::kSpan, C::kTileBytes, C::kSbo,
-                             C::kLayout);
-        };
+        // operand descriptors: each buffer's is built once, and a K step or a ring stage advances
+        // its start-address field (fewer instructions for this warp, which shares its issue slots
+        // with four softmax warps)
+        const uint64_t dQl = smem_desc(sbase + C::kOffQl, 16, C::kSbo, C::kLayout);
+        const uint64_t dK = smem_desc(sbase + C::kOffK, 16, C::kSbo, C::kLayout);
+        const uint64_t dV = smem_desc(sbase + C::kOffV, C::kTileBytes, C::kSbo, C::kLayout);
+        auto descQl = [&](int k) { return desc_advance(dQl, k * 32); };
+        auto descK = [&](int st, int k) { return desc_advance(dK, st * C::kTileBytes + k * 32); };
+        auto descV = [&](int st, int k) { return desc_advance(dV, st * C::kTileBytes + k * 16 * C::kSpan); };
         auto wait = [&](uint64_t* bar, uint32_t parity) { return warp_all(mbar_wait(bar, parity)); };
         for (int item = blockIdx.x; item < prm.total_items && ok && !warp_any(*abort_flag != 0);
              item += gridDim.x, ++it) {
