@@ -436,6 +436,46 @@ int launch_simt(const Plan& p, const DeviceState& st, const T* q, const T* k, co
     return cudaGetLastError() == cudaSuccess ? NYS_OK : NYS_ERR_CUDA;
 }
 
+// Contiguous tile ranges for the output pass's persistent CTAs. A range that crosses into a new
+// head pays for the change of per-head constants (the pipeline drains, the Toeplitz strip is
+// rebuilt): about two tiles' time. The ranges are chosen greedily against a bound C on
+// (tiles + 2 per head crossed), none longer than an even share of the tiles left, with the
+// smallest C that fits `ctas` ranges (binary search); where no range crosses, this is the even
+// split. Writes ctas + 1 boundaries.
+void output_tile_ranges(int total, int tph, int ctas, int* start) {
+    constexpr int kCross = 2;
+    auto fill = [&](int C, bool write) {
+        int t = 0, b = 0;
+        while (t < total) {
+            if (b == ctas) return false;
+            if (write) start[b] = t;
+            const int first = t;
+            // no more tiles than an even share of what is left, so that ranges that cross no head
+            // are not packed beyond the even split
+            const int cap = (total - t + (ctas - b) - 1) / (ctas - b);
+            int cost = 0;
+            while (t < total && t - first < cap) {
+                const int add = 1 + (t > first && t % tph == 0 ? kCross : 0);
+                if (t > first && cost + add > C) break;
+                cost += add;
+                ++t;
+            }
+            ++b;
+        }
+        if (write)
+            for (; b <= ctas; ++b) start[b] = total;
+        return true;
+    };
+    // the even split costs at most (1 + kCross) per tile, so fill(hi) succeeds; fill(lo) fails
+    const int even = (total + ctas - 1) / ctas;
+    int lo = even - 1, hi = even * (1 + kCross);
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) / 2;
+        (fill(mid, false) ? hi : lo) = mid;
+    }
+    fill(hi, true);
+}
+
 template <int D, int M>
 int launch_output_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* q, const __nv_bfloat16* v,
                      const float* conv_w, __nv_bfloat16* out, const __nv_bfloat16* kl16,
@@ -448,8 +488,9 @@ int launch_output_tc(const Plan& p, const DeviceState& st, const __nv_bfloat16* 
         !map_bf16_3d(&mo, out, D, n, BH, D, 128, sw) || !map_bf16_3d(&mkl, kl16, D, M, BH, D, M, sw) ||
         !map_bf16_3d(&mwt, wt16, M, D, BH, 64, D, CU_TENSOR_MAP_SWIZZLE_128B))
         return NYS_ERR_CUDA;
-    OutTcParams prm{conv_w, p.H, p.n, p.n / 128, p.BH * (p.n / 128)};
-    const int grid = std::min(prm.total_tiles, st.sm_count);
+    OutTcParams prm{conv_w, p.H, p.n, p.n / 128, p.BH * (p.n / 128), {}};
+    const int grid = std::min(std::min(prm.total_tiles, st.sm_count), kOutMaxCtas);
+    output_tile_ranges(prm.total_tiles, prm.tiles_per_head, grid, prm.tile_start);
     static bool attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaGetDevice(&dev);

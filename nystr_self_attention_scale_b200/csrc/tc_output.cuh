@@ -84,9 +84,13 @@ struct OutTc {
     static constexpr uint32_t kIdConv = sm100::make_idesc(128, D, sm100::kFmtBf16, sm100::kFmtBf16, 0, 1);
 };
 
+constexpr int kOutMaxCtas = 160;
+
 struct OutTcParams {
     const float* conv_w;   // [H, 65] or null
     int H, n, tiles_per_head, total_tiles;
+    // CTA b takes tiles tile_start[b] .. tile_start[b + 1] - 1 (contiguous, in order)
+    int tile_start[kOutMaxCtas + 1];
 };
 
 template <int D, int M>
@@ -121,9 +125,8 @@ output_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // contiguous tile range of this CTA
-    const int per = prm.total_tiles / gridDim.x, extra = prm.total_tiles % gridDim.x;
-    const int t0 = blockIdx.x * per + min((int)blockIdx.x, extra);
-    const int count = per + ((int)blockIdx.x < extra ? 1 : 0);
+    const int t0 = prm.tile_start[blockIdx.x];
+    const int count = prm.tile_start[blockIdx.x + 1] - t0;
     const int tph = prm.tiles_per_head;
     auto head_start = [&](int i) { return i == 0 || ((t0 + i) % tph) == 0; };
 
