@@ -19,10 +19,14 @@
 // rescaled once. Every exponential of a row uses the same reference, so the
 // result is the exact softmax; P stays below 256, well inside bf16 range.
 // An item's chunks run as two independent streams: chunk c goes to stream
-// c % 2, which has its own S buffer, P buffer, O accumulator, reference max
-// and running sum in TMEM / registers. P has its own TMEM columns, so a
-// stream's next S MMA only waits until the softmax has loaded the current
-// scores, and runs while the exponentials are computed. At the end of an item
+// c % 2, which has its own O accumulator, reference max and running sum in
+// TMEM / registers. The S products go to a ring of three 128-column TMEM
+// buffers shared by the two streams (chunk g of the CTA's sequence to buffer
+// g % 3); each softmax group writes its P (bf16 pairs) over the first half of
+// its own 64 score columns, which it has read, and the P V product takes P from
+// there. A buffer is reused once that P V is done, so a stream's next S product
+// waits for the P V of the chunk three places back (the other stream's previous
+// chunk) and is in place before the stream's softmax needs it. At the end of an item
 // the threads of stream 0 merge the two streams' (O, reference max, running
 // sum) row by row and write the unnormalised partial of the split; a
 // deterministic combine over splits follows. The stream of a chunk depends
@@ -34,8 +38,7 @@
 // behind the other's), warps 2-17 the softmax: stream t owns warps 2 + 8 t .. 9 + 8 t, two
 // warpgroups that split each of its chunks' 128 keys (64 each), exchanging the
 // chunk max through shared memory. Each SM sub-partition runs four softmax
-// warps, two per stream. Each group writes its P (bf16 pairs) into its half
-// of the stream's P buffer.
+// warps, two per stream.
 // K/V chunks use a 6-stage shared-memory ring (three chunks of lookahead per stream).
 #pragma once
 
@@ -55,7 +58,7 @@ struct K3vTc {
     static constexpr uint32_t kOffK = kOffQl + kTileBytes;
     static constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;
     static constexpr uint32_t kOffBar = kOffV + kStages * kTileBytes;
-    static constexpr int kNumBars = 2 + 2 * kStages + 10 + 1;
+    static constexpr int kNumBars = 2 + 2 * kStages + 12 + 1;
     static constexpr int kStreams = 2;                                    // softmax streams
     static constexpr int kTeamThreads = 256;                              // two warpgroups per stream
     static constexpr int kThreads = 96 + kStreams * kTeamThreads;        // warps 0, 1, 18 + the streams
@@ -67,8 +70,9 @@ struct K3vTc {
     static constexpr uint32_t kSmemNeed = kOffMisc + 16 + 1024;
     static constexpr uint32_t kSmemBytes = kSmemNeed > 118784 ? kSmemNeed : 118784;
     static constexpr int kTmemCols = 512;
-    // TMEM columns of stream t: S at 128 t, P (bf16 pairs) at 256 + 64 t, O at 384 + D t
-    static constexpr int kColS = 0, kColP = 256, kColO = 384;
+    // TMEM columns: S ring buffer b at 128 b (b = 0, 1, 2; P over the first half of each
+    // group's 64 columns), O of stream t at 384 + D t
+    static constexpr int kColS = 0, kColO = 384;
     static constexpr uint32_t kIdS = sm100::make_idesc(128, kChunk, sm100::kFmtBf16, sm100::kFmtBf16, 0, 0);
     static constexpr uint32_t kIdPV = sm100::make_idesc(128, D, sm100::kFmtBf16, sm100::kFmtBf16, 0, 1);
 };
@@ -97,12 +101,14 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
     uint64_t* ql_empty = bars + 1;
     uint64_t* kv_full = bars + 2;                  // [kStages]
     uint64_t* kv_empty = bars + 2 + C::kStages;    // [kStages]
-    uint64_t* s_full = bars + 2 + 2 * C::kStages;  // [stream] S of its current chunk in TMEM
-    uint64_t* p_full = s_full + 2;                 // [stream] P in TMEM (256 arrivals)
-    uint64_t* pv_done = s_full + 4;                // [stream] P V accumulated into its O
-    uint64_t* o_free = s_full + 6;                 // [stream] the item's O has been read (256 arrivals)
-    uint64_t* s_free = s_full + 8;                 // [stream] its S has been loaded (256 arrivals)
-    uint64_t* mma_done = s_full + 10;
+    // [3] S of the chunk in ring buffer b in TMEM: one barrier per buffer, so that a stream's next
+    // S (in another buffer) may complete before its softmax has waited for the current one
+    uint64_t* s_full = bars + 2 + 2 * C::kStages;
+    uint64_t* p_full = s_full + 3;                 // [stream] P in TMEM (256 arrivals)
+    uint64_t* pv_done = s_full + 5;                // [stream] P V accumulated into its O
+    uint64_t* o_free = s_full + 7;                 // [stream] the item's O has been read (256 arrivals)
+    uint64_t* buf_free = s_full + 9;               // [3] S ring buffer reusable: the P V reading it is done
+    uint64_t* mma_done = s_full + 12;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + C::kOffMisc + 4);
 
@@ -124,11 +130,13 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             mbar_init(&kv_empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&s_full[b], 1);
             mbar_init(&p_full[b], C::kTeamThreads);
             mbar_init(&pv_done[b], 1);
             mbar_init(&o_free[b], C::kTeamThreads);
-            mbar_init(&s_free[b], C::kTeamThreads);
+        }
+        for (int b = 0; b < 3; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&buf_free[b], 1);
         }
         mbar_init(mma_done, 64);   // one commit per lane of the two MMA warps
         *abort_flag = 0;
@@ -204,27 +212,27 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             ok = wait(ql_full, it & 1);
             if (!ok) break;
             tc_fence_after();
-            // S of chunk c (the stream's u-th): its S buffer is free once the softmax has loaded
-            // the previous scores
-            auto issue_S = [&](int c, int uu) -> bool {
-                const int gc = g + c, st = gc % C::kStages;
-                if (uu > 0 && !wait(&s_free[t], (uu - 1) & 1)) return false;
+            // S of chunk c into ring buffer (g + c) % 3, once the P V of the chunk three places
+            // back (which read its P from that buffer) is done
+            auto issue_S = [&](int c) -> bool {
+                const int gc = g + c, st = gc % C::kStages, b = gc % 3;
+                if (gc >= 3 && !wait(&buf_free[b], (gc / 3 - 1) & 1)) return false;
                 if (!wait(&kv_full[st], (gc / C::kStages) & 1)) return false;
                 tc_fence_after();
                 if (elect_one()) {
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_bf16_ss(tmem + C::kColS + t * 128, descQl(k), descK(st, k), C::kIdS, k > 0);
+                        mma_bf16_ss(tmem + C::kColS + b * 128, descQl(k), descK(st, k), C::kIdS, k > 0);
                 }
-                if (elect_one()) mma_commit(&s_full[t]);
+                if (elect_one()) mma_commit(&s_full[b]);
                 return true;
             };
-            if (t < nch) ok = issue_S(t, u);
+            if (t < nch) ok = issue_S(t);
             for (int c = t; c < nch && ok; c += 2, ++u) {
-                const int gc = g + c, st = gc % C::kStages;
+                const int gc = g + c, st = gc % C::kStages, b = gc % 3;
                 // the next S of the stream goes first, so that it runs during this chunk's softmax
                 if (c + 2 < nch) {
-                    if (!(ok = issue_S(c + 2, u + 1))) break;
+                    if (!(ok = issue_S(c + 2))) break;
                 } else if (elect_one()) {
                     mma_commit(ql_empty);   // this stream's last S of the item is issued
                 }
@@ -237,8 +245,9 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 if (elect_one()) {
 #pragma unroll
                     for (int k = 0; k < C::kChunk / 16; ++k) {
-                        // keys 16k .. 16k+15: P of group k / 4, in its 32 columns of the P buffer
-                        const uint32_t pa = tmem + C::kColP + t * 64 + 32 * (k >> 2) + 8 * (k & 3);
+                        // keys 16k .. 16k+15: P of group k / 4, over the first half of its 64
+                        // score columns in the chunk's ring buffer
+                        const uint32_t pa = tmem + C::kColS + b * 128 + 64 * (k >> 2) + 8 * (k & 3);
                         mma_bf16_ts(tmem + C::kColO + t * D, pa, descV(st, k), C::kIdPV,
                                     (first && k == 0) ? 0u : 1u);
                     }
@@ -246,6 +255,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 if (elect_one()) {
                     mma_commit(&pv_done[t]);
                     mma_commit(&kv_empty[st]);
+                    mma_commit(&buf_free[b]);
                 }
             }
             // a stream with no chunk in this item still releases Q_l once
@@ -272,10 +282,9 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
         float* lx_all = reinterpret_cast<float*>(sm + C::kOffLx);   // [2 streams][2 groups][128]
         float* mx_all = reinterpret_cast<float*>(sm + C::kOffMx);   // [2 streams][128]
         constexpr int kCta = 2 * C::kTeamThreads;   // both streams: named barrier 3
-        const uint32_t sbuf = tmem + lane_base + C::kColS + t * 128 + 64 * grp;
-        const uint32_t pbuf = tmem + lane_base + C::kColP + t * 64 + 32 * grp;
         const uint32_t obuf = tmem + lane_base + C::kColO + t * D + 32 * grp;
         int u = 0, it = 0;   // chunks this stream has taken, items
+        int g = 0;           // chunks of the CTA's earlier items (the S ring position)
         for (int item = blockIdx.x; item < prm.total_items; item += gridDim.x, ++it) {
             // both streams take every item-level decision together (barrier 3), so that neither
             // waits at that barrier for a stream that has left
@@ -290,6 +299,10 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
             int mine = 0;                           // chunks of this item taken by the stream
             for (int c = t; c < nch; c += 2, ++u, ++mine) {
                 const int key0 = (c0 + c) * C::kChunk + 64 * grp;
+                // this group's 64 score columns in the chunk's ring buffer; its P goes over their
+                // first half once they are read
+                const uint32_t sbuf = tmem + lane_base + C::kColS + ((g + c) % 3) * 128 + 64 * grp;
+                const uint32_t pbuf = sbuf;
                 // key-validity bits of this group's 64 keys (bit k of word h = key key0 + 32 h + k)
                 uint32_t mb[2] = {~0u, ~0u};
                 if (prm.mask_bits != nullptr) {
@@ -300,7 +313,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 const bool full = (mb[0] & mb[1]) == ~0u;
                 // a wait that runs out leaves S unread: the group still passes the chunk's one
                 // barrier below (which also ORs the failure across the two groups) and then stops
-                ok = warp_all(mbar_wait(&s_full[t], u & 1));
+                ok = warp_all(mbar_wait(&s_full[(g + c) % 3], ((g + c) / 3) & 1));
                 tc_fence_after();
                 // pass 1: the max of this group's 64 scores (the scores are loaded again for the
                 // exponentials, which keeps the register footprint small)
@@ -358,8 +371,6 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 tmem_ld32(sbuf, vv[0]);
                 tmem_ld32(sbuf + 32, vv[1]);
                 tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(&s_free[t]);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t* v = vv[h];
@@ -400,12 +411,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                             acc[e & 1] = f2_add(acc[e & 1], f2(e0, e1));
                         }
                     }
-                    // this group's P (keys 32 h ..) into its 32 columns of the P buffer, which the
-                    // stream's previous P V must have finished reading
-                    if (h == 0 && u > 0) {
-                        if (!warp_all(mbar_wait(&pv_done[t], (u - 1) & 1))) ok = false;
-                        tc_fence_after();
-                    }
+                    // this group's P (keys 32 h ..) over scores it has read (all 64 are in registers)
                     tmem_st16(pbuf + 16 * h, pk);
                 }
                 float sum;
@@ -475,6 +481,7 @@ k3v_tc_kernel(const __grid_constant__ CUtensorMap map_ql, const __grid_constant_
                 mbar_arrive(&o_free[1]);
             }
             named_barrier(3, kCta);   // the statistics are read before the next item overwrites them
+            g += nch;
         }
     }
 
