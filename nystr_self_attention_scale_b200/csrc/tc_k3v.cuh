@@ -26,7 +26,8 @@
 // its own 64 score columns, which it has read, and the P V product takes P from
 // there. A buffer is reused once that P V is done, so a stream's next S product
 // waits for the P V of the chunk three places back (the other stream's previous
-// chunk) and is in place before the stream's softmax needs it. At the end of an item
+// chunk), not for this stream's softmax, and is mostly in place by the time the
+// softmax needs it. At the end of an item
 // the threads of stream 0 merge the two streams' (O, reference max, running
 // sum) row by row and write the unnormalised partial of the split; a
 // deterministic combine over splits follows. The stream of a chunk depends
@@ -34,8 +35,8 @@
 // rest of the batch.
 //
 // Warp roles (608 threads): warp 0 TMA producer and TMEM allocator, warps 1
-// and 18 the MMA issuers of streams 0 and 1 (so that neither stream's MMAs wait
-// behind the other's), warps 2-17 the softmax: stream t owns warps 2 + 8 t .. 9 + 8 t, two
+// and 18 the MMA issuers of streams 0 and 1 (each issues in its own stream's
+// order, so neither waits in program order behind the other's), warps 2-17 the softmax: stream t owns warps 2 + 8 t .. 9 + 8 t, two
 // warpgroups that split each of its chunks' 128 keys (64 each), exchanging the
 // chunk max through shared memory. Each SM sub-partition runs four softmax
 // warps, two per stream.
