@@ -443,34 +443,38 @@ int launch_simt(const Plan& p, const DeviceState& st, const T* q, const T* k, co
 // smallest C that fits `ctas` ranges (binary search); where no range crosses, this is the even
 // split. Writes ctas + 1 boundaries.
 void output_tile_ranges(int total, int tph, int ctas, int* start) {
-    constexpr int kCross = 2;
-    auto fill = [&](int C, bool write) {
-        int t = 0, b = 0;
-        while (t < total) {
-            if (b == ctas) return false;
-            if (write) start[b] = t;
-            const int first = t;
+    constexpr long long kCross = 2;
+    // head starts strictly inside the range of `len` tiles from `first` (its first tile excluded)
+    auto crossings = [&](long long first, long long len) {
+        return len <= 1 ? 0LL : (first + len - 1) / tph - first / tph;
+    };
+    auto fill = [&](long long C, bool write) {
+        long long t = 0;
+        int b = 0;
+        for (; b < ctas && t < total; ++b) {
             // no more tiles than an even share of what is left, so that ranges that cross no head
-            // are not packed beyond the even split
-            const int cap = (total - t + (ctas - b) - 1) / (ctas - b);
-            int cost = 0;
-            while (t < total && t - first < cap) {
-                const int add = 1 + (t > first && t % tph == 0 ? kCross : 0);
-                if (t > first && cost + add > C) break;
-                cost += add;
-                ++t;
+            // are not packed beyond the even split; then the longest range within the bound C
+            // (its cost grows with its length)
+            const long long cap = std::min<long long>((total - t + (ctas - b) - 1) / (ctas - b), total - t);
+            long long lo = 1, hi = cap;
+            while (lo < hi) {
+                const long long mid = (lo + hi + 1) / 2;
+                if (mid + kCross * crossings(t, mid) <= C) lo = mid;
+                else hi = mid - 1;
             }
-            ++b;
+            if (write) start[b] = (int)t;
+            t += lo;
         }
+        if (t < total) return false;
         if (write)
             for (; b <= ctas; ++b) start[b] = total;
         return true;
     };
     // the even split costs at most (1 + kCross) per tile, so fill(hi) succeeds; fill(lo) fails
-    const int even = (total + ctas - 1) / ctas;
-    int lo = even - 1, hi = even * (1 + kCross);
+    const long long even = (total + ctas - 1) / ctas;
+    long long lo = even - 1, hi = even * (1 + kCross);
     while (hi - lo > 1) {
-        const int mid = (lo + hi) / 2;
+        const long long mid = (lo + hi) / 2;
         (fill(mid, false) ? hi : lo) = mid;
     }
     fill(hi, true);
