@@ -489,7 +489,8 @@ def main():
 
     # per-kernel breakdown: a separate, untimed pass in which every kernel launch is bracketed by
     # CUDA events (the event records delay each following launch, so the timed loop below
-    # brackets only the dominant kernel, the one the roofline reports)
+    # brackets only the dominant kernel, the one the roofline reports, and only in its last
+    # tenth of steps: the brackets add a few microseconds to each step they are in)
     breakdown_steps = 10
     nys.profile_mask(None)
     nys.profile_enable(True)
@@ -516,8 +517,10 @@ def main():
         dist.barrier()
     torch.cuda.synchronize()
     nys.profile_mask([dom])
-    nys.profile_enable(True)
+    prof_steps = max(1, args.steps // 10)
     for i in range(args.steps):
+        if i == args.steps - prof_steps:
+            nys.profile_enable(True)
         if not args.no_flush:
             flush_l2()
         starts[i].record(stream)
@@ -560,6 +563,7 @@ def main():
     if args.path == "exact":
         traffic = None   # the ncu traffic figures are for the Nystrom path's kernels
     roof = roofline_for(w, dom, prof[dom][1] / max(1, prof[dom][0]), peaks, simt, traffic, args.path)
+    roof["launches_timed"] = int(prof[dom][0])   # the dominant kernel's launches in the timed steps
     roof["peak_source"] = f"{peak_src} ({'MEASURED_PEAKS.json' if peak_src == 'measured' else 'recipe fallback'})"
     if args.path == "exact":
         t_roof, ideal_bytes, total_flops = roofline_bound_time_exact(w, peaks)
@@ -628,7 +632,7 @@ def main():
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
             "kernels": kernels,
             "kernels_source": f"separate untimed pass of {breakdown_steps} steps, every launch bracketed by "
-                              "CUDA events; the timed loop brackets only the roofline kernel",
+                              "CUDA events; the timed loop brackets only the roofline kernel, in its last tenth of steps",
             "clocks": clocks, "device_status": status,
         }
         print(json.dumps(line), flush=True)
