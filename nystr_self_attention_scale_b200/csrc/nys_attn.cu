@@ -232,7 +232,7 @@ struct Plan {
     int BH, splits, keys_per_split;
     size_t off_ql, off_kl, off_ql16, off_kl16, off_k3v, off_w, off_wt16, off_z, off_pinv;
     size_t off_po, off_pm, off_pl, off_mbits, total;
-    size_t off_k2b, off_k2tb, off_zb;   // CTA-pair inverse (m = 256): k2, k2^T and W^T scratch
+    size_t off_k2b, off_zb;   // CTA-pair inverse (m = 256): k2 and W^T scratch
     int tc_cps, tc_splits;  // tensor-core kernel_3 V: 128-key chunks per split, splits
     GuardList guards;       // guard zones (guard mode only; guards.n == 0 otherwise)
 };
@@ -360,7 +360,6 @@ Plan make_plan(int B, int H, int n, int d, int m, int n_iter, int dtype, int sm_
     p.off_mbits = take((size_t)B * ((n + 31) / 32) * 4);
     if (dtype == NYS_BF16 && m == 256) {
         p.off_k2b = take(BH * mm * 4);
-        p.off_k2tb = take(BH * mm * 4);
         p.off_zb = take(BH * mm * 4);
     }
     if (guard) zone();
@@ -607,7 +606,6 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
         attr_set[dev] = true;
     }
     float* k2 = reinterpret_cast<float*>(ws + p.off_k2b);
-    float* k2t = reinterpret_cast<float*>(ws + p.off_k2tb);
     float* zs = reinterpret_cast<float*>(ws + p.off_zb);
     PinvPairMaps maps;
     const uint64_t BH = p.BH;
@@ -616,10 +614,10 @@ int launch_pinv_pair(const Plan& p, const DeviceState& st, const float* ql, cons
     if (!map_3d(&maps.ql, f32, 4, ql, p.d, M, BH, 32, 128, sw) ||
         !map_3d(&maps.kl, f32, 4, kl, p.d, M, BH, 32, 128, sw) ||
         !map_3d(&maps.k2, f32, 4, k2, M, M, BH, 32, 128, sw) ||
-        !map_3d(&maps.k2t, f32, 4, k2t, M, M, BH, 32, 128, sw) ||
+        !map_3d(&maps.k2mn, f32, 4, k2, M, M, BH, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) ||
         !map_3d(&maps.wt, f32, 4, zs, M, M, BH, 32, 128, sw))
         return NYS_ERR_CUDA;
-    PinvPairParams prm{k2, k2t, zs, z, p.d, p.n_iter, inv_init};
+    PinvPairParams prm{k2, zs, z, p.d, p.n_iter, inv_init};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.BH * 2);
     cfg.blockDim = dim3(C::kThreads);

@@ -20,9 +20,10 @@
 // peer's) -- X is symmetric only in exact arithmetic, and using its rows as
 // its columns loses accuracy on ill-conditioned k2 -- and, streamed from L2 one
 // 32-wide K atom at a time behind the previous product's MMAs, the columns of W
-// (for P4; the P4 epilogue writes W^T row-major to scratch) and the last three
-// K atoms of k2's rows (for P1; its first five K atoms stay in shared memory
-// for the whole kernel).
+// (for P4; the P4 epilogue writes W^T row-major to scratch; the first P4 reads
+// W_0 = c k2 by rows instead, as an MN-major operand, so that no transpose of k2
+// is written) and the last three K atoms of k2's rows (for P1; its first five K
+// atoms stay in shared memory for the whole kernel).
 //
 // One head per cluster of two CTAs, one 2-CTA tcgen05 MMA per K step
 // (cta_group::2, kind::tf32, M = N = 256): CTA r holds rows 128r .. 128r+127 of
@@ -137,13 +138,13 @@ struct PinvPairMaps {
     CUtensorMap ql;    // Q_l  [BH][256][d] fp32, box 32 x 128, 128-byte swizzle: A of the kernel_2 product
     CUtensorMap kl;    // K_l, same box: B lines of the kernel_2 product
     CUtensorMap k2;    // k2   [BH][256][256] fp32, box 32 x 128: B atoms of the later P1s (and its TMA store)
-    CUtensorMap k2t;   // k2^T, same box: B atoms of the first P4 (columns of W_0 = c k2)
+    CUtensorMap k2mn;  // k2 again, box 32 x 32, 32-byte-granule 128-byte swizzle: the first P4's B atoms,
+                       // MN-major (W_0 = c k2 read by rows: K row k = row k of k2)
     CUtensorMap wt;    // W^T scratch, same box: B atoms of the later P4s
 };
 
 struct PinvPairParams {
     float* k2;         // [BH][256][256] k2 (tf32), written here, read back by TMA
-    float* k2t;        // [BH][256][256] k2^T (tf32), written here, read back by TMA
     float* wt;         // [BH][256][256] W^T scratch (row g = column g of W)
     float* z_out;      // [BH][256][256]
     int d, n_iter;
@@ -173,6 +174,10 @@ struct PinvPair {
     static constexpr uint32_t kSmemBytes = kSmemNeed < 200 * 1024 ? 200 * 1024 : kSmemNeed;
     static constexpr int kThreads = 320;
     static constexpr uint32_t kIdesc = sm100::make_idesc(256, 256, sm100::kFmtTf32, sm100::kFmtTf32, 0, 0);
+    // the first P4: B MN-major (K atom kc = rows 32 kc .. + 31 of k2, this CTA's 128 columns as four
+    // 4 KB column blocks of 32 rows x 128 bytes; an MMA K step is 8 rows = 1 KB into each block)
+    static constexpr uint32_t kIdescBmn = sm100::make_idesc(256, 256, sm100::kFmtTf32, sm100::kFmtTf32, 0, 1);
+    static constexpr uint32_t kMnBlock = 32 * 128;
 };
 static_assert(PinvPair::kSmemBytes <= 227 * 1024, "pair inverse: shared memory");
 
@@ -196,7 +201,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
     uint64_t* mma_done = bfree + 8;      // kernel_2 and P1..P3 accumulators complete (both CTAs)
     uint64_t* mma4_done = mma_done + 1;  // P4 accumulator complete (both CTAs)
     uint64_t* e_ready = mma4_done + 1;   // epilogue output in place for the next product (CTA 0)
-    uint64_t* wl_ready = e_ready + 1;    // k2 / k2^T / W^T scratch written by both CTAs (each CTA)
+    uint64_t* wl_ready = e_ready + 1;    // k2 / W^T scratch written by both CTAs (each CTA)
     uint64_t* drain = wl_ready + 1;
     uint64_t* pro_full = drain + 1;      // Q_l / K_l tiles landed (each CTA)
     uint64_t* cs_ready = pro_full + 1;   // the peer's column sums are in cs_peer (each CTA)
@@ -243,7 +248,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             prefetch_tmap(&maps.ql);
             prefetch_tmap(&maps.kl);
             prefetch_tmap(&maps.k2);
-            prefetch_tmap(&maps.k2t);
+            prefetch_tmap(&maps.k2mn);
             prefetch_tmap(&maps.wt);
             // kernel_2 operands: this CTA's rows of Q_l (A) and of K_l (its B lines)
             mbar_arrive_expect_tx(pro_full, 2u * nka * C::kAtomBytes);
@@ -259,9 +264,9 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 for (int part = 0; part < 2 && ok; ++part) {
                     const int p = part == 0 ? 0 : 3;
                     if (p == 0 && it == 0) continue;   // the first P1 reads k2 staged by the prologue
-                    const CUtensorMap* mp = p == 0 ? &maps.k2 : (it == 0 ? &maps.k2t : &maps.wt);
+                    const CUtensorMap* mp = p == 0 ? &maps.k2 : &maps.wt;
                     if (p == 3) {
-                        // k2 / k2^T (prologue) or W^T (previous P4) of both CTAs is in global memory
+                        // k2 (prologue) or W^T (previous P4) of both CTAs is in global memory
                         ok = wait_acq_cluster(wl_ready, (uint32_t)it & 1u);
                         fence_proxy_async_global();
                     }
@@ -277,7 +282,14 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                         if (!ok) break;
                         if (p == 0 && kc < C::kK2Resident) continue;
                         if (leader) mbar_arrive_expect_tx(&bfull[kc], 2 * C::kAtomBytes);
-                        tma_load_3d_pair(bbuf + kc * C::kAtomBytes, mp, bfull0 + 8 * kc, 32 * kc, r0, bh, keep_policy);
+                        if (p == 3 && it == 0) {
+                            // rows 32 kc .. + 31 of k2, this CTA's columns r0 .. r0 + 127
+                            for (int t = 0; t < 4; ++t)
+                                tma_load_3d_pair(bbuf + kc * C::kAtomBytes + t * C::kMnBlock, &maps.k2mn, bfull0 + 8 * kc,
+                                                 r0 + 32 * t, 32 * kc, bh, keep_policy);
+                        } else {
+                            tma_load_3d_pair(bbuf + kc * C::kAtomBytes, mp, bfull0 + 8 * kc, 32 * kc, r0, bh, keep_policy);
+                        }
                     }
                 }
             }
@@ -345,12 +357,20 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                             tc_fence_after();
                         }
                         if (elect_one()) {
+                            if (p == 3 && it == 0) {
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma2_ts(d_col, a_col + kc * 32 + kk * 8,
-                                        smem_desc((resident ? bs + C::kOffK2r : bs) + kc * C::kAtomBytes + kk * 32, 16,
-                                                  1024, kLayoutSw128),
-                                        C::kIdesc, (i | kk) != 0 ? 1u : 0u);
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma2_ts(d_col, a_col + kc * 32 + kk * 8,
+                                            smem_desc(bs + kc * C::kAtomBytes + kk * 1024, C::kMnBlock, 512, kLayoutSw128B32),
+                                            C::kIdescBmn, (i | kk) != 0 ? 1u : 0u);
+                            } else {
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma2_ts(d_col, a_col + kc * 32 + kk * 8,
+                                            smem_desc((resident ? bs + C::kOffK2r : bs) + kc * C::kAtomBytes + kk * 32, 16,
+                                                      1024, kLayoutSw128),
+                                            C::kIdesc, (i | kk) != 0 ? 1u : 0u);
+                            }
                             if (p >= 2) commit2(&bfree[kc], 3);   // the producer refills this atom next
                         }
                     }
@@ -481,7 +501,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             named_barrier(3, 256);
             const float inv = 1.f / (sx[lrow] + sx[128 + lrow]);
             // k2 = e / sum: into TMEM as W_0 (R0) and into the B buffer as the first P1's right
-            // factor (this CTA's rows are its own B lines); k2^T goes to global memory later
+            // factor (this CTA's rows are its own B lines)
             float rsum = 0.f;
 #pragma unroll 1
             for (int jp = 0; jp < 2; ++jp) {
@@ -513,18 +533,54 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
             rx[h * 128 + lrow] = rsum;   // rx is free: every thread read its row max before the last barrier
             fence_proxy_async_shared();   // the staged k2 rows feed the MMA and a TMA store
             named_barrier(3, 256);
-            // column sums over this CTA's rows (thread et: column et), max row sum of this CTA
+            if (n_iter > 0) {
+                // W_0 in TMEM and k2's lines in the B buffer are all that the first P1 reads (the
+                // coefficient only scales its epilogue): it runs beside the column sums below
+                tmem_st_wait();
+                arrive_e();
+                // the rows of k2 go to global memory for the later P1s. The copy has read the B
+                // buffer before this CTA arrives on the peer's cs_ready and before the barrier that
+                // follows this CTA's own cs_ready wait, so before either CTA's P1 epilogue writes -X
+                // lines into it.
+                if (et == 0) {
+                    for (int a = 0; a < 8; ++a) tma_store_3d(&maps.k2, bbuf + a * C::kAtomBytes, 32 * a, r0, bh);
+                    tma_store_commit();
+                }
+            }
+            // column sums over this CTA's rows, max row sum of this CTA. Warp w sums K atom w:
+            // lane (c, rq) = (lane % 8, lane / 8) adds the 16-byte chunk of columns 32 w + 4 c .. + 3
+            // over rows rq, rq + 4, ... (a warp load covers four whole rows), then the four row
+            // quarters are added across lanes
             {
-                const int a = et >> 5, j = et & 31;
-                float c4[4] = {0.f, 0.f, 0.f, 0.f};   // four independent chains
+                const int c = lane & 7, rq = lane >> 3;
+                float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;   // two independent chains
 #pragma unroll 8
-                for (int l = 0; l < 128; ++l)
-                    c4[l & 3] += *reinterpret_cast<const float*>(
-                        bbuf + (uint32_t)a * C::kAtomBytes + (uint32_t)l * 128u +
-                        ((((uint32_t)j >> 2) ^ (uint32_t)(l & 7)) << 4) + (uint32_t)(j & 3) * 4u);
-                const float cs = (c4[0] + c4[1]) + (c4[2] + c4[3]);
-                cs_own[et] = cs;
-                st_remote(mapa(smem_u32(cs_peer + et), rank ^ 1u), cs);
+                for (int i = 0; i < 32; i += 2) {
+                    const int l0 = rq + 4 * i, l1 = l0 + 4;
+                    const float4 x0 = *reinterpret_cast<const float4*>(
+                        bbuf + (uint32_t)warp * C::kAtomBytes + (uint32_t)l0 * 128u + (((uint32_t)c ^ (uint32_t)(l0 & 7)) << 4));
+                    const float4 x1 = *reinterpret_cast<const float4*>(
+                        bbuf + (uint32_t)warp * C::kAtomBytes + (uint32_t)l1 * 128u + (((uint32_t)c ^ (uint32_t)(l1 & 7)) << 4));
+                    s0.x += x0.x; s0.y += x0.y; s0.z += x0.z; s0.w += x0.w;
+                    s1.x += x1.x; s1.y += x1.y; s1.z += x1.z; s1.w += x1.w;
+                }
+                float4 cs = make_float4(s0.x + s1.x, s0.y + s1.y, s0.z + s1.z, s0.w + s1.w);
+#pragma unroll
+                for (int o = 8; o <= 16; o <<= 1) {
+                    cs.x += __shfl_xor_sync(0xffffffffu, cs.x, o);
+                    cs.y += __shfl_xor_sync(0xffffffffu, cs.y, o);
+                    cs.z += __shfl_xor_sync(0xffffffffu, cs.z, o);
+                    cs.w += __shfl_xor_sync(0xffffffffu, cs.w, o);
+                }
+                if (rq == 0) {
+                    const int col = 32 * warp + 4 * c;
+                    *reinterpret_cast<float4*>(cs_own + col) = cs;
+                    const uint32_t pa = mapa(smem_u32(cs_peer + col), rank ^ 1u);
+                    st_remote(pa, cs.x);
+                    st_remote(pa + 4, cs.y);
+                    st_remote(pa + 8, cs.z);
+                    st_remote(pa + 12, cs.w);
+                }
                 const float rs = warp_max(et < 128 ? rx[et] + rx[128 + et] : 0.f);
                 if (lane == 0) wmax[warp] = rs;
             }
@@ -534,6 +590,7 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                 rmax[0] = rm;
                 st_remote(mapa(smem_u32(rmax + 1), rank ^ 1u), rm);
             }
+            if (et == 0 && n_iter > 0) tma_store_wait_read<0>();   // k2's copy has read the B buffer
             __syncwarp();
             if (lane == 0) arrive_cluster(mapa(smem_u32(cs_ready), rank ^ 1u));
             const bool ok = wait_acq_cluster(cs_ready, 0);
@@ -563,37 +620,6 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                         zc[(size_t)(32 * a + 4 * c + 3) * M] = coeff * f4.w;
                     }
                 }
-            } else if (!failed) {
-                tmem_st_wait();
-                arrive_e();     // W_0 in TMEM, k2 lines in the B buffer: the first P1 may start
-                // the rows of k2 go to global memory for the later P1s (TMA store of the staging),
-                // issued only now: a cluster-scope release waits for the issuing thread's
-                // outstanding bulk copies, and the first P1's release must not wait for this one
-                if (et == 0) {
-                    for (int a = 0; a < 8; ++a) tma_store_3d(&maps.k2, bbuf + a * C::kAtomBytes, 32 * a, r0, bh);
-                    tma_store_commit();
-                }
-                // k2^T (the first P4's right factor, streamed back by TMA): this thread's row of
-                // k2 from the staged B lines into column `row` of k2^T. Written only now, so that
-                // the cluster-scope release above does not wait for these global stores.
-                float* k2t_col = prm.k2t + (size_t)bh * M * M + row;
-#pragma unroll 1
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int a = 4 * h + jj;
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) {
-                        const float4 f4 = *reinterpret_cast<const float4*>(bbuf + stage_off(a, c));
-                        k2t_col[(size_t)(32 * a + 4 * c) * M] = f4.x;
-                        k2t_col[(size_t)(32 * a + 4 * c + 1) * M] = f4.y;
-                        k2t_col[(size_t)(32 * a + 4 * c + 2) * M] = f4.z;
-                        k2t_col[(size_t)(32 * a + 4 * c + 3) * M] = f4.w;
-                    }
-                }
-                // the TMA store of k2's rows only reads the B buffer, as the first P1 does; it is
-                // complete before the producer reads k2 back (wl_ready) and before the P1
-                // epilogue, behind the next named barrier, overwrites the B buffer
-                if (et == 0) tma_store_wait_all<0>();
-                arrive_wl();    // k2 and k2^T in global memory
             }
         }
 
@@ -673,9 +699,18 @@ pinv_pair_kernel(const __grid_constant__ PinvPairMaps maps, const PinvPairParams
                     tmem_st_wait();
                     fence_proxy_async_cluster();   // X lines (here and in the peer) feed the MMA
                     arrive_e();
+                    if (it == 0) {
+                        // k2's rows, the first P4's right factor (by rows, MN-major), are in global
+                        // memory: the producer may stream them once P3 frees the B buffer
+                        if (et == 0) tma_store_wait_all<0>();
+                        arrive_wl();
+                    }
                 }
             }
         }
+        // k2's bulk copy (waited for above unless a wait ran out) has completed before the shared
+        // memory is released
+        if (et == 0) tma_store_wait_all<0>();
     }
 
     tc_fence_before();
