@@ -266,7 +266,12 @@ class ClockSampler:
             return
         self.t = threading.Thread(target=self._read, daemon=True)
         self.t.start()
-        time.sleep(0.3)
+        # nvidia-smi can take a second or more to start on a fresh machine: the timed steps begin
+        # only once it prints, so that its samples cover them
+        t0 = time.time()
+        while not self.lines and self.proc.poll() is None and time.time() - t0 < 5.0:
+            time.sleep(0.02)
+        time.sleep(0.05)
 
     def _read(self):
         for line in self.proc.stdout:
