@@ -253,6 +253,7 @@ class ClockSampler:
         self.gpu_id = gpu_id
         self.proc = None
         self.lines = []
+        self.times = []
 
     def start(self):
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
@@ -276,8 +277,11 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
+            self.times.append(time.time())
 
-    def stop(self):
+    def stop(self, window=None):
+        """Summary of the samples; with window = (t0, t1) (host seconds) only those printed
+        during it (plus one polling interval), unless there are none."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         time.sleep(0.1)
@@ -289,7 +293,12 @@ class ClockSampler:
         self.t.join(timeout=2)
         sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lines, scope = self.lines, "sampler lifetime"
+        if window is not None:
+            inside = [ln for ln, t in zip(self.lines, self.times) if window[0] <= t <= window[1] + 0.025]
+            if inside:
+                lines, scope = inside, "timed steps"
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -305,7 +314,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "samples": len(sm),
-                "power_w_max": max(power), "reasons": sorted(reasons)}
+                "samples_from": scope, "power_w_max": max(power), "reasons": sorted(reasons)}
 
 
 # ---------------------------------------------------------------- CPU oracle timing
@@ -521,6 +530,7 @@ def main():
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    t_timed0 = time.time()
     nys.profile_mask([dom])
     prof_steps = max(1, args.steps // 10)
     for i in range(args.steps):
@@ -532,9 +542,10 @@ def main():
         step()
         ends[i].record(stream)
     torch.cuda.synchronize()
+    t_timed1 = time.time()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
+    clocks = sampler.stop((t_timed0, t_timed1))
     prof = nys.profile_read()
     nys.profile_enable(False)
     nys.profile_mask(None)

@@ -102,3 +102,21 @@ def test_exact_branch_bound_counts_n_squared_work():
     assert bench.step_exponentials(w, "exact") == w.BH * w.n * w.n
     nb, fl, unit = bench.kernel_work(w, "k3v_partial", "exact")
     assert fl == w.BH * 4 * w.n * w.n * w.d and unit == "tensor"
+
+
+def test_clock_samples_are_taken_from_the_timed_window():
+    """Only the nvidia-smi lines printed during the timed steps count (plus one polling
+    interval); throttle reasons are read from the same lines; with none inside the window the
+    sampler falls back to every line."""
+    s = bench.ClockSampler(None)
+    s.proc = type("P", (), {"terminate": lambda self: None, "wait": lambda self, timeout=None: 0})()
+    s.t = type("T", (), {"join": lambda self, timeout=None: None})()
+    idle = "0, 1200, 1965, 150.0, 0x0, Not Active, Not Active, Not Active, Not Active"
+    busy = "0, 1965, 1965, 700.0, 0x4, Not Active, Not Active, Not Active, Active"
+    s.lines = [idle, busy, busy, busy, idle]
+    s.times = [10.0, 10.50, 10.52, 10.54, 11.0]
+    c = s.stop((10.49, 10.55))
+    assert c["sm_mhz"] == 1965 and c["samples"] == 3 and c["samples_from"] == "timed steps"
+    assert c["reasons"] == ["sw_power_cap"] and c["power_w_max"] == 700.0
+    c = s.stop((20.0, 20.1))
+    assert c["samples"] == 5 and c["samples_from"] == "sampler lifetime" and c["sm_mhz"] == 1965
